@@ -1,0 +1,236 @@
+"""Python wrapper of the fp64 CPU oracle (ctypes over liboracle.so).
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, the smoke check in __graft_entry__.py
+and bench.py's CPU-baseline / reference leg import this package; the product
+(the CUDA library and its binding) never does, and this package never imports
+the product.  Inputs come from numpy arrays: bf16 tensors as uint16 bit
+patterns, everything else as int32 / float32 / float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_override = None
+
+
+class use_library:
+    """Context manager: route every call of this wrapper to another build of
+    the oracle (the pin tests use it to run mutated copies)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _override
+        self._saved = _override
+        _override = _bind(ctypes.CDLL(self.path))
+        return self
+
+    def __exit__(self, *exc):
+        global _override
+        _override = self._saved
+        return False
+
+
+def lib():
+    global _lib
+    if _override is not None:
+        return _override
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def _bind(L):
+    P = ctypes.c_void_p
+    i32, f64 = ctypes.c_int, ctypes.c_double
+    L.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+    L.oracle_bf16_to_f64.restype = f64
+    L.oracle_f64_to_bf16.argtypes = [f64]
+    L.oracle_f64_to_bf16.restype = ctypes.c_uint16
+    L.oracle_round_bf16.argtypes = [P, P, ctypes.c_size_t]
+    L.oracle_round_bf16.restype = None
+    L.oracle_sigmoid.argtypes = [f64]
+    L.oracle_sigmoid.restype = f64
+    L.oracle_silu.argtypes = [f64]
+    L.oracle_silu.restype = f64
+    L.oracle_route.argtypes = [P, P, P, i32, i32, i32, i32, f64, P, P, P, P, i32]
+    L.oracle_route.restype = i32
+    L.oracle_permute.argtypes = [P, i32, i32, i32, P, P, P, P]
+    L.oracle_permute.restype = i32
+    L.oracle_swiglu_row.argtypes = [P, P, P, i32, i32, P, P]
+    L.oracle_swiglu_row.restype = None
+    L.oracle_combine.argtypes = [P, P, P, P, i32, i32, i32, P]
+    L.oracle_combine.restype = None
+    L.oracle_moe_rows.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32, P,
+                                  i32]
+    L.oracle_moe_rows.restype = i32
+    return L
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    """bf16 data as a C-contiguous uint16 numpy array (accepts torch or numpy)."""
+    if hasattr(a, "view") and hasattr(a, "dtype") and str(a.dtype) == "torch.bfloat16":
+        import torch
+        return np.ascontiguousarray(a.detach().cpu().contiguous().view(torch.int16).numpy()
+                                    .view(np.uint16))
+    arr = np.ascontiguousarray(a)
+    assert arr.dtype == np.uint16, arr.dtype
+    return arr
+
+
+def _np(a, dtype):
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def bf16_to_f64(a) -> np.ndarray:
+    u = _u16(a)
+    with np.errstate(invalid="ignore"):
+        return (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().oracle_round_bf16(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def sigmoid(z: float) -> float:
+    return lib().oracle_sigmoid(float(z))
+
+
+def silu(z: float) -> float:
+    return lib().oracle_silu(float(z))
+
+
+def route(x, w_router, bias, k: int, scale: float, nthreads: int | None = None,
+          want_scores: bool = False):
+    """Steps 1-4: returns (topk_idx int32 [T,k], topk_w f64 [T,k], gap f64 [T][, scores])."""
+    xu, wu = _u16(x), _u16(w_router)
+    b = _np(bias, np.float32)
+    T, d = xu.shape
+    E = wu.shape[0]
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    gap = np.empty((T,), np.float64)
+    scores = np.empty((T, E), np.float64) if want_scores else None
+    rc = lib().oracle_route(_ptr(xu), _ptr(wu), _ptr(b), T, d, E, k, float(scale),
+                            _ptr(idx), _ptr(w), _ptr(scores), _ptr(gap),
+                            nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_route: invalid arguments")
+    return (idx, w, gap, scores) if want_scores else (idx, w, gap)
+
+
+def permute(topk_idx, E: int):
+    """Expert-contiguous permutation: (counts, offsets, row_token, slot_row)."""
+    idx = _np(topk_idx, np.int32)
+    T, k = idx.shape
+    counts = np.empty((E,), np.int32)
+    offsets = np.empty((E + 1,), np.int32)
+    row_token = np.empty((T * k,), np.int32)
+    slot_row = np.empty((T * k,), np.int32)
+    rc = lib().oracle_permute(_ptr(idx), T, E, k, _ptr(counts), _ptr(offsets),
+                              _ptr(row_token), _ptr(slot_row))
+    if rc != 0:
+        raise ValueError("oracle_permute: invalid routing indices")
+    return counts, offsets, row_token, slot_row
+
+
+def swiglu_row(xrow, w_gate_up, w_down, want_act: bool = False):
+    xu, gu, dn = _u16(xrow), _u16(w_gate_up), _u16(w_down)
+    d = xu.shape[-1]
+    inter = gu.shape[0] // 2
+    y = np.empty((d,), np.float64)
+    act = np.empty((inter,), np.float64)
+    lib().oracle_swiglu_row(_ptr(xu), _ptr(gu), _ptr(dn), d, inter, _ptr(y), _ptr(act))
+    return (y, act) if want_act else y
+
+
+def combine(y, y_shared, topk_w, slot_row):
+    y = _np(y, np.float64)
+    ys = None if y_shared is None else _np(y_shared, np.float64)
+    w = _np(topk_w, np.float64)
+    sr = _np(slot_row, np.int32)
+    T, k = w.shape
+    d = y.shape[1]
+    out = np.empty((T, d), np.float64)
+    lib().oracle_combine(_ptr(y), _ptr(ys), _ptr(w), _ptr(sr), T, d, k, _ptr(out))
+    return out
+
+
+def moe_rows(x, topk_idx, topk_w, expert_gate_up, expert_down, shared_gate_up, shared_down,
+             tokens=None, nthreads: int | None = None):
+    """Steps 5-7 on the listed tokens (all tokens if None).
+
+    expert_gate_up / expert_down: sequences indexed by expert (uint16 arrays or
+    bf16 tensors, or None for experts no listed token selects)."""
+    xu = _u16(x)
+    T, d = xu.shape
+    idx = _np(topk_idx, np.int32)
+    w = _np(topk_w, np.float64)
+    k = idx.shape[1]
+    E = len(expert_gate_up)
+    keep = []
+    gu_ptrs = (ctypes.c_void_p * E)()
+    dn_ptrs = (ctypes.c_void_p * E)()
+    inter = None
+    for e in range(E):
+        if expert_gate_up[e] is None:
+            continue
+        g, dn = _u16(expert_gate_up[e]), _u16(expert_down[e])
+        keep += [g, dn]
+        inter = g.shape[0] // 2
+        gu_ptrs[e] = g.ctypes.data
+        dn_ptrs[e] = dn.ctypes.data
+    sgu, sdn = _u16(shared_gate_up), _u16(shared_down)
+    inter = sgu.shape[0] // 2
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tok is None else tok.shape[0]
+    out = np.empty((n, d), np.float64)
+    rc = lib().oracle_moe_rows(_ptr(xu), T, d, E, k, inter, _ptr(idx), _ptr(w),
+                               ctypes.cast(gu_ptrs, ctypes.c_void_p),
+                               ctypes.cast(dn_ptrs, ctypes.c_void_p),
+                               _ptr(sgu), _ptr(sdn), _ptr(tok), n, _ptr(out),
+                               nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_moe_rows: a selected expert's weights are missing")
+    del keep
+    return out
+
+
+def moe_forward(inputs: dict, k: int, scale: float, tokens=None, nthreads: int | None = None):
+    """Whole layer: route all tokens, then evaluate the listed rows.
+
+    inputs: dict from moe_inputs.make_inputs (CPU tensors).  Returns
+    (out f64 [n,d], topk_idx, topk_w, gap)."""
+    idx, w, gap = route(inputs["x"], inputs["w_router"], inputs["bias"], k, scale, nthreads)
+    E = inputs["w_router"].shape[0]
+    gu = inputs["w_gate_up"]
+    dn = inputs["w_down"]
+    need = set(np.unique(idx if tokens is None else idx[np.asarray(tokens)]).tolist())
+    egu = [gu[e] if e in need else None for e in range(E)]
+    edn = [dn[e] if e in need else None for e in range(E)]
+    out = moe_rows(inputs["x"], idx, w, egu, edn, inputs["ws_gate_up"], inputs["ws_down"],
+                   tokens=tokens, nthreads=nthreads)
+    return out, idx, w, gap

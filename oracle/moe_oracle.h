@@ -1,0 +1,113 @@
+/*
+ * moe_oracle.h -- plain, slow, fp64 CPU oracle for one Kimi-K2-style MoE FFN
+ * layer (forward pass).  TEST INFRASTRUCTURE ONLY: only the tests, the smoke
+ * check and the benchmark's CPU-baseline leg may load this library.  The
+ * product path (the CUDA library) never calls it and shares no code with it.
+ *
+ * What it computes, step by step, as the pages give it:
+ *   "Kimi K2.5 deep dive", CH4.2 (routing) and CH10.2 (MoE 7-step dataflow):
+ *     1. s = sigmoid(x . W_router^T)                       (scoring_func=sigmoid)
+ *     2. b = s + e_score_correction_bias                   (selection-only bias)
+ *     3. top-k of b over all E experts (n_group = 1, "K2 inference" answer, 2.4)
+ *     4. weights = s_sel / sum(s_sel), then * routed_scaling_factor
+ *     5. shared expert on every token, unscaled
+ *     6. routed experts: SwiGLU y = W_down (silu(W_gate x) * (W_up x))
+ *     7. out = shared + sum_j w_j * y_j
+ *   "Kimi K2.5 Q&A" Q8.3 gives the same order (router -> shared || routed -> add).
+ *
+ * Readings where the pages are silent or disagree (each listed in the design doc):
+ *   - step 4 uses the UNBIASED sigmoid scores (the bias only picks experts);
+ *   - ties in step 3 go to the lower expert index; slot j = j-th largest b;
+ *   - no epsilon in the renormalisation (a sum of k sigmoids is > 0);
+ *   - every token gets exactly k experts (no capacity, no dropping);
+ *   - within an expert, rows are in ascending token order (the per-expert mask
+ *     of the pages' dispatch loop visits tokens in order).
+ *
+ * Precision: bf16 inputs are widened exactly to double; all arithmetic is fp64;
+ * results are returned in fp64.  bf16 values travel as their uint16 bit pattern.
+ *
+ * Parity pins (what checks this oracle against something other than itself)
+ * live in tests/test_oracle_pins.py.
+ */
+#ifndef MOE_ORACLE_H
+#define MOE_ORACLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bf16 bit pattern -> double (exact). */
+double oracle_bf16_to_f64(uint16_t v);
+/* double -> bf16 bit pattern, one rounding, to nearest, ties to even. */
+uint16_t oracle_f64_to_bf16(double v);
+/* bulk version of the rounding above */
+void oracle_round_bf16(const double* in, uint16_t* out, size_t n);
+
+double oracle_sigmoid(double z);           /* 1 / (1 + exp(-z)) */
+double oracle_silu(double z);              /* z * sigmoid(z) */
+
+/*
+ * Router (steps 1-4) for T tokens.
+ *   x [T,d] bf16, w_router [E,d] bf16 (Linear out x in), bias [E] fp32.
+ *   topk_idx [T,k] int32  (slot j = j-th largest biased score, ties -> lower e)
+ *   topk_w   [T,k] double (scale * s_sel / sum s_sel, unbiased s)
+ *   scores   [T,E] double sigmoid scores, optional (NULL)
+ *   gap      [T]   double b_(k) - b_(k+1) (biased, sorted), +inf if k == E; optional
+ * Returns 0, or -1 on invalid arguments.
+ */
+int oracle_route(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                 int T, int d, int E, int k, double scale,
+                 int32_t* topk_idx, double* topk_w, double* scores, double* gap,
+                 int nthreads);
+
+/*
+ * Permutation of the (token, slot) pairs into expert-contiguous rows.
+ *   counts[e]   = #{(t,j): idx[t,j] == e}
+ *   offsets     = exclusive prefix sum of counts, offsets[E] = T*k
+ *   rows of expert e are offsets[e] .. offsets[e+1]-1, in ascending token order
+ *   row_token[row] = t,  slot_row[t*k + j] = row
+ * Returns 0, or -1 if an index is out of range or a token repeats an expert.
+ */
+int oracle_permute(const int32_t* topk_idx, int T, int E, int k,
+                   int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* slot_row);
+
+/*
+ * One SwiGLU expert on one token row:
+ *   y[d] = W_down (silu(W_gate x) * (W_up x)),  w_gate_up [2I,d] (gate rows then
+ *   up rows), w_down [d,I].  act (optional) receives the I-vector
+ *   silu(W_gate x) * (W_up x).
+ */
+void oracle_swiglu_row(const uint16_t* xrow, const uint16_t* w_gate_up, const uint16_t* w_down,
+                       int d, int inter, double* y, double* act);
+
+/*
+ * Combine (step 7) given expert outputs in permuted row order:
+ *   out[t] = y_shared[t] + sum_j topk_w[t,j] * y[slot_row[t*k+j]]
+ * y [T*k, d], y_shared [T, d] (or NULL), all double.
+ */
+void oracle_combine(const double* y, const double* y_shared, const double* topk_w,
+                    const int32_t* slot_row, int T, int d, int k, double* out);
+
+/*
+ * Whole layer on a subset of tokens (rows are independent, so any subset gives
+ * the same rows as the full batch).
+ *   expert_gate_up[e] -> [2I,d] bf16 of routed expert e, expert_down[e] -> [d,I];
+ *   pointers of experts no listed token selects may be NULL.
+ *   tokens [n_tokens] : which rows of x to evaluate (NULL = all T, n_tokens = T)
+ *   topk_idx/topk_w   : routing of ALL T tokens (from oracle_route)
+ *   out [n_tokens, d] double
+ * Returns 0, or -1 if a needed expert pointer is NULL.
+ */
+int oracle_moe_rows(const uint16_t* x, int T, int d, int E, int k, int inter,
+                    const int32_t* topk_idx, const double* topk_w,
+                    const uint16_t* const* expert_gate_up, const uint16_t* const* expert_down,
+                    const uint16_t* shared_gate_up, const uint16_t* shared_down,
+                    const int32_t* tokens, int n_tokens, double* out, int nthreads);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_ORACLE_H */

@@ -1,0 +1,328 @@
+"""Checks that pin the fp64 oracle to something other than itself.
+
+Each pin_* function raises AssertionError if the oracle (whichever build the
+`oracle` wrapper currently points at) breaks a fact fixed by the pages or by
+mathematics:
+  - closed forms and identities (sigmoid(0) = 1/2, sigma(z) + sigma(-z) = 1,
+    silu(z) - silu(-z) = z, weights summing to the scaling factor);
+  - special cases that reduce to a library routine (numpy matmul + scipy expit
+    for the router scores, torch's float->bf16 rounding);
+  - brute force on tiny inputs (full sort for top-k, lexsort for the
+    permutation, naive Python loops for a textbook SwiGLU MLP);
+  - a dense all-experts-then-mask evaluation (the MoE definition) against the
+    oracle's sparse path;
+  - invariants (bias changes selection but never weights; rows independent).
+tests/test_oracle_pins.py runs them on the oracle; tests/test_oracle_mutants.py
+runs them on deliberately broken copies of the oracle and requires each copy
+to fail at least one pin.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+from scipy.special import expit
+
+import oracle
+from moe_inputs import MoEConfig, make_inputs, make_topk_idx
+
+K2_SCALE = 2.827   # routed_scaling_factor of K2 (K2 team member's answer, "different")
+
+
+def _bf16(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _f64(t):
+    return oracle.bf16_to_f64(t)
+
+
+# ------------------------------------------------------------------ numbers
+
+def pin_bf16_rounding():
+    pats = np.arange(65536, dtype=np.uint16)
+    vals = oracle.bf16_to_f64(pats)
+    finite = np.isfinite(vals)
+    back = oracle.f64_to_bf16(vals[finite])
+    # every finite bf16 value is its own rounding (up to the sign of zero)
+    same = (back == pats[finite]) | ((vals[finite] == 0) & ((back & 0x7FFF) == 0))
+    assert same.all(), "bf16 values do not round-trip"
+    # midpoints between neighbours round to the even significand
+    rng = np.random.default_rng(1)
+    a = rng.integers(0x0080, 0x7F00, size=2000).astype(np.uint16)
+    lo, hi = oracle.bf16_to_f64(a), oracle.bf16_to_f64(a + 1)
+    mid = (lo + hi) / 2.0
+    got = oracle.f64_to_bf16(mid)
+    want = np.where(a % 2 == 0, a, a + 1).astype(np.uint16)
+    assert (got == want).all(), "ties do not go to even"
+    # slightly off the midpoint goes to the nearer neighbour
+    assert (oracle.f64_to_bf16(mid - (hi - lo) * 1e-3) == a).all()
+    assert (oracle.f64_to_bf16(mid + (hi - lo) * 1e-3) == a + 1).all()
+    # agrees with torch's fp32 -> bf16 rounding on values that are exact fp32
+    f = rng.standard_normal(5000).astype(np.float32) * np.float32(37.0)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (oracle.f64_to_bf16(f.astype(np.float64)) == ref).all()
+
+
+def pin_sigmoid_silu():
+    assert oracle.sigmoid(0.0) == 0.5
+    assert abs(oracle.sigmoid(math.log(3.0)) - 0.75) < 1e-15
+    for z in np.linspace(-30, 30, 61):
+        s, sn = oracle.sigmoid(z), oracle.sigmoid(-z)
+        assert abs(s + sn - 1.0) < 1e-15
+        assert abs(s - expit(z)) < 1e-15
+        assert abs(oracle.silu(z) - z * expit(z)) <= 1e-14 * max(1.0, abs(z))
+        assert abs(oracle.silu(z) - oracle.silu(-z) - z) <= 1e-14 * max(1.0, abs(z))
+    assert oracle.silu(0.0) == 0.0
+
+
+# ------------------------------------------------------------------- router
+
+def _rand_router(T, d, E, seed, bias_scale=0.01):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    w = (torch.randn((E, d), generator=g) / math.sqrt(d)).to(torch.bfloat16)
+    b = ((torch.rand((E,), generator=g) * 2 - 1) * bias_scale).to(torch.float32)
+    return x, w, b
+
+
+def pin_route_worked_example():
+    """Hand-built: x = e_0, router column 0 carries the logits."""
+    d, E, k = 8, 5, 2
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    L = np.array([0.0, 2.0, -2.0, 0.0, 1.0], np.float32)   # all exact in bf16
+    w_r = np.zeros((E, d), np.float32)
+    w_r[:, 0] = L
+    # biased scores: [0.5, s(2), s(-2)+0.9, 0.5-0.1, s(1)-0.5] ->
+    # order: e2 (1.019) > e1 (0.881) > e0 (0.5) > e3 (0.4) > e4 (0.231)
+    bias = np.array([0.0, 0.0, 0.9, -0.1, -0.5], np.float32)
+    idx, w, gap = oracle.route(_bf16(x), _bf16(w_r), bias, k, K2_SCALE)
+    assert idx.tolist() == [[2, 1]], idx
+    # unbiased: s(-2) + s(2) = 1 exactly in exact arithmetic
+    s2 = 1.0 / (1.0 + math.exp(-2.0))
+    assert abs(w[0, 0] - K2_SCALE * (1.0 - s2)) < 1e-14
+    assert abs(w[0, 1] - K2_SCALE * s2) < 1e-14
+    assert abs(gap[0] - (s2 - 0.5)) < 1e-7    # b_(2) - b_(3), bias is fp32 0.0
+    # E = k: every expert, weights from all unbiased scores
+    idx, w, gap = oracle.route(_bf16(x), _bf16(w_r), bias, E, K2_SCALE)
+    assert idx.tolist() == [[2, 1, 0, 3, 4]]
+    s = expit(L.astype(np.float64))
+    assert np.allclose(w[0], K2_SCALE * s[[2, 1, 0, 3, 4]] / s.sum(), rtol=0, atol=1e-14)
+    assert gap[0] == np.inf
+
+
+def pin_router_scores_library():
+    x, w, b = _rand_router(40, 64, 19, seed=3)
+    idx, tw, gap, scores = oracle.route(x, w, b, 4, K2_SCALE, want_scores=True)
+    ref = expit(_f64(x) @ _f64(w).T)
+    assert np.abs(scores - ref).max() < 1e-13, "router scores differ from expit(x W^T)"
+
+
+def pin_topk_brute_force():
+    for (T, d, E, k, seed) in [(50, 32, 5, 1, 0), (50, 32, 9, 3, 1), (60, 64, 33, 8, 2),
+                               (20, 16, 7, 7, 4), (30, 32, 40, 32, 5)]:
+        x, w, b = _rand_router(T, d, E, seed, bias_scale=0.2)
+        idx, tw, gap, scores = oracle.route(x, w, b, k, K2_SCALE, want_scores=True)
+        bb = scores + b.numpy().astype(np.float64)[None, :]
+        for t in range(T):
+            order = sorted(range(E), key=lambda e: (-bb[t, e], e))
+            assert idx[t].tolist() == order[:k], (t, idx[t], order[:k])
+            want_gap = bb[t, order[k - 1]] - bb[t, order[k]] if k < E else np.inf
+            assert gap[t] == want_gap
+            assert len(set(idx[t].tolist())) == k
+
+
+def pin_exact_ties():
+    d, E, k = 16, 6, 3
+    g = torch.Generator().manual_seed(7)
+    row = torch.randn((1, d), generator=g)
+    w = row.repeat(E, 1).to(torch.bfloat16)         # six identical router rows
+    x = torch.randn((5, d), generator=g).to(torch.bfloat16)
+    idx, tw, gap = oracle.route(x, w, np.zeros(E, np.float32), k, K2_SCALE)
+    assert (idx == np.array([0, 1, 2])[None, :]).all(), idx   # ties -> lower index
+    assert np.allclose(tw, K2_SCALE / k, rtol=0, atol=1e-15)
+    assert (gap == 0).all()
+    # a strictly larger bias on expert 4 lifts it to slot 0, the rest keep index order
+    bias = np.zeros(E, np.float32)
+    bias[4] = 1e-3
+    idx, tw, gap = oracle.route(x, w, bias, k, K2_SCALE)
+    assert (idx == np.array([4, 0, 1])[None, :]).all(), idx
+    assert np.allclose(tw, K2_SCALE / k, rtol=0, atol=1e-15)
+
+
+def pin_weights_closed_form():
+    x, w, b = _rand_router(64, 64, 24, seed=9)
+    k = 6
+    idx, tw, gap = oracle.route(x, w, b, k, K2_SCALE)
+    s = expit(_f64(x) @ _f64(w).T)
+    sel = np.take_along_axis(s, idx.astype(np.int64), axis=1)
+    assert np.abs(tw.sum(1) - K2_SCALE).max() <= 1e-12 * K2_SCALE
+    assert (tw > 0).all()
+    assert np.abs(tw - K2_SCALE * sel / sel.sum(1, keepdims=True)).max() < 1e-12
+    # the DeepSeek-V3 factor works the same way
+    _, tw25, _ = oracle.route(x, w, b, k, 2.5)
+    assert np.abs(tw25.sum(1) - 2.5).max() <= 1e-12 * 2.5
+
+
+def pin_bias_selection_only():
+    x, w, b = _rand_router(80, 64, 16, seed=11, bias_scale=0.05)
+    k = 4
+    idx0, tw0, _ = oracle.route(x, w, np.zeros(16, np.float32), k, K2_SCALE)
+    idx1, tw1, _ = oracle.route(x, w, b, k, K2_SCALE)
+    changed = 0
+    for t in range(80):
+        m0 = dict(zip(idx0[t].tolist(), tw0[t].tolist()))
+        m1 = dict(zip(idx1[t].tolist(), tw1[t].tolist()))
+        if set(m0) == set(m1):
+            assert m0 == m1, "bias changed a weight of an unchanged selection"
+        else:
+            changed += 1
+    assert changed > 0, "bias never changed a selection (test is too weak)"
+    # a large bias forces expert 5 in; its weight still comes from unbiased scores
+    big = np.zeros(16, np.float32)
+    big[5] = 10.0
+    idx2, tw2, _ = oracle.route(x, w, big, k, K2_SCALE)
+    assert (idx2[:, 0] == 5).all()
+    s = expit(_f64(x) @ _f64(w).T)
+    sel = np.take_along_axis(s, idx2.astype(np.int64), axis=1)
+    assert np.abs(tw2[:, 0] - K2_SCALE * s[:, 5] / sel.sum(1)).max() < 1e-12
+
+
+# ------------------------------------------------------------- permutation
+
+def pin_permute_brute_force():
+    cases = [(37, 11, 3, 0, 0.0), (64, 32, 4, 1, 0.0), (200, 384, 8, 2, 0.0),
+             (128, 16, 8, 3, 3.0), (1, 5, 5, 4, 0.0), (50, 9, 1, 5, 1.0)]
+    for T, E, k, seed, skew in cases:
+        idx = make_topk_idx(T, E, k, seed=seed, skew=skew).numpy()
+        counts, offsets, row_token, slot_row = oracle.permute(idx, E)
+        flat_e = idx.reshape(-1).astype(np.int64)
+        flat_t = np.repeat(np.arange(T), k)
+        order = np.lexsort((flat_t, flat_e))          # by expert, then token
+        assert (counts == np.bincount(flat_e, minlength=E)).all()
+        assert counts.sum() == T * k
+        assert offsets[0] == 0 and (np.diff(offsets) == counts).all()
+        assert (row_token == flat_t[order]).all()
+        want_slot = np.empty(T * k, np.int64)
+        want_slot[order] = np.arange(T * k)
+        assert (slot_row == want_slot).all()
+        assert sorted(slot_row.tolist()) == list(range(T * k))
+        assert (row_token[slot_row] == flat_t).all()
+        for e in range(E):
+            seg = row_token[offsets[e]:offsets[e + 1]]
+            assert (np.diff(seg) > 0).all()
+
+
+# ------------------------------------------------------------------ experts
+
+def pin_swiglu_textbook():
+    """Naive loops: h_n = silu(sum_i G[n,i] x_i) * (sum_i U[n,i] x_i); y_o = sum_n D[o,n] h_n."""
+    d, I = 12, 5
+    g = torch.Generator().manual_seed(13)
+    x = torch.randn((d,), generator=g).to(torch.bfloat16)
+    gu = torch.randn((2 * I, d), generator=g).to(torch.bfloat16)
+    dn = torch.randn((d, I), generator=g).to(torch.bfloat16)
+    xf, guf, dnf = _f64(x), _f64(gu), _f64(dn)
+    h = []
+    for n in range(I):
+        gate = sum(guf[n, i] * xf[i] for i in range(d))
+        up = sum(guf[I + n, i] * xf[i] for i in range(d))
+        h.append(gate * expit(gate) * up)
+    y = [sum(dnf[o, n] * h[n] for n in range(I)) for o in range(d)]
+    got, act = oracle.swiglu_row(x, gu, dn, want_act=True)
+    assert np.abs(np.array(h) - act).max() < 1e-12
+    assert np.abs(np.array(y) - got).max() < 1e-12
+
+
+def _tiny_cfg():
+    return MoEConfig("pin", T=24, d=64, E=10, k=3, inter=32, scale=K2_SCALE)
+
+
+def pin_dense_vs_sparse():
+    """MoE by definition: every expert on every token, masked by the routing weights."""
+    cfg = _tiny_cfg()
+    inp = make_inputs(cfg, seed=21)
+    out, idx, tw, gap = oracle.moe_forward(inp, cfg.k, cfg.scale)
+    xf = _f64(inp["x"])
+    gu, dn = _f64(inp["w_gate_up"]), _f64(inp["w_down"])
+    I = cfg.inter
+
+    def ffn(gu_e, dn_e):
+        G, U = xf @ gu_e[:I].T, xf @ gu_e[I:].T
+        return (G * expit(G) * U) @ dn_e.T
+
+    mask = np.zeros((cfg.T, cfg.E))
+    np.put_along_axis(mask, idx.astype(np.int64), tw, axis=1)
+    dense = ffn(_f64(inp["ws_gate_up"]), _f64(inp["ws_down"]))
+    for e in range(cfg.E):
+        dense += mask[:, e:e + 1] * ffn(gu[e], dn[e])
+    assert np.abs(dense - out).max() <= 1e-12 * np.abs(dense).max()
+
+
+def pin_special_cases():
+    cfg = _tiny_cfg()
+    inp = make_inputs(cfg, seed=22)
+    I = cfg.inter
+    xf = _f64(inp["x"])
+    sg, sd = _f64(inp["ws_gate_up"]), _f64(inp["ws_down"])
+    G = xf @ sg[:I].T
+    shared_only = (G * expit(G) * (xf @ sg[I:].T)) @ sd.T
+    # routed gate_proj = 0  =>  silu(0) = 0  =>  output is the shared expert alone
+    z = dict(inp)
+    z["w_gate_up"] = inp["w_gate_up"].clone()
+    z["w_gate_up"][:, :I] = 0
+    out, *_ = oracle.moe_forward(z, cfg.k, cfg.scale)
+    assert np.abs(out - shared_only).max() <= 1e-12 * np.abs(shared_only).max()
+    # the shared expert is always there: zeroing its down_proj leaves only routed rows
+    z2 = dict(inp)
+    z2["ws_down"] = torch.zeros_like(inp["ws_down"])
+    out2, idx, tw, _ = oracle.moe_forward(z2, cfg.k, cfg.scale)
+    full, *_ = oracle.moe_forward(inp, cfg.k, cfg.scale)
+    assert np.abs((full - out2) - shared_only).max() <= 1e-11 * np.abs(shared_only).max()
+
+
+def pin_row_independence():
+    cfg = _tiny_cfg()
+    inp = make_inputs(cfg, seed=23)
+    full, idx, tw, _ = oracle.moe_forward(inp, cfg.k, cfg.scale)
+    sub = np.array([5, 0, 23, 11, 11], np.int32)
+    part, *_ = oracle.moe_forward(inp, cfg.k, cfg.scale, tokens=sub)
+    assert np.array_equal(part, full[sub])
+
+
+def pin_combine():
+    T, d, k = 9, 16, 3
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((T * k, d))
+    ys = rng.standard_normal((T, d))
+    w = rng.random((T, k))
+    slot_row = rng.permutation(T * k).astype(np.int32)
+    out = oracle.combine(y, ys, w, slot_row)
+    for t in range(T):
+        want = ys[t] + sum(w[t, j] * y[slot_row[t * k + j]] for j in range(k))
+        assert np.abs(out[t] - want).max() < 1e-13
+    # one-hot weights pick the row the slot points at
+    w1 = np.zeros((T, k))
+    w1[:, 1] = 1.0
+    out1 = oracle.combine(y, None, w1, slot_row)
+    assert np.array_equal(out1, y[slot_row.reshape(T, k)[:, 1]])
+
+
+ALL_PINS = [pin_bf16_rounding, pin_sigmoid_silu, pin_route_worked_example,
+            pin_router_scores_library, pin_topk_brute_force, pin_exact_ties,
+            pin_weights_closed_form, pin_bias_selection_only, pin_permute_brute_force,
+            pin_swiglu_textbook, pin_dense_vs_sparse, pin_special_cases,
+            pin_row_independence, pin_combine]
+
+
+def failing_pins():
+    """Names of the pins the current oracle build fails (exceptions count as failures)."""
+    bad = []
+    for p in ALL_PINS:
+        try:
+            p()
+        except Exception:  # noqa: BLE001 - any error is a caught mistake
+            bad.append(p.__name__)
+    return bad
