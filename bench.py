@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Throughput of one K2-style MoE FFN layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload k2_decode|k2_prefill|k2_skew|v3|tiny]
+
+One step = one full layer forward (route, permute, grouped SwiGLU experts with
+the shared expert, combine) over one batch of T synthetic tokens, inputs and
+weights resident in HBM.  Prints ONE JSON line on rank 0.
+
+  ours       the CUDA library through its C ABI (moe_layer_forward)
+  reference  the fp64 CPU oracle on the host cores, on a bounded token sample
+             of the same workload (rows are independent, so tokens/s of a
+             sample is the oracle's rate on the workload)
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica on
+its own batch (weak scaling; the layer has no exchange step on one GPU per
+replica); the time is the max over ranks and value counts all ranks' tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "K2 MoE-layer tokens/s; % of HBM (decode) / bf16 tensor (prefill) roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_STEPS = {"k2_decode": 400, "tiny": 400, "v3": 100, "k2_skew": 100, "k2_prefill": 60}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="k2_decode")
+    p.add_argument("--cpu-sample", type=int, default=None,
+                   help="tokens in the oracle's timed sample (default: sized from the core count)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    a = p.parse_args(argv)
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS.get(a.workload, 100)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        return time.time()
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self, t0, t1):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = ["sparse_moe_ffn_sigmoid_b200/csrc/gemm.cuh", "sparse_moe_ffn_sigmoid_b200/csrc/ptx.cuh",
+                  "sparse_moe_ffn_sigmoid_b200/csrc/common.cuh"]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel sources are unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest(KERNEL_SOURCES)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and parts[0] == workload and parts[1] == kernel and \
+                    parts[3] == digest:
+                return float(parts[2])
+    return None
+
+
+# ----------------------------------------------------- accounting (per step)
+
+def layer_accounting(cfg, touched: int):
+    """Algorithmic bytes and FLOPs of one layer forward, and of its two GEMMs.
+
+    touched: routed experts with at least one token this step (the shared
+    expert is always touched on top).  Weight bytes per expert follow the
+    pages' 3 x d x inter parameter count ("Kimi K2.5 Q&A", Q2.1)."""
+    T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
+    rows = T * (k + 1)
+    w_gu = 2 * I * d * 2                 # gate + up weights of one expert, bytes
+    w_dn = d * I * 2
+    acc = {}
+    acc["gate_up_bytes"] = (touched + 1) * w_gu + rows * d * 2 + rows * I * 2
+    acc["down_bytes"] = (touched + 1) * w_dn + rows * I * 2 + rows * d * 2
+    acc["gate_up_flops"] = 2.0 * rows * 2 * I * d
+    acc["down_flops"] = 2.0 * rows * I * d
+    acc["router_flops"] = 2.0 * T * d * E
+    acc["weight_bytes"] = (touched + 1) * (w_gu + w_dn) + E * d * 2
+    acc["flops"] = acc["gate_up_flops"] + acc["down_flops"] + acc["router_flops"]
+    return acc
+
+
+# ------------------------------------------------------------------- oracle
+
+def run_oracle_sample(cfg, inputs_dev, n_tokens, seed=0):
+    """Oracle (routing + experts) on n_tokens evenly spread tokens; returns
+    (seconds, threads, description)."""
+    import numpy as np
+    import oracle
+    T = cfg.T
+    n = max(1, min(n_tokens, T))
+    tok = sorted(set(int(round(i * (T - 1) / max(n - 1, 1))) for i in range(n)))
+    import torch
+    sel = torch.tensor(tok, device=inputs_dev["x"].device)
+    x_s = inputs_dev["x"].index_select(0, sel).cpu()
+    wr = inputs_dev["w_router"].cpu()
+    bias = inputs_dev["bias"].cpu()
+    threads = min(host_cores(), len(tok))
+    # routing of the sampled rows (a row's routing depends on that row only)
+    ridx, rw, _ = oracle.route(x_s, wr, bias, cfg.k, cfg.scale, nthreads=threads)
+    need = sorted(set(ridx.reshape(-1).tolist()))
+    egu = [None] * cfg.E
+    edn = [None] * cfg.E
+    for e in need:
+        egu[e] = inputs_dev["w_gate_up"][e].cpu()
+        edn[e] = inputs_dev["w_down"][e].cpu()
+    sgu, sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
+    t0 = time.perf_counter()
+    ridx, rw, _ = oracle.route(x_s, wr, bias, cfg.k, cfg.scale, nthreads=threads)
+    oracle.moe_rows(x_s, ridx, rw, egu, edn, sgu, sdn, nthreads=threads)
+    dt = time.perf_counter() - t0
+    desc = (f"{len(tok)} of {T} tokens (evenly spaced), full routing + {len(need)} routed "
+            f"experts + shared expert, fp64")
+    return dt, threads, len(tok), desc
+
+
+def default_cpu_sample(cfg):
+    # ~0.8 GFLOP of fp64 per K2 token; one thread per token
+    return min(cfg.T, max(2, host_cores()))
+
+
+# --------------------------------------------------------------------- main
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    from moe_inputs import CONFIGS, make_inputs
+    if args.workload not in CONFIGS:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {sorted(CONFIGS)}")
+    cfg = CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, cfg, world)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    import sparse_moe_ffn_sigmoid_b200 as moe
+
+    dev = torch.device("cuda", local_rank)
+    g = make_inputs(cfg, seed=rank, device=dev)
+    T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.moe_layer_forward(g["x"], g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                              g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if moe.moe_device_status() != 0:
+        raise SystemExit("device status not clean after warm-up")
+    launches_per_step = moe.moe_last_launch_count()
+
+    # touched experts of this batch (our own route + permute kernels)
+    ws = torch.empty(moe.moe_workspace_size(T, d, E, k, I), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    moe.moe_route(g["x"], g["w_router"], g["bias"], k, cfg.scale, idx, w, ws)
+    i32 = lambda n: torch.empty((n,), dtype=torch.int32, device=dev)
+    counts, offs, rtok, srow = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+    moe.moe_permute(idx, E, counts, offs, rtok, srow, ws)
+    touched = int((counts > 0).sum().item())
+    del ws
+
+    # ---------------------------------------------------------- timed region
+    moe.moe_profile_begin(args.steps)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_wall0 = clk.mark()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall1 = clk.mark()
+        if world > 1:
+            dist.barrier()
+    ms_total = start.elapsed_time(end)
+    n_calls, kernel_ms = moe.moe_profile_end()
+    if moe.moe_device_status() != 0:
+        raise SystemExit("device status not clean after the timed region")
+    clocks = clk.summary(t_wall0, t_wall1)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1e3)
+
+    # ---------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        x_host = g["x"].cpu().pin_memory()
+        out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(g["x"])
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            moe.moe_layer_forward(x_dev, g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                                  g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+            out_host.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * T * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+               "ms_per_step": ms_e2e / args.steps}
+
+    # ---------------------------------------------------------- roofline
+    peaks, peak_src = load_peaks()
+    acc = layer_accounting(cfg, touched)
+    kname = "gemm_gate_up_swiglu"
+    k_ms = kernel_ms.get(kname, 0.0) / max(n_calls, 1)
+    decode_like = cfg.T * (cfg.k + 1) <= 4096 and args.workload != "k2_skew"
+    if decode_like:
+        achieved = acc["gate_up_bytes"] / (k_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "kernel": kname,
+                "algorithmic_bytes_per_launch": acc["gate_up_bytes"],
+                "avg_launch_ms": k_ms, "peak_source": f"{peak_src} hbm_gbs"}
+        layer_t = acc["weight_bytes"] / (peak * 1e9)
+        layer_roof = {"bound": "hbm", "ideal_ms": layer_t * 1e3, "frac": layer_t / (ms_step / 1e3),
+                      "weight_bytes": acc["weight_bytes"], "touched_experts": touched}
+    else:
+        achieved = acc["gate_up_flops"] / (k_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "kernel": kname,
+                "algorithmic_flops_per_launch": acc["gate_up_flops"],
+                "avg_launch_ms": k_ms, "peak_source": f"{peak_src} bf16_tflops_sustained"}
+        t_tc = acc["flops"] / (peak * 1e12)
+        t_hbm = acc["weight_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        layer_roof = {"bound": "tensor", "ideal_ms": t_tc * 1e3, "frac": t_tc / (ms_step / 1e3),
+                      "hbm_ideal_ms": t_hbm * 1e3, "hbm_frac": t_hbm / (ms_step / 1e3),
+                      "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
+                      "touched_experts": touched}
+    roof["traffic"] = profiled_traffic(args.workload, kname)
+
+    # ---------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample or default_cpu_sample(cfg)
+        dt, threads, nt, desc = run_oracle_sample(cfg, g, n)
+        cpu = {"value": nt / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "T": T, "d": d, "E": E, "k": k, "inter": I,
+                       "scale": cfg.scale, "bias": cfg.bias, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2: every step streams "
+                             f"{acc['weight_bytes'] / 1e9:.1f} GB of expert weights"},
+            "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "kernel_ms_per_step": {kk: v / max(n_calls, 1) for kk, v in kernel_ms.items()},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args, cfg, world):
+    """The oracle on the host cores, --warmup + --steps bounded samples."""
+    import torch
+    from moe_inputs import make_inputs
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    g = make_inputs(cfg, seed=0, device=dev)
+    n = args.cpu_sample or max(2, min(cfg.T, host_cores()))
+    # each step a bounded sample so the whole run stays within minutes
+    per_step = []
+    threads, nt, desc = 1, n, ""
+    for i in range(args.warmup + args.steps):
+        dt, threads, nt, desc = run_oracle_sample(cfg, g, n)
+        if i >= args.warmup:
+            per_step.append(dt)
+    total = sum(per_step)
+    value = nt * len(per_step) / total
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / len(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "inter": cfg.inter, "scale": cfg.scale, "bias": cfg.bias},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

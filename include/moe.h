@@ -1,0 +1,205 @@
+/*
+ * moe.h -- C ABI of a single-GPU (B200, sm_100a) forward pass of one
+ * Kimi-K2-style sparse MoE FFN layer with a sigmoid router.
+ *
+ * The layer ("Kimi K2.5 deep dive", CH4.2 routing and CH10.2 "MoE 7-step
+ * dataflow"; "Kimi K2.5 Q&A", Q8.3; K2 team member's answer, "different"):
+ *     s   = sigmoid(x W_r^T)                      scores, [T, E]
+ *     b   = s + bias                              selection-only bias
+ *     S_t = top-k of b_t over all E experts      (n_group = 1)
+ *     w_j = scale * s_j / sum_{i in S_t} s_i      unbiased, renormalised, scaled
+ *     out = shared(x) + sum_j w_j * f_{S_t[j]}(x)
+ *     f_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x))     SwiGLU expert
+ *
+ * Conventions for every entry point:
+ *   - bf16 tensors are passed as uint16_t* holding bf16 bit patterns;
+ *   - every tensor pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned, row-major and densely packed with the shape given;
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ *     call is asynchronous on it and never synchronises the host;
+ *   - arguments are checked on the host before anything is launched; on
+ *     error nothing is launched and a negative moe_status is returned;
+ *   - T == 0 is a no-op that returns MOE_OK;
+ *   - limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), d and inter multiples of
+ *     64 (>= 64), T * (k + 1) < 2^31;
+ *   - kernels never trap: problems they can only see on the device (an
+ *     out-of-range expert index, a wait that timed out) are recorded in a
+ *     per-device status word that moe_device_status() reads.
+ * There is no CPU fallback: a missing GPU or a failed launch is an error.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,       /* null / misaligned pointer, bad count */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2, /* d or inter not a multiple of 64, E or k out of range */
+    MOE_ERR_CUDA = -3,              /* a CUDA call or launch failed */
+    MOE_ERR_TIMEOUT = -4,           /* a device-side wait gave up (see moe_device_status) */
+    MOE_ERR_NO_MEMORY = -5          /* workspace growth failed (moe_layer_forward) */
+} moe_status;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int status);
+
+/*
+ * Bytes of device scratch that any staged call below needs for a layer of
+ * this size (the largest of their needs).  Routing, permutation and expert
+ * calls take the scratch as (workspace, workspace_bytes); its contents are not
+ * preserved between calls, and two calls that overlap on the GPU must not
+ * share it.
+ */
+size_t moe_workspace_size(int T, int d, int E, int k, int inter);
+
+/*
+ * Router, steps 1-4 ("Kimi K2.5 deep dive", CH4.2; CH10.2 steps 1-4).
+ *   x        [T, d]  bf16    hidden states
+ *   w_router [E, d]  bf16    router Linear weight (out x in)
+ *   bias     [E]     fp32    e_score_correction_bias; affects selection only
+ *   scale            fp32    routed_scaling_factor (2.827 for K2, 2.5 for DeepSeek-V3)
+ *   topk_idx [T, k]  int32   out: slot j = expert with the j-th largest biased
+ *                            score; ties go to the lower expert index
+ *   topk_w   [T, k]  fp32    out: scale * s / sum(s) over the selected set,
+ *                            s the UNBIASED sigmoid score
+ * Logits accumulate in fp32 on tensor cores; selection is taken in fp32.
+ */
+int moe_route(const uint16_t* x, const uint16_t* w_router, const float* bias, int T, int d, int E,
+              int k, float scale, int32_t* topk_idx, float* topk_w, void* workspace,
+              size_t workspace_bytes, void* stream);
+
+/*
+ * Dispatch: group the T*k (token, slot) pairs by expert ("Kimi K2.5 deep
+ * dive", CH10.2 step 6, the per-expert token mask).  Bit-exact and
+ * deterministic.
+ *   topk_idx  [T, k]  int32  in: k distinct experts in [0, E) per token
+ *   counts    [E]     int32  out: rows per expert
+ *   offsets   [E+1]   int32  out: exclusive prefix sum of counts, offsets[E] = T*k
+ *   row_token [T*k]   int32  out: row -> token; rows of expert e are
+ *                            offsets[e] .. offsets[e+1]-1 in ascending token order
+ *   slot_row  [T*k]   int32  out: (t*k + j) -> row
+ * An index outside [0, E) is skipped and recorded as MOE_ERR_INVALID_ARG in
+ * the device status; a token that repeats an expert gives unspecified (but
+ * in-bounds) rows.
+ */
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                int32_t* row_token, int32_t* slot_row, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/*
+ * Grouped SwiGLU experts ("Kimi K2.5 Q&A", Q8.3 step 5; "Kimi K2.5 deep
+ * dive", CH4.3 and CH10.2 step 6): for every row r of expert e,
+ *     y[r] = W_down,e ( silu(W_gate,e x[row_token[r]]) * (W_up,e x[row_token[r]]) )
+ *   x         [T, d]        bf16
+ *   row_token [T*k]         int32  (from moe_permute)
+ *   offsets   [E+1]         int32  (from moe_permute), offsets[E] == T*k
+ *   w_gate_up [E, 2*inter, d] bf16 rows [0, inter) = gate_proj, [inter, 2*inter) = up_proj
+ *   w_down    [E, d, inter] bf16   down_proj
+ *   y         [T*k, d]      bf16   out, in row (permuted) order
+ * bf16 x bf16 -> fp32 on tcgen05 tensor cores; the intermediate
+ * silu(gate) * up is rounded to bf16.  The shared expert is the case E = 1,
+ * k = 1, row_token = 0..T-1, offsets = {0, T}.
+ */
+int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* offsets,
+                   const uint16_t* w_gate_up, const uint16_t* w_down, int T, int d, int E, int k,
+                   int inter, uint16_t* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Combine, step 7 ("Kimi K2.5 deep dive", CH10.2; "Kimi K2.5 Q&A", Q8.3):
+ *     out[t] = y_shared[t] + sum_{j<k} topk_w[t, j] * y[slot_row[t*k + j]]
+ * accumulated in fp32 in slot order j = 0..k-1 (deterministic), rounded
+ * once to bf16.
+ *   y        [T*k, d] bf16   routed expert outputs in row order
+ *   y_shared [T, d]   bf16   shared expert output, or NULL for none
+ *   topk_w   [T, k]   fp32   (already includes the scaling factor)
+ *   slot_row [T*k]    int32
+ *   out      [T, d]   bf16
+ */
+int moe_combine(const uint16_t* y, const uint16_t* y_shared, const float* topk_w,
+                const int32_t* slot_row, int T, int d, int k, uint16_t* out, void* stream);
+
+/*
+ * The whole layer in one call: route -> permute -> grouped SwiGLU experts
+ * (routed and shared in the same grouped launches) -> combine
+ * ("Kimi K2.5 deep dive", CH10.2 steps 1-7).
+ *   x          [T, d]            bf16
+ *   w_router   [E, d]            bf16
+ *   bias       [E]               fp32
+ *   w_gate_up  [E, 2*inter, d]   bf16  routed experts, gate rows then up rows
+ *   w_down     [E, d, inter]     bf16
+ *   ws_gate_up [2*inter, d]      bf16  shared expert
+ *   ws_down    [d, inter]        bf16
+ *   out        [T, d]            bf16
+ * Scratch is library-owned: one buffer per (device, stream), grown with
+ * cudaMallocAsync on `stream` when a larger layer arrives and kept for later
+ * calls (MOE_ERR_NO_MEMORY if growth fails).  Calls on one stream are
+ * ordered; calls on different streams use different buffers.
+ */
+int moe_layer_forward(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                      const uint16_t* w_gate_up, const uint16_t* w_down,
+                      const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d, int E,
+                      int k, int inter, float scale, uint16_t* out, void* stream);
+
+/*
+ * moe_layer_forward with caller-owned scratch of at least
+ * moe_workspace_size(T, d, E, k, inter) bytes (nothing is allocated).
+ */
+int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                         const uint16_t* w_gate_up, const uint16_t* w_down,
+                         const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                         int E, int k, int inter, float scale, uint16_t* out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's status word:
+ * *device_status = MOE_OK, or the first problem a kernel recorded since the
+ * last read (MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT).  Returns MOE_OK or
+ * MOE_ERR_CUDA if the synchronisation itself failed.
+ */
+int moe_device_status(void* stream, int* device_status);
+
+/*
+ * Upper bound, in nanoseconds, on every device-side wait of the library's
+ * kernels (default 2e9 = 2 s).  A wait that runs out records MOE_ERR_TIMEOUT,
+ * and the kernel winds down and returns instead of hanging.
+ */
+void moe_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/*
+ * Failure-detection self-test: launches one block that waits on an mbarrier
+ * nobody arrives on, bounded by `timeout_ns`.  The wait runs out, the kernel
+ * records MOE_ERR_TIMEOUT and returns; the context stays usable.
+ */
+int moe_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Kernels the last moe_layer_forward / moe_layer_forward_ws launched. */
+int moe_last_launch_count(void);
+
+/*
+ * Optional per-kernel timing of layer calls with CUDA events (measurement
+ * support; no counterpart in the method).  After moe_profile_begin(n), the
+ * next n calls of moe_layer_forward / moe_layer_forward_ws on the current
+ * device record one event before their first kernel and one after each
+ * kernel, on the call's stream.  moe_profile_end synchronises those events,
+ * writes into total_ms[i] (i < max_kernels) the summed time of the i-th
+ * kernel of a call over the recorded calls, stores the number of recorded
+ * calls in *n_calls, frees the events and returns the number of kernels per
+ * call (or a negative moe_status).
+ */
+int moe_profile_begin(int max_calls);
+int moe_profile_end(float* total_ms, int max_kernels, int* n_calls);
+
+/* Name of the i-th kernel a layer call launches ("" if out of range). */
+const char* moe_kernel_name(int i);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

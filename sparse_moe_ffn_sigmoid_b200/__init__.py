@@ -1,0 +1,222 @@
+"""Python binding of libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: every function takes torch CUDA tensors (PyTorch
+provides device memory and streams), checks dtype / device / contiguity,
+passes raw pointers to the C entry point of the same name on the current
+torch stream, and raises MoeError on a non-zero status.  All arithmetic runs
+in the library's CUDA kernels; there is no CPU fallback, and importing this
+package fails loudly if the library cannot be built or loaded.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "MoeError", "lib", "moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
+    "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_ws",
+    "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
+    "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
+    "EXPORTED_SYMBOLS",
+]
+
+# Every function declared in include/moe.h.
+EXPORTED_SYMBOLS = [
+    "moe_status_string", "moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn",
+    "moe_combine", "moe_layer_forward", "moe_layer_forward_ws", "moe_device_status",
+    "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
+    "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
+]
+
+MOE_OK = 0
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {moe_status_string(code)} ({code})")
+
+
+def _load():
+    path = _build.build()
+    L = ctypes.CDLL(path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    SZ, U64 = ctypes.c_size_t, ctypes.c_uint64
+    sig = {
+        "moe_status_string": ([I], ctypes.c_char_p),
+        "moe_workspace_size": ([I, I, I, I, I], SZ),
+        "moe_route": ([P, P, P, I, I, I, I, F, P, P, P, SZ, P], I),
+        "moe_permute": ([P, I, I, I, P, P, P, P, P, SZ, P], I),
+        "moe_expert_ffn": ([P, P, P, P, P, I, I, I, I, I, P, P, SZ, P], I),
+        "moe_combine": ([P, P, P, P, I, I, I, P, P], I),
+        "moe_layer_forward": ([P, P, P, P, P, P, P, I, I, I, I, I, F, P, P], I),
+        "moe_layer_forward_ws": ([P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, SZ, P], I),
+        "moe_device_status": ([P, ctypes.POINTER(I)], I),
+        "moe_set_wait_timeout_ns": ([U64], None),
+        "moe_selftest_wait_timeout": ([U64, P], I),
+        "moe_last_launch_count": ([], I),
+        "moe_profile_begin": ([I], I),
+        "moe_profile_end": ([ctypes.POINTER(F), I, ctypes.POINTER(I)], I),
+        "moe_kernel_name": ([I], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+_LIB = _load()
+
+
+def lib():
+    return _LIB
+
+
+# ------------------------------------------------------------- marshalling
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t, dtype, name, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn, rc):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+# ------------------------------------------------------------------- calls
+
+def moe_status_string(code: int) -> str:
+    return _LIB.moe_status_string(int(code)).decode()
+
+
+def moe_workspace_size(T: int, d: int, E: int, k: int, inter: int) -> int:
+    return int(_LIB.moe_workspace_size(T, d, E, k, inter))
+
+
+def moe_route(x, w_router, bias, k: int, scale: float, topk_idx, topk_w, workspace, stream=None):
+    T, d = x.shape
+    E = w_router.shape[0]
+    rc = _LIB.moe_route(_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"),
+                        _ptr(bias, F32, "bias"), T, d, E, k, float(scale),
+                        _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
+                        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                        _stream(stream))
+    _check("moe_route", rc)
+
+
+def moe_permute(topk_idx, E: int, counts, offsets, row_token, slot_row, workspace, stream=None):
+    T, k = topk_idx.shape
+    rc = _LIB.moe_permute(_ptr(topk_idx, I32, "topk_idx"), T, E, k, _ptr(counts, I32, "counts"),
+                          _ptr(offsets, I32, "offsets"), _ptr(row_token, I32, "row_token"),
+                          _ptr(slot_row, I32, "slot_row"),
+                          _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                          _stream(stream))
+    _check("moe_permute", rc)
+
+
+def moe_expert_ffn(x, row_token, offsets, w_gate_up, w_down, k: int, y, workspace, stream=None):
+    T, d = x.shape
+    E, two_i, _ = w_gate_up.shape
+    rc = _LIB.moe_expert_ffn(_ptr(x, BF16, "x"), _ptr(row_token, I32, "row_token"),
+                             _ptr(offsets, I32, "offsets"), _ptr(w_gate_up, BF16, "w_gate_up"),
+                             _ptr(w_down, BF16, "w_down"), T, d, E, k, two_i // 2,
+                             _ptr(y, BF16, "y"), _ptr(workspace, torch.uint8, "workspace"),
+                             workspace.numel(), _stream(stream))
+    _check("moe_expert_ffn", rc)
+
+
+def moe_combine(y, y_shared, topk_w, slot_row, out, stream=None):
+    T, k = topk_w.shape
+    d = y.shape[1]
+    rc = _LIB.moe_combine(_ptr(y, BF16, "y"), _ptr(y_shared, BF16, "y_shared", optional=True),
+                          _ptr(topk_w, F32, "topk_w"), _ptr(slot_row, I32, "slot_row"), T, d, k,
+                          _ptr(out, BF16, "out"), _stream(stream))
+    _check("moe_combine", rc)
+
+
+def _layer_args(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down):
+    T, d = x.shape
+    E = w_router.shape[0]
+    inter = w_gate_up.shape[1] // 2
+    return ([_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"), _ptr(bias, F32, "bias"),
+             _ptr(w_gate_up, BF16, "w_gate_up"), _ptr(w_down, BF16, "w_down"),
+             _ptr(ws_gate_up, BF16, "ws_gate_up"), _ptr(ws_down, BF16, "ws_down")],
+            T, d, E, inter)
+
+
+def moe_layer_forward(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, k: int,
+                      scale: float, out, stream=None):
+    ptrs, T, d, E, inter = _layer_args(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward(*ptrs, T, d, E, k, inter, float(scale), _ptr(out, BF16, "out"),
+                                _stream(stream))
+    _check("moe_layer_forward", rc)
+
+
+def moe_layer_forward_ws(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, k: int,
+                         scale: float, out, workspace, stream=None):
+    ptrs, T, d, E, inter = _layer_args(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_ws(*ptrs, T, d, E, k, inter, float(scale),
+                                   _ptr(out, BF16, "out"),
+                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                   _stream(stream))
+    _check("moe_layer_forward_ws", rc)
+
+
+def moe_device_status(stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check("moe_device_status", _LIB.moe_device_status(_stream(stream), ctypes.byref(v)))
+    return v.value
+
+
+def moe_set_wait_timeout_ns(ns: int) -> None:
+    _LIB.moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_selftest_wait_timeout(ns: int, stream=None) -> None:
+    _check("moe_selftest_wait_timeout", _LIB.moe_selftest_wait_timeout(int(ns), _stream(stream)))
+
+
+def moe_last_launch_count() -> int:
+    return int(_LIB.moe_last_launch_count())
+
+
+def moe_profile_begin(max_calls: int) -> None:
+    _check("moe_profile_begin", _LIB.moe_profile_begin(int(max_calls)))
+
+
+def moe_profile_end():
+    """-> (n_calls, {kernel name: summed ms over the recorded calls})."""
+    buf = (ctypes.c_float * 32)()
+    n = ctypes.c_int(0)
+    nk = _LIB.moe_profile_end(buf, 32, ctypes.byref(n))
+    if nk < 0:
+        raise MoeError("moe_profile_end", nk)
+    return n.value, {moe_kernel_name(i): float(buf[i]) for i in range(nk)}
+
+
+def moe_kernel_name(i: int) -> str:
+    return _LIB.moe_kernel_name(int(i)).decode()

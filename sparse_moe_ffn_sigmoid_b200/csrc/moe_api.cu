@@ -1,0 +1,666 @@
+// moe_api.cu -- the C ABI of include/moe.h: argument checks, scratch layout,
+// TMA descriptors and the launch sequence of the MoE layer forward pass.
+//
+// Everything here is host code except the kernels it includes; it is built
+// as one translation unit (kernels in the *.cuh files next to it).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "combine.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTargetCtas = 148;          // SMs of a B200: the router's split heuristic
+constexpr int kMaxSplits = 64;
+constexpr size_t kMaxDynSmem = 232448;    // 227 KB opt-in per block on sm_100
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<int> g_last_launches{0};
+
+// Kernels of one layer call, in launch order (moe_kernel_name).
+constexpr int kLayerKernels = 9;
+const char* const kKernelNames[kLayerKernels] = {
+    "router_gemm", "topk", "permute_hist", "scan_plan", "permute_scatter",
+    "gather_rows", "gemm_gate_up_swiglu", "gemm_down", "combine"};
+
+// Optional per-kernel CUDA-event timing of layer calls (moe_profile_begin/end).
+struct Profile {
+    std::mutex mu;
+    std::vector<cudaEvent_t> ev;   // [calls][kLayerKernels + 1]
+    int max_calls = 0;
+    int calls = 0;
+} g_prof;
+
+// Counts the kernels a call launches and, when a profile slot is given,
+// records an event on the stream after each of them.
+struct Recorder {
+    cudaEvent_t* ev = nullptr;     // kLayerKernels + 1 events, or null
+    int n = 0;
+    void start(cudaStream_t st) {
+        if (ev) cudaEventRecord(ev[0], st);
+    }
+    void mark(cudaStream_t st) {
+        ++n;
+        if (ev && n <= kLayerKernels) cudaEventRecord(ev[n], st);
+    }
+};
+
+// ------------------------------------------------------------------ checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(int T, int d, int E, int k, int inter) {
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (d < 64 || d % 64 != 0 || inter < 64 || inter % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(T) * (k + 1) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(E) * 2 * inter >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(E) * d >= (1ll << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+template <typename... P>
+bool all_ok(P... p) {
+    return ((p != nullptr && aligned16(p)) && ...);
+}
+
+// ------------------------------------------------------------------ layout
+
+int router_splits(int T, int d, int E) {
+    const int nt = (T + kMaxN - 1) / kMaxN;
+    const int mslabs = (E + kSlabRows - 1) / kSlabRows;
+    const int base = std::max(1, nt * mslabs);
+    const int ks = d / kBK;
+    int best = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= std::min(ks, kMaxSplits); ++s) {
+        const int waves = (base * s + kTargetCtas - 1) / kTargetCtas;
+        const double cost = waves * static_cast<double>((ks + s - 1) / s) + 0.02 * s;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+struct Layout {
+    size_t partials, topk_idx, topk_w, blk, counts, offsets, row_token, slot_row;
+    size_t tiles1, tiles2, ntiles, xperm, h, y, total;
+    int splits, nblk, max_tiles1, max_tiles2;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+Layout make_layout(int T, int d, int E, int k, int inter) {
+    Layout L{};
+    const size_t Tk = static_cast<size_t>(T) * k;
+    const size_t rows = Tk + T;   // routed rows, then the shared expert's rows
+    L.splits = router_splits(T, d, E);
+    L.nblk = (T + kPermTokens - 1) / kPermTokens;
+    const long long token_tiles = static_cast<long long>(Tk / kMaxN) +
+                                  std::min<long long>(E, static_cast<long long>(Tk)) + 1 +
+                                  (T + kMaxN - 1) / kMaxN;
+    L.max_tiles1 = static_cast<int>(token_tiles * ((inter + kSlabRows - 1) / kSlabRows));
+    L.max_tiles2 = static_cast<int>(token_tiles * ((d + 2 * kSlabRows - 1) / (2 * kSlabRows)));
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.partials = take(static_cast<size_t>(L.splits) * T * E * sizeof(float));
+    L.topk_idx = take(Tk * sizeof(int));
+    L.topk_w = take(Tk * sizeof(float));
+    L.blk = take(static_cast<size_t>(std::max(L.nblk, 1)) * E * sizeof(int));
+    L.counts = take(static_cast<size_t>(E) * sizeof(int));
+    L.offsets = take(static_cast<size_t>(E + 2) * sizeof(int));
+    L.row_token = take(Tk * sizeof(int));
+    L.slot_row = take(Tk * sizeof(int));
+    L.tiles1 = take(static_cast<size_t>(L.max_tiles1) * 2 * sizeof(int4));
+    L.tiles2 = take(static_cast<size_t>(L.max_tiles2) * 2 * sizeof(int4));
+    L.ntiles = take(4 * sizeof(int));
+    L.xperm = take(Tk * d * sizeof(bf16));
+    L.h = take(rows * inter * sizeof(bf16));
+    L.y = take(rows * d * sizeof(bf16));
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------- device info
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        di.ready = true;
+    }
+    *out = di;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of box_rows x 64 columns,
+// 128-byte swizzled (the layout the UMMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * sizeof(bf16)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- launches
+
+void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
+    a.nslab = nslab;
+    a.n_max = n_max;
+    const size_t stage = static_cast<size_t>(nslab) * kSlabBytes + static_cast<size_t>(n_max) * kBK * 2;
+    int stages = static_cast<int>((kMaxDynSmem - 1024 - 256) / stage);
+    a.stages = std::max(2, std::min(stages, 8));
+    a.acc_stride = nslab * n_max;
+    a.acc_bufs = (2 * a.acc_stride <= kTmemCols) ? 2 : 1;
+    a.timeout_ns = g_timeout_ns.load();
+}
+
+template <int EPI>
+int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
+    const size_t smem = gemm_smem_bytes(a.stages, a.nslab, a.n_max);
+    if (smem > kMaxDynSmem) return MOE_ERR_UNSUPPORTED_SHAPE;
+    moe_gemm_kernel<EPI><<<grid, kGemmThreads, smem, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const float* bias, int T,
+                 int d, int E, int k, float scale, int* idx, float* w, float* partials,
+                 int splits, cudaStream_t st, Recorder& rec) {
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int nt = (T + kMaxN - 1) / kMaxN;
+    const int chunk = (((T + nt - 1) / nt) + 15) & ~15;
+    if (!make_map(&a.a_map[0], wr, E, d, kSlabRows) || !make_map(&a.b_map[0], x, T, d, kBoxRows))
+        return MOE_ERR_CUDA;
+    a.a_map[1] = a.a_map[0];
+    a.b_map[1] = a.b_map[0];
+    a.tiles = nullptr;
+    a.dense_mslabs = (E + kSlabRows - 1) / kSlabRows;
+    a.dense_ttiles = nt;
+    a.dense_tchunk = chunk;
+    a.dense_splits = splits;
+    a.dense_T = T;
+    a.dense_ksteps = d / kBK;
+    a.ntiles_host = a.dense_mslabs * nt * splits;
+    a.out = partials;
+    a.out_ld = E;
+    a.col_limit = E;
+    fill_pipeline(a, 1, chunk);
+    int rc = launch_gemm<kEpiStoreF32>(a, std::min(a.ntiles_host, di.sms), st);
+    if (rc != MOE_OK) return rc;
+    rec.mark(st);
+    const int npl = (E + 31) / 32;
+    const dim3 grid((T + 7) / 8), block(256);
+    const long long sstride = static_cast<long long>(T) * E;
+#define MOE_TOPK(N)                                                                          \
+    topk_kernel<N><<<grid, block, 0, st>>>(partials, splits, sstride, T, E, k, bias, scale, idx, \
+                                           w)
+    if (npl <= 1) MOE_TOPK(1);
+    else if (npl <= 2) MOE_TOPK(2);
+    else if (npl <= 4) MOE_TOPK(4);
+    else if (npl <= 8) MOE_TOPK(8);
+    else if (npl <= 12) MOE_TOPK(12);
+    else if (npl <= 16) MOE_TOPK(16);
+    else if (npl <= 24) MOE_TOPK(24);
+    else MOE_TOPK(32);
+#undef MOE_TOPK
+    rec.mark(st);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offsets, int* row_token,
+                   int* slot_row, int* blk, const PlanArgs& plan, cudaStream_t st, Recorder& rec) {
+    const int nblk = (T + kPermTokens - 1) / kPermTokens;
+    permute_hist_kernel<<<nblk, kPermTokens, 4 * E * sizeof(uint32_t), st>>>(idx, T, E, k, blk);
+    rec.mark(st);
+    scan_plan_kernel<<<1, 1024, 0, st>>>(blk, nblk, E, counts, offsets, plan);
+    rec.mark(st);
+    permute_scatter_kernel<<<nblk, kPermTokens, 8 * E * sizeof(uint32_t), st>>>(
+        idx, T, E, k, blk, row_token, slot_row);
+    rec.mark(st);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// gather + gate|up + down over a planned tile list.
+//   rows_b0: rows of the permuted token matrix (T*k); h_rows / y rows: rows_b0 (+ T if shared)
+int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T, int d, int E,
+               int k, int inter, const bf16* w_gate_up, const bf16* w_down,
+               const bf16* ws_gate_up, const bf16* ws_down, bool shared, bf16* xperm, bf16* h,
+               bf16* y, const int4* tiles1, const int4* tiles2, const int* ntiles,
+               int max_tiles1, int max_tiles2, cudaStream_t st, Recorder& rec) {
+    const int rows_routed = T * k;
+    const int rows_all = rows_routed + (shared ? T : 0);
+    if (rows_routed > 0) {
+        gather_rows_kernel<<<(rows_routed + 7) / 8, 256, 0, st>>>(x, row_token, T, rows_routed, d,
+                                                                  xperm);
+        rec.mark(st);
+    }
+    // largest token tile: an expert never holds more rows than its token count
+    const int max_rows = shared ? T : rows_routed;
+    const int n_max = std::min(kMaxN, (max_rows + 15) & ~15);
+
+    GemmArgs g1;
+    std::memset(&g1, 0, sizeof(g1));
+    const bf16* xp = rows_routed > 0 ? xperm : x;
+    if (!make_map(&g1.a_map[0], w_gate_up, static_cast<uint64_t>(E) * 2 * inter, d, kSlabRows) ||
+        !make_map(&g1.b_map[0], xp, std::max(rows_routed, 1), d, kBoxRows) ||
+        !make_map(&g1.b_map[1], x, T, d, kBoxRows))
+        return MOE_ERR_CUDA;
+    if (shared) {
+        if (!make_map(&g1.a_map[1], ws_gate_up, 2ull * inter, d, kSlabRows)) return MOE_ERR_CUDA;
+    } else {
+        g1.a_map[1] = g1.a_map[0];   // no tile refers to slot 1
+    }
+    g1.tiles = tiles1;
+    g1.ntiles_dev = ntiles;
+    g1.out = h;
+    g1.out_ld = inter;
+    g1.col_limit = inter;
+    fill_pipeline(g1, 2, n_max);
+    int rc = launch_gemm<kEpiSwiGLU>(g1, std::min(max_tiles1, di.sms), st);
+    if (rc != MOE_OK) return rc;
+    rec.mark(st);
+
+    GemmArgs g2;
+    std::memset(&g2, 0, sizeof(g2));
+    if (!make_map(&g2.a_map[0], w_down, static_cast<uint64_t>(E) * d, inter, kSlabRows) ||
+        !make_map(&g2.b_map[0], h, rows_all, inter, kBoxRows))
+        return MOE_ERR_CUDA;
+    if (shared) {
+        if (!make_map(&g2.a_map[1], ws_down, d, inter, kSlabRows)) return MOE_ERR_CUDA;
+    } else {
+        g2.a_map[1] = g2.a_map[0];
+    }
+    g2.b_map[1] = g2.b_map[0];
+    g2.tiles = tiles2;
+    g2.ntiles_dev = ntiles + 1;
+    g2.out = y;
+    g2.out_ld = d;
+    g2.col_limit = d;
+    fill_pipeline(g2, 2, n_max);
+    rc = launch_gemm<kEpiStoreBF16>(g2, std::min(max_tiles2, di.sms), st);
+    if (rc != MOE_OK) return rc;
+    rec.mark(st);
+    return MOE_OK;
+}
+
+int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* slot_row, int T,
+                   int d, int k, bf16* out, cudaStream_t st, Recorder& rec) {
+    combine_kernel<<<T, 128, 0, st>>>(y, ysh, w, slot_row, T, d, k,
+                                      static_cast<long long>(T) * k, out);
+    rec.mark(st);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+        // nobody arrives: the bounded wait must give up and record a timeout
+        wait_bounded(&bar, 0, nullptr, timeout_ns);
+    }
+}
+
+int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* wgu,
+                  const bf16* wdn, const bf16* sgu, const bf16* sdn, int T, int d, int E, int k,
+                  int inter, float scale, bf16* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+    const Layout L = make_layout(T, d, E, k, inter);
+    if (ws == nullptr || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    auto P = [&](size_t off) { return base + off; };
+    int* idx = reinterpret_cast<int*>(P(L.topk_idx));
+    float* w = reinterpret_cast<float*>(P(L.topk_w));
+    int* counts = reinterpret_cast<int*>(P(L.counts));
+    int* offsets = reinterpret_cast<int*>(P(L.offsets));
+    int* row_token = reinterpret_cast<int*>(P(L.row_token));
+    int* slot_row = reinterpret_cast<int*>(P(L.slot_row));
+    int4* tiles1 = reinterpret_cast<int4*>(P(L.tiles1));
+    int4* tiles2 = reinterpret_cast<int4*>(P(L.tiles2));
+    int* ntiles = reinterpret_cast<int*>(P(L.ntiles));
+    bf16* xperm = reinterpret_cast<bf16*>(P(L.xperm));
+    bf16* h = reinterpret_cast<bf16*>(P(L.h));
+    bf16* y = reinterpret_cast<bf16*>(P(L.y));
+    Recorder rec;
+    {
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        if (g_prof.calls < g_prof.max_calls) {
+            rec.ev = g_prof.ev.data() + static_cast<size_t>(g_prof.calls) * (kLayerKernels + 1);
+            ++g_prof.calls;
+        }
+    }
+    rec.start(st);
+    rc = launch_route(di, x, wr, bias, T, d, E, k, scale, idx, w,
+                      reinterpret_cast<float*>(P(L.partials)), L.splits, st, rec);
+    if (rc != MOE_OK) return rc;
+    PlanArgs plan{E, 1, T, d, inter, T * k, tiles1, tiles2, ntiles};
+    rc = launch_permute(idx, T, E, k, counts, offsets, row_token, slot_row,
+                        reinterpret_cast<int*>(P(L.blk)), plan, st, rec);
+    if (rc != MOE_OK) return rc;
+    rc = launch_ffn(di, x, row_token, T, d, E, k, inter, wgu, wdn, sgu, sdn, true, xperm, h, y,
+                    tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec);
+    if (rc != MOE_OK) return rc;
+    rc = launch_combine(y, y + static_cast<size_t>(T) * k * d, w, slot_row, T, d, k, out, st, rec);
+    g_last_launches.store(rec.n);
+    return rc;
+}
+
+// Library-owned scratch of moe_layer_forward, one buffer per (device, stream).
+struct WsEntry {
+    int dev;
+    cudaStream_t stream;
+    void* ptr;
+    size_t bytes;
+};
+std::mutex g_ws_mu;
+std::vector<WsEntry> g_ws;
+
+int owned_workspace(cudaStream_t st, size_t need, void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (WsEntry& e : g_ws) {
+        if (e.dev == dev && e.stream == st) {
+            if (e.bytes < need) {
+                if (e.ptr) cudaFreeAsync(e.ptr, st);
+                e.ptr = nullptr;
+                e.bytes = 0;
+                if (cudaMallocAsync(&e.ptr, need, st) != cudaSuccess) {
+                    cudaGetLastError();
+                    return MOE_ERR_NO_MEMORY;
+                }
+                e.bytes = need;
+            }
+            *out = e.ptr;
+            return MOE_OK;
+        }
+    }
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, need, st) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_NO_MEMORY;
+    }
+    g_ws.push_back({dev, st, p, need});
+    *out = p;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+        case MOE_ERR_NO_MEMORY: return "MOE_ERR_NO_MEMORY";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+size_t moe_workspace_size(int T, int d, int E, int k, int inter) {
+    if (check_dims(T, d, E, k, inter) != MOE_OK) return 0;
+    return make_layout(T, d, E, k, inter).total;
+}
+
+int moe_route(const uint16_t* x, const uint16_t* w_router, const float* bias, int T, int d, int E,
+              int k, float scale, int32_t* topk_idx, float* topk_w, void* workspace,
+              size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, 64);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, topk_idx, topk_w, workspace)) return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    const int splits = router_splits(T, d, E);
+    if (workspace_bytes < static_cast<size_t>(splits) * T * E * sizeof(float))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    Recorder rec;
+    return launch_route(di, reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                        bias, T, d, E, k, scale, topk_idx, topk_w, static_cast<float*>(workspace),
+                        splits, static_cast<cudaStream_t>(stream), rec);
+}
+
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
+                int32_t* row_token, int32_t* slot_row, void* workspace, size_t workspace_bytes,
+                void* stream) {
+    int rc = check_dims(T, 64, E, k, 64);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(topk_idx, counts, offsets, row_token, slot_row, workspace))
+        return MOE_ERR_INVALID_ARG;
+    const int nblk = (T + kPermTokens - 1) / kPermTokens;
+    if (workspace_bytes < static_cast<size_t>(nblk) * E * sizeof(int)) return MOE_ERR_INVALID_ARG;
+    PlanArgs none{};
+    Recorder rec;
+    return launch_permute(topk_idx, T, E, k, counts, offsets, row_token, slot_row,
+                          static_cast<int*>(workspace), none, static_cast<cudaStream_t>(stream),
+                          rec);
+}
+
+int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* offsets,
+                   const uint16_t* w_gate_up, const uint16_t* w_down, int T, int d, int E, int k,
+                   int inter, uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, row_token, offsets, w_gate_up, w_down, y, workspace)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(T, d, E, k, inter);
+    if (workspace_bytes < L.total) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    int4* tiles1 = reinterpret_cast<int4*>(base + L.tiles1);
+    int4* tiles2 = reinterpret_cast<int4*>(base + L.tiles2);
+    int* ntiles = reinterpret_cast<int*>(base + L.ntiles);
+    PlanArgs plan{E, 0, T, d, inter, T * k, tiles1, tiles2, ntiles};
+    plan_kernel<<<1, 1024, 0, st>>>(offsets, plan);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    Recorder rec;
+    return launch_ffn(di, reinterpret_cast<const bf16*>(x), row_token, T, d, E, k, inter,
+                      reinterpret_cast<const bf16*>(w_gate_up), reinterpret_cast<const bf16*>(w_down),
+                      nullptr, nullptr, false, reinterpret_cast<bf16*>(base + L.xperm),
+                      reinterpret_cast<bf16*>(base + L.h), reinterpret_cast<bf16*>(y), tiles1,
+                      tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec);
+}
+
+int moe_combine(const uint16_t* y, const uint16_t* y_shared, const float* topk_w,
+                const int32_t* slot_row, int T, int d, int k, uint16_t* out, void* stream) {
+    if (T < 0 || k < 1 || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (d < 8 || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(y, topk_w, slot_row, out)) return MOE_ERR_INVALID_ARG;
+    if (y_shared != nullptr && !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
+    Recorder rec;
+    return launch_combine(reinterpret_cast<const bf16*>(y), reinterpret_cast<const bf16*>(y_shared),
+                          topk_w, slot_row, T, d, k, reinterpret_cast<bf16*>(out),
+                          static_cast<cudaStream_t>(stream), rec);
+}
+
+int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                         const uint16_t* w_gate_up, const uint16_t* w_down,
+                         const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                         int E, int k, int inter, float scale, uint16_t* out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, out, workspace))
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    return layer_forward(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                         bias, reinterpret_cast<const bf16*>(w_gate_up),
+                         reinterpret_cast<const bf16*>(w_down),
+                         reinterpret_cast<const bf16*>(ws_gate_up),
+                         reinterpret_cast<const bf16*>(ws_down), T, d, E, k, inter, scale,
+                         reinterpret_cast<bf16*>(out), workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int moe_layer_forward(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                      const uint16_t* w_gate_up, const uint16_t* w_down,
+                      const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d, int E,
+                      int k, int inter, float scale, uint16_t* out, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, out))
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    const size_t need = make_layout(T, d, E, k, inter).total;
+    void* ws = nullptr;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = owned_workspace(st, need, &ws);
+    if (rc != MOE_OK) return rc;
+    return moe_layer_forward_ws(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, T, d, E,
+                                k, inter, scale, out, ws, need, stream);
+}
+
+int moe_device_status(void* stream, int* device_status) {
+    if (device_status == nullptr) return MOE_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    *device_status = v;
+    return MOE_OK;
+}
+
+void moe_set_wait_timeout_ns(uint64_t timeout_ns) {
+    g_timeout_ns.store(timeout_ns == 0 ? 1 : timeout_ns);
+}
+
+int moe_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_last_launch_count(void) { return g_last_launches.load(); }
+
+int moe_profile_begin(int max_calls) {
+    if (max_calls < 0) return MOE_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+    g_prof.ev.clear();
+    g_prof.calls = 0;
+    g_prof.max_calls = 0;
+    const size_t n = static_cast<size_t>(max_calls) * (kLayerKernels + 1);
+    g_prof.ev.resize(n);
+    for (size_t i = 0; i < n; ++i)
+        if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) {
+            for (size_t j = 0; j < i; ++j) cudaEventDestroy(g_prof.ev[j]);
+            g_prof.ev.clear();
+            return MOE_ERR_CUDA;
+        }
+    g_prof.max_calls = max_calls;
+    return MOE_OK;
+}
+
+int moe_profile_end(float* total_ms, int max_kernels, int* n_calls) {
+    if (total_ms == nullptr || n_calls == nullptr || max_kernels < 0) return MOE_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    for (int i = 0; i < max_kernels; ++i) total_ms[i] = 0.0f;
+    int rc = MOE_OK;
+    for (int c = 0; c < g_prof.calls; ++c) {
+        cudaEvent_t* ev = g_prof.ev.data() + static_cast<size_t>(c) * (kLayerKernels + 1);
+        if (cudaEventSynchronize(ev[kLayerKernels]) != cudaSuccess) rc = MOE_ERR_CUDA;
+        for (int i = 0; i < std::min(max_kernels, kLayerKernels); ++i) {
+            float ms = 0.0f;
+            if (cudaEventElapsedTime(&ms, ev[i], ev[i + 1]) != cudaSuccess) rc = MOE_ERR_CUDA;
+            total_ms[i] += ms;
+        }
+    }
+    *n_calls = g_prof.calls;
+    for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+    g_prof.ev.clear();
+    g_prof.calls = 0;
+    g_prof.max_calls = 0;
+    return rc == MOE_OK ? kLayerKernels : rc;
+}
+
+const char* moe_kernel_name(int i) {
+    return (i >= 0 && i < kLayerKernels) ? kKernelNames[i] : "";
+}
+
+}  // extern "C"

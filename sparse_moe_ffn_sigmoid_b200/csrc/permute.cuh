@@ -1,0 +1,286 @@
+// permute.cuh -- deterministic token dispatch: per-expert histogram, exclusive
+// scan, stable scatter into expert-contiguous rows, and the row gather.
+//
+// The pages dispatch with one boolean mask per expert ("Kimi K2.5 deep dive",
+// CH10.2 step 6: token_mask = topk_indices == expert_i), which visits the
+// tokens of an expert in ascending order.  This file builds the same grouping
+// in three passes, bit-exact and independent of scheduling:
+//   1. permute_hist:    per 128-token block, a bitmask per (warp, expert) of
+//                       the lanes that chose the expert (atomicOr: order-free),
+//                       popcounts -> block counts [nblk][E]
+//   2. scan_plan:       block counts -> per-(block, expert) bases, counts,
+//                       offsets (exclusive scan), optional GEMM tile lists
+//   3. permute_scatter: rank inside the block = warp prefix + popc(mask & lanes
+//                       below) -> row_token[row] = t, slot_row[t*k+j] = row
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+
+constexpr int kPermTokens = 128;   // tokens per block (4 warps)
+
+__global__ void __launch_bounds__(kPermTokens) permute_hist_kernel(
+    const int* __restrict__ topk_idx, int T, int E, int k, int* __restrict__ blk_counts) {
+    extern __shared__ uint32_t mask[];   // [4][E]
+    for (int i = threadIdx.x; i < 4 * E; i += blockDim.x) mask[i] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kPermTokens + threadIdx.x;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(long long)t * k + j];
+            if (e >= 0 && e < E)
+                atomicOr(&mask[w * E + e], 1u << lane);
+            else
+                record_status(kStatusInvalidArg);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+        for (int ww = 0; ww < 4; ++ww) c += __popc(mask[ww * E + e]);
+        blk_counts[(long long)blockIdx.x * E + e] = c;
+    }
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* scratch /*[32]*/) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) scratch[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int s = scratch[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, off);
+            if (lane >= off) s += y;
+        }
+        scratch[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    const int warp_base = w > 0 ? scratch[w - 1] : 0;
+    const int tot = scratch[31];
+    __syncthreads();
+    *total = tot;
+    return warp_base + x - v;
+}
+
+// Tile plan of the grouped SwiGLU FFN.  Expert g (0..G-1) owns rows
+// [row0_g, row0_g + c_g); the shared expert (if present) is g = G-1 and reads
+// its tokens from the unpermuted map.  Each expert's rows are cut into
+// ceil(c/256) token tiles of equal 16-multiple size; tiles are listed expert
+// by expert, feature tile by feature tile, token tile fastest, so that tiles
+// sharing a weight slab or a token tile run side by side.
+struct PlanArgs {
+    int E;                 // routed experts
+    int has_shared;        // 1: append the shared expert over T tokens
+    int T, d, inter;
+    int rows_routed;       // T*k
+    int4* tiles1;          // gate|up tiles
+    int4* tiles2;          // down tiles
+    int* ntiles;           // [0] = gate|up count, [1] = down count
+};
+
+__device__ __forceinline__ void plan_expert(const PlanArgs& p, int g, int c, int row0, int pos1,
+                                            int pos2) {
+    if (c <= 0) return;
+    const bool shared = (g == p.E);
+    const int nt = (c + kMaxN - 1) / kMaxN;
+    const int chunk = pad16((c + nt - 1) / nt);
+    const int ft1 = (p.inter + kSlabRows - 1) / kSlabRows;
+    const int ft2 = (p.d + 2 * kSlabRows - 1) / (2 * kSlabRows);
+    const int map = shared ? 1 : 0;
+    const int e = shared ? 0 : g;
+    const int out_row = shared ? p.rows_routed : row0;
+    const int b_row = shared ? 0 : row0;
+    for (int f = 0; f < ft1; ++f)
+        for (int tt = 0; tt < nt; ++tt) {
+            const int n = min(chunk, c - tt * chunk);
+            const int a0 = e * 2 * p.inter + f * kSlabRows;
+            p.tiles1[2 * pos1] = make_int4(a0, a0 + p.inter, b_row + tt * chunk, n | (map << 16));
+            p.tiles1[2 * pos1 + 1] = make_int4(out_row + tt * chunk, f * kSlabRows, 0, p.d / kBK);
+            ++pos1;
+        }
+    for (int f = 0; f < ft2; ++f)
+        for (int tt = 0; tt < nt; ++tt) {
+            const int n = min(chunk, c - tt * chunk);
+            const int a0 = e * p.d + f * 2 * kSlabRows;
+            // down reads h rows where gate|up wrote them; both B map slots of the
+            // down launch point at h, the slot only picks routed / shared weights
+            p.tiles2[2 * pos2] = make_int4(a0, a0 + kSlabRows, out_row + tt * chunk, n | (map << 16));
+            p.tiles2[2 * pos2 + 1] = make_int4(out_row + tt * chunk, f * 2 * kSlabRows, 0,
+                                               p.inter / kBK);
+            ++pos2;
+        }
+}
+
+__device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, int* n2) {
+    if (c <= 0) {
+        *n1 = *n2 = 0;
+        return;
+    }
+    const int nt = (c + kMaxN - 1) / kMaxN;
+    *n1 = nt * ((p.inter + kSlabRows - 1) / kSlabRows);
+    *n2 = nt * ((p.d + 2 * kSlabRows - 1) / (2 * kSlabRows));
+}
+
+// Plan over experts g = tid and g = tid + 1024 (G <= 2048).  offsets: [E+1].
+__device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) {
+    const int G = p.E + p.has_shared;
+    int c[2], r0[2], n1[2], n2[2];
+    for (int h = 0; h < 2; ++h) {
+        const int g = threadIdx.x + h * 1024;
+        c[h] = 0;
+        r0[h] = 0;
+        if (g < p.E) {
+            r0[h] = offsets[g];
+            c[h] = offsets[g + 1] - offsets[g];
+            // caller-supplied offsets must describe rows inside [0, T*k): a
+            // malformed range gets no tiles (nothing is read or written for it)
+            if (r0[h] < 0 || c[h] < 0 || offsets[g + 1] > p.rows_routed) {
+                record_status(kStatusInvalidArg);
+                c[h] = 0;
+            }
+        } else if (g < G) {
+            c[h] = p.T;
+        }
+        plan_counts(p, c[h], &n1[h], &n2[h]);
+    }
+    int tot1a, tot2a, tot1b, tot2b;
+    const int s1a = block_exclusive_scan(n1[0], &tot1a, scratch);
+    const int s2a = block_exclusive_scan(n2[0], &tot2a, scratch);
+    const int s1b = block_exclusive_scan(n1[1], &tot1b, scratch);
+    const int s2b = block_exclusive_scan(n2[1], &tot2b, scratch);
+    plan_expert(p, threadIdx.x, c[0], r0[0], s1a, s2a);
+    if (threadIdx.x + 1024 < G) plan_expert(p, threadIdx.x + 1024, c[1], r0[1], tot1a + s1b, tot2a + s2b);
+    if (threadIdx.x == 0) {
+        p.ntiles[0] = tot1a + tot1b;
+        p.ntiles[1] = tot2a + tot2b;
+    }
+}
+
+// One block of 1024 threads.  blk_counts [nblk][E] is turned into per-block
+// bases in place.  If plan.tiles1 is set, the GEMM tile lists are built too.
+__global__ void __launch_bounds__(1024) scan_plan_kernel(int* __restrict__ blk_counts, int nblk,
+                                                         int E, int* __restrict__ counts,
+                                                         int* __restrict__ offsets, PlanArgs plan) {
+    __shared__ int scratch[32];
+    __shared__ int s_total[2];
+    int tot[2];
+    for (int h = 0; h < 2; ++h) {
+        const int e = threadIdx.x + h * 1024;
+        int run = 0;
+        if (e < E) {
+            for (int b = 0; b < nblk; ++b) {
+                const int v = blk_counts[(long long)b * E + e];
+                blk_counts[(long long)b * E + e] = run;
+                run += v;
+            }
+        }
+        tot[h] = run;
+    }
+    int sum0, sum1;
+    const int base0 = block_exclusive_scan(tot[0], &sum0, scratch);
+    const int base1 = block_exclusive_scan(tot[1], &sum1, scratch) + sum0;
+    if (threadIdx.x == 0) {
+        s_total[0] = sum0 + sum1;
+    }
+    for (int h = 0; h < 2; ++h) {
+        const int e = threadIdx.x + h * 1024;
+        const int base = h == 0 ? base0 : base1;
+        if (e < E) {
+            counts[e] = tot[h];
+            offsets[e] = base;
+            for (int b = 0; b < nblk; ++b) blk_counts[(long long)b * E + e] += base;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) offsets[E] = s_total[0];
+    if (plan.tiles1 != nullptr) {
+        __syncthreads();
+        __threadfence_block();
+        plan_tiles(plan, offsets, scratch);
+    }
+}
+
+// Tile plan alone, from offsets already in memory (staged expert FFN).
+__global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ offsets, PlanArgs plan) {
+    __shared__ int scratch[32];
+    plan_tiles(plan, offsets, scratch);
+}
+
+__global__ void __launch_bounds__(kPermTokens) permute_scatter_kernel(
+    const int* __restrict__ topk_idx, int T, int E, int k, const int* __restrict__ blk_base,
+    int* __restrict__ row_token, int* __restrict__ slot_row) {
+    extern __shared__ uint32_t sm[];
+    uint32_t* mask = sm;                                  // [4][E]
+    int* wbase = reinterpret_cast<int*>(sm + 4 * E);      // [4][E]
+    for (int i = threadIdx.x; i < 4 * E; i += blockDim.x) mask[i] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * kPermTokens + threadIdx.x;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(long long)t * k + j];
+            if (e >= 0 && e < E) atomicOr(&mask[w * E + e], 1u << lane);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = blk_base[(long long)blockIdx.x * E + e];
+        for (int ww = 0; ww < 4; ++ww) {
+            wbase[ww * E + e] = run;
+            run += __popc(mask[ww * E + e]);
+        }
+    }
+    __syncthreads();
+    if (t < T) {
+        const uint32_t below = (1u << lane) - 1u;
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[(long long)t * k + j];
+            if (e < 0 || e >= E) continue;
+            const int row = wbase[w * E + e] + __popc(mask[w * E + e] & below);
+            row_token[row] = t;
+            slot_row[(long long)t * k + j] = row;
+        }
+    }
+}
+
+// xperm[r, :] = x[row_token[r], :]   (one warp per row, 16-byte vectors)
+__global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict__ x,
+                                                          const int* __restrict__ row_token,
+                                                          int T, int rows, int d,
+                                                          bf16* __restrict__ xperm) {
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const int t = row_token[r];
+    uint4* dst = reinterpret_cast<uint4*>(xperm + (long long)r * d);
+    const int nv = d / 8;
+    if (t < 0 || t >= T) {
+        if (lane == 0) record_status(kStatusInvalidArg);
+        for (int v = lane; v < nv; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * d);
+    int v = lane;
+    for (; v + 96 < nv; v += 128) {
+        const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64),
+                    e = __ldg(src + v + 96);
+        dst[v] = a;
+        dst[v + 32] = b;
+        dst[v + 64] = c;
+        dst[v + 96] = e;
+    }
+    for (; v < nv; v += 32) dst[v] = __ldg(src + v);
+}
+
+}  // namespace moe

@@ -1,0 +1,105 @@
+"""C-ABI host logic without a GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_moe_ffn_sigmoid_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+OK, INVALID, SHAPE = 0, -1, -2
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks fail first
+NULL = None
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(moe.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = moe.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    assert moe.moe_status_string(0) == "MOE_OK"
+    assert moe.moe_status_string(-1) == "MOE_ERR_INVALID_ARG"
+    assert moe.moe_status_string(-2) == "MOE_ERR_UNSUPPORTED_SHAPE"
+    assert moe.moe_status_string(-4) == "MOE_ERR_TIMEOUT"
+    assert moe.moe_status_string(-5) == "MOE_ERR_NO_MEMORY"
+
+
+def _layer(T=64, d=7168, E=384, k=8, inter=2048, scale=2.827, ptrs=None, out=FAKE):
+    p = ptrs if ptrs is not None else [FAKE] * 7
+    return moe.lib().moe_layer_forward(*p, T, d, E, k, inter, ctypes.c_float(scale), out, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=7100), SHAPE), (dict(d=0), SHAPE), (dict(inter=2000), SHAPE), (dict(inter=32), SHAPE),
+    (dict(E=0), SHAPE), (dict(E=1025), SHAPE), (dict(k=0), SHAPE), (dict(k=33, E=64), SHAPE),
+    (dict(k=9, E=8), SHAPE), (dict(T=-1), INVALID), (dict(T=2**30, k=8), SHAPE),
+    (dict(scale=float("nan")), INVALID),
+])
+def test_layer_rejects_bad_shapes(kw, code):
+    assert _layer(**kw) == code
+
+
+def test_layer_rejects_null_and_misaligned_pointers():
+    for i in range(7):
+        p = [FAKE] * 7
+        p[i] = NULL
+        assert _layer(ptrs=p) == INVALID
+        p[i] = ctypes.c_void_p(0x10002)
+        assert _layer(ptrs=p) == INVALID
+    assert _layer(out=NULL) == INVALID
+
+
+def test_zero_tokens_is_a_noop():
+    # nothing is validated against memory and nothing launches for T == 0
+    assert _layer(T=0) == OK
+    L = moe.lib()
+    assert L.moe_route(FAKE, FAKE, FAKE, 0, 512, 32, 4, ctypes.c_float(1.0), FAKE, FAKE, FAKE, 0,
+                       NULL) == OK
+    assert L.moe_permute(FAKE, 0, 32, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 0, NULL) == OK
+    assert L.moe_combine(FAKE, NULL, FAKE, FAKE, 0, 512, 4, FAKE, NULL) == OK
+
+
+def test_staged_calls_check_workspace_size():
+    L = moe.lib()
+    need = moe.moe_workspace_size(64, 512, 32, 4, 128)
+    assert need > 0
+    assert L.moe_route(FAKE, FAKE, FAKE, 64, 512, 32, 4, ctypes.c_float(1.0), FAKE, FAKE, FAKE, 16,
+                       NULL) == INVALID
+    assert L.moe_permute(FAKE, 64, 32, 4, FAKE, FAKE, FAKE, FAKE, FAKE, 4, NULL) == INVALID
+    assert L.moe_expert_ffn(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 512, 32, 4, 128, FAKE, FAKE, need - 1,
+                            NULL) == INVALID
+    assert L.moe_layer_forward_ws(*([FAKE] * 7), 64, 512, 32, 4, 128, ctypes.c_float(2.827), FAKE,
+                                  FAKE, need - 1, NULL) == INVALID
+
+
+def test_workspace_size_grows_with_the_layer():
+    assert moe.moe_workspace_size(64, 512, 32, 4, 128) < moe.moe_workspace_size(128, 512, 32, 4, 128)
+    assert moe.moe_workspace_size(64, 512, 0, 4, 128) == 0       # invalid shape -> 0
+    dec = moe.moe_workspace_size(64, 7168, 384, 8, 2048)
+    pre = moe.moe_workspace_size(8192, 7168, 384, 8, 2048)
+    # prefill scratch: permuted x, h and y dominate (T*k*d + T*(k+1)*(inter+d) bf16)
+    assert pre > 8192 * 8 * 7168 * 2 + 8192 * 9 * (2048 + 7168) * 2
+    assert dec < 64 * 1024 * 1024
+
+
+def test_combine_rejects_bad_shapes():
+    L = moe.lib()
+    assert L.moe_combine(FAKE, NULL, FAKE, FAKE, 4, 12, 4, FAKE, NULL) == SHAPE
+    assert L.moe_combine(FAKE, NULL, FAKE, FAKE, 4, 512, 33, FAKE, NULL) == SHAPE
+    assert L.moe_combine(NULL, NULL, FAKE, FAKE, 4, 512, 4, FAKE, NULL) == INVALID
