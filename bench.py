@@ -228,8 +228,9 @@ def run_oracle_sample(cfg, inputs_dev, n_tokens, seed=0):
 
 
 def default_cpu_sample(cfg):
-    # ~0.8 GFLOP of fp64 per K2 token; one thread per token
-    return min(cfg.T, max(2, host_cores()))
+    # ~0.8 GFLOP of fp64 per K2 token, one thread per token: 64 tokens keep a
+    # 16-core host busy for several seconds without copying every expert
+    return min(cfg.T, max(64, 4 * host_cores()))
 
 
 # --------------------------------------------------------------------- main
