@@ -156,6 +156,45 @@ int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const floa
                          int E, int k, int inter, float scale, uint16_t* out, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Size, in bytes, of the scratch array inside the library that
+ * moe_layer_forward_noalloc works in (32 MiB). */
+#define MOE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * moe_layer_forward for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point: it exists for deployment.
+ *
+ * Some callers must not call cudaMalloc / cudaMallocAsync.  A serving engine
+ * that has reserved nearly all HBM for weights and its KV cache hands its
+ * plugins no allocator.  A latency-critical loop cannot accept the device-wide
+ * synchronisation that cudaMalloc may cause.  A deployment with an audited,
+ * fixed memory plan forbids allocation after start-up.  Such callers pass
+ * only their inputs and outputs (same arguments and layouts as
+ * moe_layer_forward), and the scratch comes from one array of
+ * MOE_NOALLOC_SCRATCH_BYTES compiled into the library.  Every GPU that loads
+ * the library holds that array until the process exits.  This call itself
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ *   - Size limit: if the layer needs more scratch than the array holds
+ *     (moe_workspace_size(T, d, E, k, inter) > MOE_NOALLOC_SCRATCH_BYTES), the
+ *     call returns MOE_ERR_UNSUPPORTED_SHAPE before launching anything.  With
+ *     K2 shapes (d = 7168, E = 384, k = 8, inter = 2048) that allows up to
+ *     T = 97 tokens; decode batches fit, prefill batches do not.
+ *   - First call on a device: it looks up the array's device address with
+ *     cudaGetSymbolAddress, with that device current.  Make that first call
+ *     before any stream capture begins.
+ *   - Sharing: every call on every stream of a device uses the same array, and
+ *     the array keeps the previous call's contents.  No kernel reads scratch it
+ *     has not written earlier in the same call, so nothing needs clearing.
+ *     Calls that overlap on the GPU (different streams, or host threads
+ *     launching at the same time) race on the array and corrupt each other's
+ *     results: order them on one stream or serialise them.
+ */
+int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                              const uint16_t* w_gate_up, const uint16_t* w_down,
+                              const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                              int E, int k, int inter, float scale, uint16_t* out, void* stream);
+
 /*
  * Synchronise `stream`, then read and clear the current device's status word:
  * *device_status = MOE_OK, or the first problem a kernel recorded since the

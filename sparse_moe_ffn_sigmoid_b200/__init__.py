@@ -20,7 +20,7 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_ws",
     "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
-    "EXPORTED_SYMBOLS",
+    "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
@@ -28,10 +28,11 @@ EXPORTED_SYMBOLS = [
     "moe_status_string", "moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_combine", "moe_layer_forward", "moe_layer_forward_ws", "moe_device_status",
     "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
-    "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
+    "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
 ]
 
 MOE_OK = 0
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024    # MOE_NOALLOC_SCRATCH_BYTES in include/moe.h
 
 
 class MoeError(RuntimeError):
@@ -61,6 +62,7 @@ def _load():
         "moe_profile_begin": ([I], I),
         "moe_profile_end": ([ctypes.POINTER(F), I, ctypes.POINTER(I)], I),
         "moe_kernel_name": ([I], ctypes.c_char_p),
+        "moe_layer_forward_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, I, F, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -184,6 +186,17 @@ def moe_layer_forward_ws(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_do
                                    _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                                    _stream(stream))
     _check("moe_layer_forward_ws", rc)
+
+
+def moe_layer_forward_noalloc(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, k: int,
+                              scale: float, out, stream=None):
+    """moe_layer_forward without any device allocation: the scratch is a fixed
+    array inside the library (see include/moe.h for the size limit and the
+    rule that overlapping calls race on it)."""
+    ptrs, T, d, E, inter = _layer_args(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_noalloc(*ptrs, T, d, E, k, inter, float(scale),
+                                        _ptr(out, BF16, "out"), _stream(stream))
+    _check("moe_layer_forward_noalloc", rc)
 
 
 def moe_device_status(stream=None) -> int:

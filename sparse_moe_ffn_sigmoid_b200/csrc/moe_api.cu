@@ -20,6 +20,12 @@
 #include "permute.cuh"
 #include "route.cuh"
 
+// Scratch of moe_layer_forward_noalloc: a fixed array in the library's device
+// image, so that entry point never allocates.  Host code must not use this
+// name as an address (on the host it is only a stand-in); noalloc_scratch()
+// obtains the device address with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_moe_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
 namespace moe {
 namespace {
 
@@ -455,6 +461,27 @@ int owned_workspace(cudaStream_t st, size_t need, void** out) {
     return MOE_OK;
 }
 
+// Device address of g_moe_noalloc_scratch on the current device, looked up on
+// the first call per device (with that device current) and cached.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -594,6 +621,30 @@ int moe_layer_forward(const uint16_t* x, const uint16_t* w_router, const float* 
     if (rc != MOE_OK) return rc;
     return moe_layer_forward_ws(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, T, d, E,
                                 k, inter, scale, out, ws, need, stream);
+}
+
+int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                              const uint16_t* w_gate_up, const uint16_t* w_down,
+                              const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                              int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, w_gate_up, w_down, ws_gate_up, ws_down, out))
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    if (make_layout(T, d, E, k, inter).total > MOE_NOALLOC_SCRATCH_BYTES)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    void* ws = nullptr;
+    rc = noalloc_scratch(&ws);
+    if (rc != MOE_OK) return rc;
+    return layer_forward(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                         bias, reinterpret_cast<const bf16*>(w_gate_up),
+                         reinterpret_cast<const bf16*>(w_down),
+                         reinterpret_cast<const bf16*>(ws_gate_up),
+                         reinterpret_cast<const bf16*>(ws_down), T, d, E, k, inter, scale,
+                         reinterpret_cast<bf16*>(out), ws, MOE_NOALLOC_SCRATCH_BYTES,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int moe_device_status(void* stream, int* device_status) {
