@@ -46,4 +46,8 @@ __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)
 
 __device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// SiLU for the SwiGLU epilogue, with the fast exponential and division
+// intrinsics (the result is rounded to bf16 right after).
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 }  // namespace moe

@@ -12,13 +12,17 @@
 // every weight byte is streamed from HBM once per token tile, and an expert
 // with few tokens (decode) wastes no weight traffic on padding rows.
 //
-// Roles inside a 192-thread CTA (one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer   (one lane): A slab(s) 128x64 + B rows Nx64 per stage
-//   warp 1      MMA issuer     (one lane): 4 x tcgen05.mma (K=16) per slab per stage;
+// Roles inside a 224-thread CTA (one CTA per SM, persistent over tiles):
+//   warp 0      weight producer (one lane): A slab(s) 128 x 64 per K step
+//   warp 6      token producer  (one lane): B rows N x 64 per K step
+//   warp 1      MMA issuer      (one lane): 4 x tcgen05.mma (K=16) per slab per step;
 //               the whole warp allocates / frees the 512 TMEM columns
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, convert, store
-// Stages are guarded by full/empty mbarriers; accumulators (1 or 2 buffers)
-// by acc_full/acc_empty.  Every wait is bounded (see wait_bounded).
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, convert, store
+// Weights come from HBM and tokens mostly from L2, so the two operands have
+// separate rings: a deep one for weights (their HBM latency needs many bytes
+// in flight) and a short one for tokens.  Each ring slot has full/empty
+// mbarriers; accumulators (1 or 2 TMEM buffers) have acc_full/acc_empty.
+// Every wait is bounded (see wait_bounded).
 #pragma once
 
 #include "common.cuh"
@@ -28,9 +32,16 @@ namespace moe {
 constexpr int kBK = 64;                       // K elements per pipeline stage (128 B rows)
 constexpr int kSlabRows = 128;                // MMA M
 constexpr int kSlabBytes = kSlabRows * kBK * 2;
-constexpr int kBoxRows = 16;                  // TMA box height for token rows
-constexpr int kMaxN = 256;                    // MMA N limit
-constexpr int kGemmThreads = 192;
+constexpr int kBoxRows = 16;                  // TMA box height for token rows (tail)
+constexpr int kBoxRowsBig = 64;               // TMA box height for token rows (bulk)
+constexpr int kEpiWarps = 4;
+constexpr int kStageRows = 32;                // epilogue staging block: 32 tokens x 32 features
+constexpr int kStagingBytes = kEpiWarps * kStageRows * 32 * 2;
+constexpr int kMaxN = 256;                    // MMA N limit (router tiles)
+// Token rows per tile of the grouped expert GEMMs.  One tile covers a whole
+// expert up to 256 tokens, so each weight byte is streamed once per expert.
+constexpr int kTileN = 256;
+constexpr int kGemmThreads = 224;
 constexpr int kTmemCols = 512;
 
 enum GemmEpilogue : int {
@@ -49,6 +60,7 @@ struct Tile {
 struct __align__(64) GemmArgs {
     CUtensorMap a_map[2];     // weights: [0] routed (or router), [1] shared expert
     CUtensorMap b_map[2];     // tokens:  [0] permuted rows,       [1] rows in token order
+    CUtensorMap b_map64[2];   // the same token matrices read in 64-row boxes
     const int4* tiles;        // grouped tile list (2 x int4 per tile), or null = dense mode
     const int* ntiles_dev;    // grouped mode: number of tiles (device)
     int ntiles_host;          // dense mode: number of tiles
@@ -59,7 +71,8 @@ struct __align__(64) GemmArgs {
     int col_limit;            // output features >= col_limit are not stored
     int nslab;                // A slabs per tile (1 or 2)
     int n_max;                // largest tile N of the launch (multiple of 16)
-    int stages;
+    int stages_a;             // weight ring depth
+    int stages_b;             // token ring depth
     int acc_bufs;             // accumulator buffers in TMEM (1 or 2)
     int acc_stride;           // TMEM columns per accumulator buffer
     unsigned long long timeout_ns;
@@ -99,17 +112,60 @@ __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int i) {
 
 __device__ __forceinline__ int pad16(int n) { return (n + 15) & ~15; }
 
+// Position in a ring of n slots; the phase bit flips on every wrap.
+struct Ring {
+    uint32_t stage, phase;
+    int n;
+    __device__ __forceinline__ void next() {
+        if (++stage == static_cast<uint32_t>(n)) {
+            stage = 0;
+            phase ^= 1;
+        }
+    }
+};
+
+// Writes one warp's block of an output tile: v[j] is the value of token row
+// (row0 + j) and feature (fbase + lane), j < ncol.  The block goes through the
+// warp's shared staging buffer [32 rows][32 features] so that global memory
+// sees 16-byte stores of 8 consecutive features instead of 2-byte ones.  Rows
+// >= nrows and features >= col_limit are not written.
+__device__ __forceinline__ void store_block_bf16(bf16* stg, const float (&v)[kStageRows], int ncol,
+                                                 bf16* out, long long ld, int row0, int nrows,
+                                                 int fbase, int col_limit, int lane) {
+#pragma unroll
+    for (int j = 0; j < kStageRows; ++j)
+        if (j < ncol) stg[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kStageRows * 4 / 32; ++i) {
+        const int vi = lane + 32 * i;
+        const int r = vi >> 2, part = vi & 3;
+        const int f = fbase + part * 8;
+        if (r < nrows && f < col_limit)
+            *reinterpret_cast<uint4*>(out + (long long)(row0 + r) * ld + f) =
+                *reinterpret_cast<const uint4*>(stg + r * 32 + part * 8);
+    }
+    __syncwarp();
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_constant__ GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    const int S = args.stages;
+    const int SA = args.stages_a;
+    const int SB = args.stages_b;
     const int nslab = args.nslab;
-    const uint32_t stage_bytes = nslab * kSlabBytes + args.n_max * kBK * 2;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
-    uint64_t* empty = full + S;
-    uint64_t* acc_full = empty + S;
+    const uint32_t a_bytes = nslab * kSlabBytes;
+    const uint32_t b_bytes = args.n_max * kBK * 2;
+    uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
+    uint8_t* ring_b = ring_a + SA * a_bytes;                 // [SB][n_max x 64] bf16
+    bf16* staging = reinterpret_cast<bf16*>(ring_b + SB * b_bytes);
+    uint64_t* full_a = reinterpret_cast<uint64_t*>(ring_b + SB * b_bytes + kStagingBytes);
+    uint64_t* empty_a = full_a + SA;
+    uint64_t* full_b = empty_a + SA;
+    uint64_t* empty_b = full_b + SB;
+    uint64_t* acc_full = empty_b + SB;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -119,9 +175,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 1);
+        for (int s = 0; s < SA; ++s) {
+            ptx::mbar_init(&full_a[s], 1);
+            ptx::mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            ptx::mbar_init(&full_b[s], 1);
+            ptx::mbar_init(&empty_b[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
@@ -136,6 +196,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
         ptx::prefetch_tensormap(&args.a_map[1]);
         ptx::prefetch_tensormap(&args.b_map[0]);
         ptx::prefetch_tensormap(&args.b_map[1]);
+        ptx::prefetch_tensormap(&args.b_map64[0]);
+        ptx::prefetch_tensormap(&args.b_map64[1]);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_holder, kTmemCols);
@@ -149,46 +211,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     const int ntiles = args.tiles != nullptr ? *args.ntiles_dev : args.ntiles_host;
     const uint64_t tmo = args.timeout_ns;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == 6) {
+        // ----------------------------------------------------------- producers
         if (lane == 0) {
-            const uint64_t pol_w = ptx::policy_evict_first();   // weights: streamed once
-            const uint64_t pol_x = ptx::policy_evict_last();    // tokens: re-read by tiles
-            uint32_t stage = 0, phase = 0;
-            uint32_t issued = 0, issued_parity = 0;             // per-stage bits, for draining
+            const bool weights = (warp == 0);
+            // weights are streamed once; token rows are re-read by the next tiles
+            const uint64_t pol = weights ? ptx::policy_evict_first() : ptx::policy_evict_last();
+            Ring ring{0, 0, weights ? SA : SB};
+            uint32_t issued = 0, issued_parity = 0;             // per-slot bits, for draining
+            uint64_t* full = weights ? full_a : full_b;
+            uint64_t* empty = weights ? empty_a : empty_b;
             bool ok = true;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
                 const Tile t = load_tile(args, i);
                 const int npad = pad16(t.n);
-                const uint32_t tx = nslab * kSlabBytes + npad * kBK * 2;
-                const CUtensorMap* am = &args.a_map[t.map];
-                const CUtensorMap* bm = &args.b_map[t.map];
+                const uint32_t tx = weights ? a_bytes : npad * kBK * 2;
                 for (int ks = t.ks0; ks < t.ks1; ++ks) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1, abort_flag, tmo)) {
+                    if (!wait_bounded(&empty[ring.stage], ring.phase ^ 1, abort_flag, tmo)) {
                         ok = false;
                         break;
                     }
-                    uint8_t* sa = smem + stage * stage_bytes;
-                    uint8_t* sb = sa + nslab * kSlabBytes;
-                    ptx::mbar_arrive_expect_tx(&full[stage], tx);
-                    ptx::tma_load_2d_hint(sa, am, &full[stage], ks * kBK, t.a_row0, pol_w);
-                    if (nslab == 2)
-                        ptx::tma_load_2d_hint(sa + kSlabBytes, am, &full[stage], ks * kBK,
-                                              t.a_row1, pol_w);
-                    for (int r = 0; r < npad; r += kBoxRows)
-                        ptx::tma_load_2d_hint(sb + r * kBK * 2, bm, &full[stage], ks * kBK,
-                                              t.b_row0 + r, pol_x);
-                    issued |= 1u << stage;
-                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == static_cast<uint32_t>(S)) {
-                        stage = 0;
-                        phase ^= 1;
+                    uint64_t* bar = &full[ring.stage];
+                    ptx::mbar_arrive_expect_tx(bar, tx);
+                    if (weights) {
+                        uint8_t* sa = ring_a + ring.stage * a_bytes;
+                        const CUtensorMap* am = &args.a_map[t.map];
+                        ptx::tma_load_2d_hint(sa, am, bar, ks * kBK, t.a_row0, pol);
+                        if (nslab == 2)
+                            ptx::tma_load_2d_hint(sa + kSlabBytes, am, bar, ks * kBK, t.a_row1, pol);
+                    } else {
+                        uint8_t* sb = ring_b + ring.stage * b_bytes;
+                        int r = 0;
+                        for (; r + kBoxRowsBig <= npad; r += kBoxRowsBig)
+                            ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map64[t.map], bar,
+                                                  ks * kBK, t.b_row0 + r, pol);
+                        for (; r < npad; r += kBoxRows)
+                            ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map[t.map], bar,
+                                                  ks * kBK, t.b_row0 + r, pol);
                     }
+                    issued |= 1u << ring.stage;
+                    issued_parity = (issued_parity & ~(1u << ring.stage)) | (ring.phase << ring.stage);
+                    ring.next();
                 }
             }
             if (!ok) {
                 // let every copy this thread started land before the CTA exits
-                for (int s = 0; s < S; ++s)
+                for (int s = 0; s < ring.n; ++s)
                     if (issued & (1u << s))
                         wait_bounded(&full[s], (issued_parity >> s) & 1, nullptr, tmo);
             }
@@ -196,12 +264,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0, ab = 0, aphase = 0;
+            Ring ra{0, 0, SA}, rb{0, 0, SB};
+            uint32_t ab = 0, aphase = 0;
             bool ok = true, any = false;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
                 const Tile t = load_tile(args, i);
                 const int npad = pad16(t.n);
                 const uint32_t idesc = ptx::idesc_bf16_f32(kSlabRows, npad);
+                // single-slab tiles of 32+ tokens: two N halves (multiples of 16)
+                const int n_lo = (nslab == 1 && npad >= 32) ? pad16(npad / 2) : npad;
+                const int n_hi = npad - n_lo;
+                const uint32_t idesc_lo = ptx::idesc_bf16_f32(kSlabRows, n_lo);
+                const uint32_t idesc_hi = n_hi > 0 ? ptx::idesc_bf16_f32(kSlabRows, n_hi) : idesc;
                 if (!wait_bounded(&acc_empty[ab], aphase ^ 1, abort_flag, tmo)) {
                     ok = false;
                     break;
@@ -209,28 +283,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 ptx::tc_fence_after();
                 const uint32_t dcol = tmem_base + ab * args.acc_stride;
                 for (int ks = t.ks0; ks < t.ks1; ++ks) {
-                    if (!wait_bounded(&full[stage], phase, abort_flag, tmo)) {
+                    if (!wait_bounded(&full_a[ra.stage], ra.phase, abort_flag, tmo) ||
+                        !wait_bounded(&full_b[rb.stage], rb.phase, abort_flag, tmo)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t sa = ptx::smem_u32(smem + stage * stage_bytes);
-                    const uint32_t sb = sa + nslab * kSlabBytes;
-                    for (int s = 0; s < nslab; ++s) {
+                    const uint32_t sa = ptx::smem_u32(ring_a + ra.stage * a_bytes);
+                    const uint32_t sb = ptx::smem_u32(ring_b + rb.stage * b_bytes);
+                    // Consecutive MMAs alternate between two independent accumulators
+                    // (the two slabs, or the two N halves of a single-slab tile): back-
+                    // to-back MMAs into one accumulator wait on each other.  Advancing
+                    // K by 16 elements moves the descriptors' start address by 32 B.
+                    const uint64_t a0 = ptx::sdesc_k_sw128(sa);
+                    const uint64_t a1 = ptx::sdesc_k_sw128(sa + kSlabBytes);
+                    const uint64_t b0 = ptx::sdesc_k_sw128(sb);
+                    const uint64_t b1 = ptx::sdesc_k_sw128(sb + n_lo * kBK * 2);
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk) {
-                            const uint64_t ad = ptx::sdesc_k_sw128(sa + s * kSlabBytes + kk * 32);
-                            const uint64_t bd = ptx::sdesc_k_sw128(sb + kk * 32);
-                            ptx::tc_mma_bf16(dcol + s * args.n_max, ad, bd, idesc,
-                                             (ks > t.ks0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint32_t acc = (ks > t.ks0 || kk > 0) ? 1u : 0u;
+                        if (nslab == 2) {
+                            ptx::tc_mma_bf16(dcol, a0 + 2 * kk, b0 + 2 * kk, idesc, acc);
+                            ptx::tc_mma_bf16(dcol + args.n_max, a1 + 2 * kk, b0 + 2 * kk, idesc, acc);
+                        } else if (n_hi > 0) {
+                            ptx::tc_mma_bf16(dcol, a0 + 2 * kk, b0 + 2 * kk, idesc_lo, acc);
+                            ptx::tc_mma_bf16(dcol + n_lo, a0 + 2 * kk, b1 + 2 * kk, idesc_hi, acc);
+                        } else {
+                            ptx::tc_mma_bf16(dcol, a0 + 2 * kk, b0 + 2 * kk, idesc, acc);
                         }
                     }
                     any = true;
-                    ptx::tc_commit(&empty[stage]);
-                    if (++stage == static_cast<uint32_t>(S)) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+                    ptx::tc_commit(&empty_a[ra.stage]);
+                    ptx::tc_commit(&empty_b[rb.stage]);
+                    ra.next();
+                    rb.next();
                 }
                 if (!ok) break;
                 ptx::tc_commit(&acc_full[ab]);
@@ -248,6 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
+        bf16* stg = staging + (warp - 2) * kStageRows * 32;
         uint32_t ab = 0, aphase = 0;
         for (int i = blockIdx.x; i < ntiles; i += gridDim.x) {
             const Tile t = load_tile(args, i);
@@ -256,45 +343,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
             ptx::tc_fence_after();
             const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 ab * args.acc_stride;
-            if constexpr (EPI == kEpiSwiGLU) {
-                const int f = t.out_col0 + q * 32 + lane;
-                const bool fok = f < args.col_limit;
-                bf16* out = static_cast<bf16*>(args.out) + f;
-                for (int c0 = 0; c0 < npad; c0 += 16) {
-                    uint32_t g[16], u[16];
-                    ptx::tmem_ld_x16(tq + c0, g);
-                    ptx::tmem_ld_x16(tq + args.n_max + c0, u);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int r = c0 + j;
-                        if (r < t.n && fok) {
-                            const float gv = __uint_as_float(g[j]);
-                            const float uv = __uint_as_float(u[j]);
-                            out[(long long)(t.out_row0 + r) * args.out_ld] =
-                                __float2bfloat16_rn(silu_f32(gv) * uv);
-                        }
-                    }
-                }
-            } else if constexpr (EPI == kEpiStoreBF16) {
-                for (int s = 0; s < nslab; ++s) {
-                    const int f = t.out_col0 + s * kSlabRows + q * 32 + lane;
-                    const bool fok = f < args.col_limit;
-                    bf16* out = static_cast<bf16*>(args.out) + f;
-                    for (int c0 = 0; c0 < npad; c0 += 16) {
-                        uint32_t v[16];
-                        ptx::tmem_ld_x16(tq + s * args.n_max + c0, v);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int r = c0 + j;
-                            if (r < t.n && fok)
-                                out[(long long)(t.out_row0 + r) * args.out_ld] =
-                                    __float2bfloat16_rn(__uint_as_float(v[j]));
-                        }
-                    }
-                }
-            } else {
+            if constexpr (EPI == kEpiStoreF32) {
+                // lane = output feature: 32 lanes write 128 contiguous bytes per token
                 const int f = t.out_col0 + q * 32 + lane;
                 const bool fok = f < args.col_limit;
                 float* out = static_cast<float*>(args.out) + f;
@@ -307,6 +357,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                         const int r = c0 + j;
                         if (r < t.n && fok)
                             out[(long long)(t.out_row0 + r) * args.out_ld] = __uint_as_float(v[j]);
+                    }
+                }
+            } else {
+                constexpr bool kSwiGLU = (EPI == kEpiSwiGLU);
+                const int nout = kSwiGLU ? 1 : nslab;
+                bf16* out = static_cast<bf16*>(args.out);
+                for (int s = 0; s < nout; ++s) {
+                    const int fbase = t.out_col0 + s * kSlabRows + q * 32;
+                    const uint32_t ts = tq + s * args.n_max;
+                    for (int c0 = 0; c0 < npad; c0 += kStageRows) {
+                        const int ncol = min(kStageRows, npad - c0);     // 32 or 16 (uniform)
+                        float v[kStageRows];
+                        if constexpr (kSwiGLU) {
+                            uint32_t g[kStageRows], u[kStageRows];
+                            if (ncol == kStageRows) {
+                                ptx::tmem_ld_x32(ts + c0, g);
+                                ptx::tmem_ld_x32(ts + args.n_max + c0, u);
+                            } else {
+                                ptx::tmem_ld_x16(ts + c0, *reinterpret_cast<uint32_t(*)[16]>(g));
+                                ptx::tmem_ld_x16(ts + args.n_max + c0,
+                                                 *reinterpret_cast<uint32_t(*)[16]>(u));
+                            }
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < kStageRows; ++j)
+                                v[j] = silu_fast(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                        } else {
+                            uint32_t r[kStageRows];
+                            if (ncol == kStageRows)
+                                ptx::tmem_ld_x32(ts + c0, r);
+                            else
+                                ptx::tmem_ld_x16(ts + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < kStageRows; ++j) v[j] = __uint_as_float(r[j]);
+                        }
+                        store_block_bf16(stg, v, ncol, out, args.out_ld, t.out_row0 + c0,
+                                         min(ncol, t.n - c0), fbase, args.col_limit, lane);
                     }
                 }
             }
@@ -330,9 +418,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
 }
 
 // Dynamic shared memory the kernel needs for a configuration.
-inline size_t gemm_smem_bytes(int stages, int nslab, int n_max) {
-    const size_t stage = static_cast<size_t>(nslab) * kSlabBytes + static_cast<size_t>(n_max) * kBK * 2;
-    return 1024 /* alignment slack */ + stages * stage + (2 * stages + 5) * 8 + 16;
+inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max) {
+    const size_t a = static_cast<size_t>(nslab) * kSlabBytes;
+    const size_t b = static_cast<size_t>(n_max) * kBK * 2;
+    return 1024 /* alignment slack */ + stages_a * a + stages_b * b + kStagingBytes +
+           (2 * stages_a + 2 * stages_b + 5) * 8 + 16;
 }
 
 }  // namespace moe

@@ -13,7 +13,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "combine.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
@@ -85,16 +85,21 @@ bool all_ok(P... p) {
 
 // ------------------------------------------------------------------ layout
 
+// K splits of the router GEMM: more splits fill more SMs when T is small, but
+// every split adds one fp32 [T, E] partial that is written and read back.
+// Cost model in microseconds: ~0.3 us per 64-deep K step of a tile wave, and
+// the partials at ~4 TB/s.
 int router_splits(int T, int d, int E) {
     const int nt = (T + kMaxN - 1) / kMaxN;
     const int mslabs = (E + kSlabRows - 1) / kSlabRows;
     const int base = std::max(1, nt * mslabs);
     const int ks = d / kBK;
+    const double partial_us = static_cast<double>(T) * E * 8.0 / 4e12 * 1e6;
     int best = 1;
     double best_cost = 1e30;
     for (int s = 1; s <= std::min(ks, kMaxSplits); ++s) {
         const int waves = (base * s + kTargetCtas - 1) / kTargetCtas;
-        const double cost = waves * static_cast<double>((ks + s - 1) / s) + 0.02 * s;
+        const double cost = waves * static_cast<double>((ks + s - 1) / s) * 0.3 + s * partial_us;
         if (cost < best_cost) {
             best_cost = cost;
             best = s;
@@ -117,9 +122,9 @@ Layout make_layout(int T, int d, int E, int k, int inter) {
     const size_t rows = Tk + T;   // routed rows, then the shared expert's rows
     L.splits = router_splits(T, d, E);
     L.nblk = (T + kPermTokens - 1) / kPermTokens;
-    const long long token_tiles = static_cast<long long>(Tk / kMaxN) +
+    const long long token_tiles = static_cast<long long>(Tk / kTileN) +
                                   std::min<long long>(E, static_cast<long long>(Tk)) + 1 +
-                                  (T + kMaxN - 1) / kMaxN;
+                                  (T + kTileN - 1) / kTileN;
     L.max_tiles1 = static_cast<int>(token_tiles * ((inter + kSlabRows - 1) / kSlabRows));
     L.max_tiles2 = static_cast<int>(token_tiles * ((d + 2 * kSlabRows - 1) / (2 * kSlabRows)));
     size_t off = 0;
@@ -217,12 +222,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // ----------------------------------------------------------------- launches
 
+// Ring depths: the token ring gets 3 slots, the weight ring every slot that
+// is left, up to 8 (measured on B200: a 3-slot token ring beat 2 slots on the
+// prefill, skewed and DeepSeek-V3 shapes, and is neutral at decode).
 void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
     a.nslab = nslab;
     a.n_max = n_max;
-    const size_t stage = static_cast<size_t>(nslab) * kSlabBytes + static_cast<size_t>(n_max) * kBK * 2;
-    int stages = static_cast<int>((kMaxDynSmem - 1024 - 256) / stage);
-    a.stages = std::max(2, std::min(stages, 8));
+    const size_t a_bytes = static_cast<size_t>(nslab) * kSlabBytes;
+    const size_t b_bytes = static_cast<size_t>(n_max) * kBK * 2;
+    const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 512;
+    a.stages_b = 3;
+    const int sa = static_cast<int>((budget - a.stages_b * b_bytes) / a_bytes);
+    a.stages_a = std::max(2, std::min(sa, 8));
     a.acc_stride = nslab * n_max;
     a.acc_bufs = (2 * a.acc_stride <= kTmemCols) ? 2 : 1;
     a.timeout_ns = g_timeout_ns.load();
@@ -230,7 +241,7 @@ void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
 
 template <int EPI>
 int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
-    const size_t smem = gemm_smem_bytes(a.stages, a.nslab, a.n_max);
+    const size_t smem = gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max);
     if (smem > kMaxDynSmem) return MOE_ERR_UNSUPPORTED_SHAPE;
     moe_gemm_kernel<EPI><<<grid, kGemmThreads, smem, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -243,10 +254,12 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
     std::memset(&a, 0, sizeof(a));
     const int nt = (T + kMaxN - 1) / kMaxN;
     const int chunk = (((T + nt - 1) / nt) + 15) & ~15;
-    if (!make_map(&a.a_map[0], wr, E, d, kSlabRows) || !make_map(&a.b_map[0], x, T, d, kBoxRows))
+    if (!make_map(&a.a_map[0], wr, E, d, kSlabRows) || !make_map(&a.b_map[0], x, T, d, kBoxRows) ||
+        !make_map(&a.b_map64[0], x, T, d, kBoxRowsBig))
         return MOE_ERR_CUDA;
     a.a_map[1] = a.a_map[0];
     a.b_map[1] = a.b_map[0];
+    a.b_map64[1] = a.b_map64[0];
     a.tiles = nullptr;
     a.dense_mslabs = (E + kSlabRows - 1) / kSlabRows;
     a.dense_ttiles = nt;
@@ -310,14 +323,16 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     }
     // largest token tile: an expert never holds more rows than its token count
     const int max_rows = shared ? T : rows_routed;
-    const int n_max = std::min(kMaxN, (max_rows + 15) & ~15);
+    const int n_max = std::min(kTileN, (max_rows + 15) & ~15);
 
     GemmArgs g1;
     std::memset(&g1, 0, sizeof(g1));
     const bf16* xp = rows_routed > 0 ? xperm : x;
     if (!make_map(&g1.a_map[0], w_gate_up, static_cast<uint64_t>(E) * 2 * inter, d, kSlabRows) ||
         !make_map(&g1.b_map[0], xp, std::max(rows_routed, 1), d, kBoxRows) ||
-        !make_map(&g1.b_map[1], x, T, d, kBoxRows))
+        !make_map(&g1.b_map[1], x, T, d, kBoxRows) ||
+        !make_map(&g1.b_map64[0], xp, std::max(rows_routed, 1), d, kBoxRowsBig) ||
+        !make_map(&g1.b_map64[1], x, T, d, kBoxRowsBig))
         return MOE_ERR_CUDA;
     if (shared) {
         if (!make_map(&g1.a_map[1], ws_gate_up, 2ull * inter, d, kSlabRows)) return MOE_ERR_CUDA;
@@ -337,7 +352,8 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     GemmArgs g2;
     std::memset(&g2, 0, sizeof(g2));
     if (!make_map(&g2.a_map[0], w_down, static_cast<uint64_t>(E) * d, inter, kSlabRows) ||
-        !make_map(&g2.b_map[0], h, rows_all, inter, kBoxRows))
+        !make_map(&g2.b_map[0], h, rows_all, inter, kBoxRows) ||
+        !make_map(&g2.b_map64[0], h, rows_all, inter, kBoxRowsBig))
         return MOE_ERR_CUDA;
     if (shared) {
         if (!make_map(&g2.a_map[1], ws_down, d, inter, kSlabRows)) return MOE_ERR_CUDA;
@@ -345,6 +361,7 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
         g2.a_map[1] = g2.a_map[0];
     }
     g2.b_map[1] = g2.b_map[0];
+    g2.b_map64[1] = g2.b_map64[0];
     g2.tiles = tiles2;
     g2.ntiles_dev = ntiles + 1;
     g2.out = y;

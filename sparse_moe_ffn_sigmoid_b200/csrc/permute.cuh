@@ -76,7 +76,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* scra
 // Tile plan of the grouped SwiGLU FFN.  Expert g (0..G-1) owns rows
 // [row0_g, row0_g + c_g); the shared expert (if present) is g = G-1 and reads
 // its tokens from the unpermuted map.  Each expert's rows are cut into
-// ceil(c/256) token tiles of equal 16-multiple size; tiles are listed expert
+// ceil(c/kTileN) token tiles of equal 16-multiple size; tiles are listed expert
 // by expert, feature tile by feature tile, token tile fastest, so that tiles
 // sharing a weight slab or a token tile run side by side.
 struct PlanArgs {
@@ -93,7 +93,7 @@ __device__ __forceinline__ void plan_expert(const PlanArgs& p, int g, int c, int
                                             int pos2) {
     if (c <= 0) return;
     const bool shared = (g == p.E);
-    const int nt = (c + kMaxN - 1) / kMaxN;
+    const int nt = (c + kTileN - 1) / kTileN;
     const int chunk = pad16((c + nt - 1) / nt);
     const int ft1 = (p.inter + kSlabRows - 1) / kSlabRows;
     const int ft2 = (p.d + 2 * kSlabRows - 1) / (2 * kSlabRows);
@@ -127,7 +127,7 @@ __device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, i
         *n1 = *n2 = 0;
         return;
     }
-    const int nt = (c + kMaxN - 1) / kMaxN;
+    const int nt = (c + kTileN - 1) / kTileN;
     *n1 = nt * ((p.inter + kSlabRows - 1) / kSlabRows);
     *n2 = nt * ((p.d + 2 * kSlabRows - 1) / (2 * kSlabRows));
 }
