@@ -42,6 +42,37 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
     }
 }
 
+// Warp-wide bounded wait for waits that usually last a whole tile: lane 0
+// polls with a short sleep between polls (so the idle warp does not take
+// issue slots from the single MMA-issuing thread on the same scheduler),
+// then the result is shared with the warp.
+__device__ __forceinline__ bool wait_bounded_warp(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag, uint64_t timeout_ns) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) {
+        if (!ptx::mbar_try_wait(bar, parity)) {
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (true) {
+                __nanosleep(256);
+                if (ptx::mbar_try_wait(bar, parity)) break;
+                if (abort_flag && *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+                    if (abort_flag) *abort_flag = 1;
+                    record_status(kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok;
+}
+
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
 __device__ __forceinline__ float sigmoid_f32(float z) { return 1.0f / (1.0f + expf(-z)); }

@@ -20,8 +20,13 @@
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, convert, store
 // Weights come from HBM and tokens mostly from L2, so the two operands have
 // separate rings: a deep one for weights (their HBM latency needs many bytes
-// in flight) and a short one for tokens.  Each ring slot has full/empty
-// mbarriers; accumulators (1 or 2 TMEM buffers) have acc_full/acc_empty.
+// in flight) and a short one for tokens.  K step q uses weight slot q % SA and
+// token slot q % SB (SB <= SA).  The single issuing thread is the bottleneck
+// of the MMA side (each tcgen05.mma, commit and barrier wait costs it tens of
+// cycles), so it sees one barrier per K step: full[q % SA] counts the arrivals
+// of both producers and all their bytes, and one commit to empty[q % SA]
+// releases both slots (the token producer waits on the empty barrier of step
+// q - SB).  Accumulators (1 or 2 TMEM buffers) have acc_full/acc_empty.
 // Every wait is bounded (see wait_bounded).
 #pragma once
 
@@ -161,11 +166,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
     uint8_t* ring_b = ring_a + SA * a_bytes;                 // [SB][n_max x 64] bf16
     bf16* staging = reinterpret_cast<bf16*>(ring_b + SB * b_bytes);
-    uint64_t* full_a = reinterpret_cast<uint64_t*>(ring_b + SB * b_bytes + kStagingBytes);
-    uint64_t* empty_a = full_a + SA;
-    uint64_t* full_b = empty_a + SA;
-    uint64_t* empty_b = full_b + SB;
-    uint64_t* acc_full = empty_b + SB;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring_b + SB * b_bytes + kStagingBytes);
+    uint64_t* empty = full + SA;
+    uint64_t* acc_full = empty + SA;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -176,12 +179,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
-            ptx::mbar_init(&full_a[s], 1);
-            ptx::mbar_init(&empty_a[s], 1);
-        }
-        for (int s = 0; s < SB; ++s) {
-            ptx::mbar_init(&full_b[s], 1);
-            ptx::mbar_init(&empty_b[s], 1);
+            ptx::mbar_init(&full[s], 2);     // weight producer + token producer
+            ptx::mbar_init(&empty[s], 1);    // one commit of the MMA thread
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
@@ -217,30 +216,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
             const bool weights = (warp == 0);
             // weights are streamed once; token rows are re-read by the next tiles
             const uint64_t pol = weights ? ptx::policy_evict_first() : ptx::policy_evict_last();
-            Ring ring{0, 0, weights ? SA : SB};
-            uint32_t issued = 0, issued_parity = 0;             // per-slot bits, for draining
-            uint64_t* full = weights ? full_a : full_b;
-            uint64_t* empty = weights ? empty_a : empty_b;
+            Ring rq{0, 0, SA};          // K step q: its full barrier / weight slot
+            Ring rb{0, 0, SB};          // token slot of step q
+            Ring rp{0, 0, SA};          // step q - SB, whose MMAs free token slot q % SB
+            uint32_t q = 0;
+            uint32_t issued = 0, issued_parity = 0;             // per-barrier bits, for draining
             bool ok = true;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
                 const Tile t = load_tile(args, i);
                 const int npad = pad16(t.n);
                 const uint32_t tx = weights ? a_bytes : npad * kBK * 2;
-                for (int ks = t.ks0; ks < t.ks1; ++ks) {
-                    if (!wait_bounded(&empty[ring.stage], ring.phase ^ 1, abort_flag, tmo)) {
+                for (int ks = t.ks0; ks < t.ks1; ++ks, ++q) {
+                    bool free_ok;
+                    if (weights) {
+                        // weight slot is free once the MMAs of step q - SA are done
+                        free_ok = wait_bounded(&empty[rq.stage], rq.phase ^ 1, abort_flag, tmo);
+                    } else if (q >= static_cast<uint32_t>(SB)) {
+                        free_ok = wait_bounded(&empty[rp.stage], rp.phase, abort_flag, tmo);
+                        rp.next();
+                    } else {
+                        free_ok = true;
+                    }
+                    if (!free_ok) {
                         ok = false;
                         break;
                     }
-                    uint64_t* bar = &full[ring.stage];
+                    uint64_t* bar = &full[rq.stage];
                     ptx::mbar_arrive_expect_tx(bar, tx);
                     if (weights) {
-                        uint8_t* sa = ring_a + ring.stage * a_bytes;
+                        uint8_t* sa = ring_a + rq.stage * a_bytes;
                         const CUtensorMap* am = &args.a_map[t.map];
                         ptx::tma_load_2d_hint(sa, am, bar, ks * kBK, t.a_row0, pol);
                         if (nslab == 2)
                             ptx::tma_load_2d_hint(sa + kSlabBytes, am, bar, ks * kBK, t.a_row1, pol);
                     } else {
-                        uint8_t* sb = ring_b + ring.stage * b_bytes;
+                        uint8_t* sb = ring_b + rb.stage * b_bytes;
                         int r = 0;
                         for (; r + kBoxRowsBig <= npad; r += kBoxRowsBig)
                             ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map64[t.map], bar,
@@ -249,14 +259,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                             ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map[t.map], bar,
                                                   ks * kBK, t.b_row0 + r, pol);
                     }
-                    issued |= 1u << ring.stage;
-                    issued_parity = (issued_parity & ~(1u << ring.stage)) | (ring.phase << ring.stage);
-                    ring.next();
+                    issued |= 1u << rq.stage;
+                    issued_parity = (issued_parity & ~(1u << rq.stage)) | (rq.phase << rq.stage);
+                    rq.next();
+                    rb.next();
                 }
             }
             if (!ok) {
-                // let every copy this thread started land before the CTA exits
-                for (int s = 0; s < ring.n; ++s)
+                // let every copy this thread started land before the CTA exits (a
+                // phase the other producer never joined runs out the bounded wait)
+                for (int s = 0; s < SA; ++s)
                     if (issued & (1u << s))
                         wait_bounded(&full[s], (issued_parity >> s) & 1, nullptr, tmo);
             }
@@ -264,7 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            Ring ra{0, 0, SA}, rb{0, 0, SB};
+            Ring ra{0, 0, SA}, rb{0, 0, SB};   // K step q: weight slot q % SA, token slot q % SB
             uint32_t ab = 0, aphase = 0;
             bool ok = true, any = false;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
@@ -283,8 +295,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 ptx::tc_fence_after();
                 const uint32_t dcol = tmem_base + ab * args.acc_stride;
                 for (int ks = t.ks0; ks < t.ks1; ++ks) {
-                    if (!wait_bounded(&full_a[ra.stage], ra.phase, abort_flag, tmo) ||
-                        !wait_bounded(&full_b[rb.stage], rb.phase, abort_flag, tmo)) {
+                    if (!wait_bounded(&full[ra.stage], ra.phase, abort_flag, tmo)) {
                         ok = false;
                         break;
                     }
@@ -313,8 +324,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                         }
                     }
                     any = true;
-                    ptx::tc_commit(&empty_a[ra.stage]);
-                    ptx::tc_commit(&empty_b[rb.stage]);
+                    ptx::tc_commit(&empty[ra.stage]);
                     ra.next();
                     rb.next();
                 }
@@ -339,7 +349,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
         for (int i = blockIdx.x; i < ntiles; i += gridDim.x) {
             const Tile t = load_tile(args, i);
             const int npad = pad16(t.n);
-            if (!wait_bounded(&acc_full[ab], aphase, abort_flag, tmo)) break;
+            if (!wait_bounded_warp(&acc_full[ab], aphase, abort_flag, tmo)) break;
             ptx::tc_fence_after();
             const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 ab * args.acc_stride;
@@ -422,7 +432,7 @@ inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max) 
     const size_t a = static_cast<size_t>(nslab) * kSlabBytes;
     const size_t b = static_cast<size_t>(n_max) * kBK * 2;
     return 1024 /* alignment slack */ + stages_a * a + stages_b * b + kStagingBytes +
-           (2 * stages_a + 2 * stages_b + 5) * 8 + 16;
+           (2 * stages_a + 5) * 8 + 16;
 }
 
 }  // namespace moe

@@ -233,7 +233,7 @@ void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
     const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 512;
     a.stages_b = 3;
     const int sa = static_cast<int>((budget - a.stages_b * b_bytes) / a_bytes);
-    a.stages_a = std::max(2, std::min(sa, 8));
+    a.stages_a = std::max(a.stages_b, std::min(sa, 8));   // the token ring is never deeper
     a.acc_stride = nslab * n_max;
     a.acc_bufs = (2 * a.acc_stride <= kTmemCols) ? 2 : 1;
     a.timeout_ns = g_timeout_ns.load();
