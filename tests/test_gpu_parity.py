@@ -221,7 +221,8 @@ def test_layer_deterministic_and_ws_variant(moe):
     _status_ok(moe)
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
-    assert moe.moe_last_launch_count() >= 9
+    kernels = [moe.moe_kernel_name(i) for i in range(32) if moe.moe_kernel_name(i)]
+    assert moe.moe_last_launch_count() == len(kernels)
 
 
 def test_staged_calls_compose_to_layer(moe):
