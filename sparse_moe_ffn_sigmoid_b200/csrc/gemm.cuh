@@ -12,12 +12,14 @@
 // every weight byte is streamed from HBM once per token tile, and an expert
 // with few tokens (decode) wastes no weight traffic on padding rows.
 //
-// Roles inside a 224-thread CTA (one CTA per SM, persistent over tiles):
+// Roles inside a 352-thread CTA (one CTA per SM, persistent over tiles):
 //   warp 0      weight producer (one lane): A slab(s) 128 x 64 per K step
-//   warp 6      token producer  (one lane): B rows N x 64 per K step
+//   warp 10     token producer  (one lane): B rows N x 64 per K step
 //   warp 1      MMA issuer      (one lane): 4 x tcgen05.mma (K=16) per slab per step;
 //               the whole warp allocates / frees the 512 TMEM columns
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, convert, store
+//   warps 2..9  epilogue: two warps per TMEM lane quarter, each taking every
+//               other 32-column chunk; tcgen05.ld 32 lanes x 32 columns,
+//               convert, store
 // Weights come from HBM and tokens mostly from L2, so the two operands have
 // separate rings: a deep one for weights (their HBM latency needs many bytes
 // in flight) and a short one for tokens.  K step q uses weight slot q % SA and
@@ -39,14 +41,15 @@ constexpr int kSlabRows = 128;                // MMA M
 constexpr int kSlabBytes = kSlabRows * kBK * 2;
 constexpr int kBoxRows = 16;                  // TMA box height for token rows (tail)
 constexpr int kBoxRowsBig = 64;               // TMA box height for token rows (bulk)
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;                  // two per TMEM lane quarter, splitting the columns
 constexpr int kStageRows = 32;                // epilogue staging block: 32 tokens x 32 features
 constexpr int kStagingBytes = kEpiWarps * kStageRows * 32 * 2;
 constexpr int kMaxN = 256;                    // MMA N limit (router tiles)
 // Token rows per tile of the grouped expert GEMMs.  One tile covers a whole
 // expert up to 256 tokens, so each weight byte is streamed once per expert.
 constexpr int kTileN = 256;
-constexpr int kGemmThreads = 224;
+constexpr int kGemmThreads = 352;             // 11 warps: roles below
+constexpr int kTokenWarp = 10;
 constexpr int kTmemCols = 512;
 
 enum GemmEpilogue : int {
@@ -160,7 +163,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                                                ~static_cast<uintptr_t>(1023));
     const int SA = args.stages_a;
     const int SB = args.stages_b;
-    const int nslab = args.nslab;
+    // the router has one weight slab per tile, the expert GEMMs two (gate|up,
+    // or two 128-row blocks of down); compile-time so the issuing thread
+    // runs no branches on it (the host sets args.nslab to match)
+    constexpr int nslab = (EPI == kEpiStoreF32) ? 1 : 2;
     const uint32_t a_bytes = nslab * kSlabBytes;
     const uint32_t b_bytes = args.n_max * kBK * 2;
     uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
@@ -184,7 +190,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
-            ptx::mbar_init(&acc_empty[b], 4);
+            ptx::mbar_init(&acc_empty[b], kEpiWarps);
         }
         ptx::mbar_init(drain, 1);
         *abort_flag = 0;
@@ -210,7 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     const int ntiles = args.tiles != nullptr ? *args.ntiles_dev : args.ntiles_host;
     const uint64_t tmo = args.timeout_ns;
 
-    if (warp == 0 || warp == 6) {
+    if (warp == 0 || warp == kTokenWarp) {
         // ----------------------------------------------------------- producers
         if (lane == 0) {
             const bool weights = (warp == 0);
@@ -277,6 +283,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             Ring ra{0, 0, SA}, rb{0, 0, SB};   // K step q: weight slot q % SA, token slot q % SB
+            const uint64_t desc_ring_a = ptx::sdesc_k_sw128(ptx::smem_u32(ring_a));
+            const uint64_t desc_ring_b = ptx::sdesc_k_sw128(ptx::smem_u32(ring_b));
             uint32_t ab = 0, aphase = 0;
             bool ok = true, any = false;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
@@ -300,16 +308,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint32_t sa = ptx::smem_u32(ring_a + ra.stage * a_bytes);
-                    const uint32_t sb = ptx::smem_u32(ring_b + rb.stage * b_bytes);
                     // Consecutive MMAs alternate between two independent accumulators
                     // (the two slabs, or the two N halves of a single-slab tile): back-
-                    // to-back MMAs into one accumulator wait on each other.  Advancing
-                    // K by 16 elements moves the descriptors' start address by 32 B.
-                    const uint64_t a0 = ptx::sdesc_k_sw128(sa);
-                    const uint64_t a1 = ptx::sdesc_k_sw128(sa + kSlabBytes);
-                    const uint64_t b0 = ptx::sdesc_k_sw128(sb);
-                    const uint64_t b1 = ptx::sdesc_k_sw128(sb + n_lo * kBK * 2);
+                    // to-back MMAs into one accumulator wait on each other.  The
+                    // descriptors' start-address field holds (address >> 4), so a slot,
+                    // slab or K offset of B bytes is an addition of B >> 4 (K by 16
+                    // elements = 32 B = +2); shared addresses stay below 2^18.
+                    const uint64_t a0 = desc_ring_a + ra.stage * (a_bytes >> 4);
+                    const uint64_t a1 = a0 + (kSlabBytes >> 4);
+                    const uint64_t b0 = desc_ring_b + rb.stage * (b_bytes >> 4);
+                    const uint64_t b1 = b0 + ((n_lo * kBK * 2) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         const uint32_t acc = (ks > t.ks0 || kk > 0) ? 1u : 0u;
@@ -344,6 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;          // which 32-column chunks it takes
         bf16* stg = staging + (warp - 2) * kStageRows * 32;
         uint32_t ab = 0, aphase = 0;
         for (int i = blockIdx.x; i < ntiles; i += gridDim.x) {
@@ -358,7 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 const int f = t.out_col0 + q * 32 + lane;
                 const bool fok = f < args.col_limit;
                 float* out = static_cast<float*>(args.out) + f;
-                for (int c0 = 0; c0 < npad; c0 += 16) {
+                for (int c0 = 16 * half; c0 < npad; c0 += 32) {
                     uint32_t v[16];
                     ptx::tmem_ld_x16(tq + c0, v);
                     ptx::tmem_wait_ld();
@@ -376,7 +385,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 for (int s = 0; s < nout; ++s) {
                     const int fbase = t.out_col0 + s * kSlabRows + q * 32;
                     const uint32_t ts = tq + s * args.n_max;
-                    for (int c0 = 0; c0 < npad; c0 += kStageRows) {
+                    for (int c0 = kStageRows * half; c0 < npad; c0 += 2 * kStageRows) {
                         const int ncol = min(kStageRows, npad - c0);     // 32 or 16 (uniform)
                         float v[kStageRows];
                         if constexpr (kSwiGLU) {

@@ -32,6 +32,7 @@ namespace {
 constexpr int kTargetCtas = 148;          // SMs of a B200: the router's split heuristic
 constexpr int kMaxSplits = 64;
 constexpr size_t kMaxDynSmem = 232448;    // 227 KB opt-in per block on sm_100
+constexpr size_t kScanSmem = 200 * 1024;  // shared memory for the scan's block counts
 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 std::atomic<int> g_last_launches{0};
@@ -176,7 +177,9 @@ int device_info(DeviceInfo* out) {
                                  static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess)
+                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(scan_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kScanSmem)) != cudaSuccess)
             return MOE_ERR_CUDA;
         di.ready = true;
     }
@@ -222,16 +225,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // ----------------------------------------------------------------- launches
 
-// Ring depths: the token ring gets 3 slots, the weight ring every slot that
-// is left, up to 8 (measured on B200: a 3-slot token ring beat 2 slots on the
-// prefill, skewed and DeepSeek-V3 shapes, and is neutral at decode).
+// Ring depths: the token ring gets 3 slots (2 for tiles of <= 64 tokens, whose
+// token rows are small), the weight ring every slot that is left, up to 8
+// (measured on B200: a 3-slot token ring beat 2 slots on the prefill, skewed
+// and DeepSeek-V3 shapes).
 void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
     a.nslab = nslab;
     a.n_max = n_max;
     const size_t a_bytes = static_cast<size_t>(nslab) * kSlabBytes;
     const size_t b_bytes = static_cast<size_t>(n_max) * kBK * 2;
     const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 512;
-    a.stages_b = 3;
+    a.stages_b = n_max <= 64 ? 2 : 3;
     const int sa = static_cast<int>((budget - a.stages_b * b_bytes) / a_bytes);
     a.stages_a = std::max(a.stages_b, std::min(sa, 8));   // the token ring is never deeper
     a.acc_stride = nslab * n_max;
@@ -299,7 +303,11 @@ int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offset
     const int nblk = (T + kPermTokens - 1) / kPermTokens;
     permute_hist_kernel<<<nblk, kPermTokens, 4 * E * sizeof(uint32_t), st>>>(idx, T, E, k, blk);
     rec.mark(st);
-    scan_plan_kernel<<<1, 1024, 0, st>>>(blk, nblk, E, counts, offsets, plan);
+    // block counts are staged in shared memory when they fit (prefill: 98 KB)
+    const long long n = static_cast<long long>(nblk) * E;
+    const int smem_counts = n * 4 <= static_cast<long long>(kScanSmem) ? static_cast<int>(n) : 0;
+    scan_plan_kernel<<<1, 1024, smem_counts * 4, st>>>(blk, nblk, E, counts, offsets, plan,
+                                                     smem_counts);
     rec.mark(st);
     permute_scatter_kernel<<<nblk, kPermTokens, 8 * E * sizeof(uint32_t), st>>>(
         idx, T, E, k, blk, row_token, slot_row);
@@ -553,6 +561,9 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
         return MOE_ERR_INVALID_ARG;
     const int nblk = (T + kPermTokens - 1) / kPermTokens;
     if (workspace_bytes < static_cast<size_t>(nblk) * E * sizeof(int)) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;                  // sets the kernels' shared-memory limits on first use
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
     PlanArgs none{};
     Recorder rec;
     return launch_permute(topk_idx, T, E, k, counts, offsets, row_token, slot_row,

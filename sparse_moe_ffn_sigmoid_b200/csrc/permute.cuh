@@ -169,19 +169,30 @@ __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) 
 
 // One block of 1024 threads.  blk_counts [nblk][E] is turned into per-block
 // bases in place.  If plan.tiles1 is set, the GEMM tile lists are built too.
+// When nblk * E counts fit the dynamic shared memory the launch provides
+// (smem_counts), the per-expert scans over blocks run out of shared memory.
 __global__ void __launch_bounds__(1024) scan_plan_kernel(int* __restrict__ blk_counts, int nblk,
                                                          int E, int* __restrict__ counts,
-                                                         int* __restrict__ offsets, PlanArgs plan) {
+                                                         int* __restrict__ offsets, PlanArgs plan,
+                                                         int smem_counts) {
+    extern __shared__ int sc[];
     __shared__ int scratch[32];
     __shared__ int s_total[2];
+    const long long n = static_cast<long long>(nblk) * E;
+    const bool staged = n <= smem_counts;
+    int* cnt = staged ? sc : blk_counts;
+    if (staged) {
+        for (long long i = threadIdx.x; i < n; i += blockDim.x) sc[i] = blk_counts[i];
+        __syncthreads();
+    }
     int tot[2];
     for (int h = 0; h < 2; ++h) {
         const int e = threadIdx.x + h * 1024;
         int run = 0;
         if (e < E) {
             for (int b = 0; b < nblk; ++b) {
-                const int v = blk_counts[(long long)b * E + e];
-                blk_counts[(long long)b * E + e] = run;
+                const int v = cnt[(long long)b * E + e];
+                cnt[(long long)b * E + e] = run;
                 run += v;
             }
         }
@@ -199,14 +210,15 @@ __global__ void __launch_bounds__(1024) scan_plan_kernel(int* __restrict__ blk_c
         if (e < E) {
             counts[e] = tot[h];
             offsets[e] = base;
-            for (int b = 0; b < nblk; ++b) blk_counts[(long long)b * E + e] += base;
+            for (int b = 0; b < nblk; ++b) cnt[(long long)b * E + e] += base;
         }
     }
     __syncthreads();
+    if (staged)
+        for (long long i = threadIdx.x; i < n; i += blockDim.x) blk_counts[i] = sc[i];
     if (threadIdx.x == 0) offsets[E] = s_total[0];
     if (plan.tiles1 != nullptr) {
         __syncthreads();
-        __threadfence_block();
         plan_tiles(plan, offsets, scratch);
     }
 }
