@@ -36,7 +36,10 @@ sys.path.insert(0, ROOT)
 METRIC = "K2 MoE-layer tokens/s; % of HBM (decode) / bf16 tensor (prefill) roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DEFAULT_STEPS = {"k2_decode": 400, "tiny": 400, "v3": 100, "k2_skew": 100, "k2_prefill": 60}
+# timed steps per workload: the device-timed region stays near a second (for
+# the clock samples) and the oracle reference arm (about a second per step on
+# a K2 token) within a few minutes
+DEFAULT_STEPS = {"k2_decode": 150, "tiny": 200, "v3": 100, "k2_skew": 100, "k2_prefill": 60}
 
 
 def parse_args(argv=None):
@@ -173,6 +176,24 @@ def profiled_traffic(workload: str, kernel: str):
     return None
 
 
+# ----------------------------------------------------------- multi-rank
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest per-rank value over all ranks (the slowest rank's time)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_total: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_total / 1e3)
+
+
 # ----------------------------------------------------- accounting (per step)
 
 def layer_accounting(cfg, touched: int):
@@ -198,36 +219,47 @@ def layer_accounting(cfg, touched: int):
 
 # ------------------------------------------------------------------- oracle
 
-def run_oracle_sample(cfg, inputs_dev, n_tokens, seed=0):
-    """Oracle (routing + experts) on n_tokens evenly spread tokens; returns
-    (seconds, threads, description)."""
-    import numpy as np
-    import oracle
-    T = cfg.T
-    n = max(1, min(n_tokens, T))
-    tok = sorted(set(int(round(i * (T - 1) / max(n - 1, 1))) for i in range(n)))
-    import torch
-    sel = torch.tensor(tok, device=inputs_dev["x"].device)
-    x_s = inputs_dev["x"].index_select(0, sel).cpu()
-    wr = inputs_dev["w_router"].cpu()
-    bias = inputs_dev["bias"].cpu()
-    threads = min(host_cores(), len(tok))
-    # routing of the sampled rows (a row's routing depends on that row only)
-    ridx, rw, _ = oracle.route(x_s, wr, bias, cfg.k, cfg.scale, nthreads=threads)
-    need = sorted(set(ridx.reshape(-1).tolist()))
-    egu = [None] * cfg.E
-    edn = [None] * cfg.E
-    for e in need:
-        egu[e] = inputs_dev["w_gate_up"][e].cpu()
-        edn[e] = inputs_dev["w_down"][e].cpu()
-    sgu, sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
-    t0 = time.perf_counter()
-    ridx, rw, _ = oracle.route(x_s, wr, bias, cfg.k, cfg.scale, nthreads=threads)
-    oracle.moe_rows(x_s, ridx, rw, egu, edn, sgu, sdn, nthreads=threads)
-    dt = time.perf_counter() - t0
-    desc = (f"{len(tok)} of {T} tokens (evenly spaced), full routing + {len(need)} routed "
-            f"experts + shared expert, fp64")
-    return dt, threads, len(tok), desc
+class OracleSample:
+    """A fixed, evenly spaced token sample of the workload with everything the
+    oracle needs copied to the host once (x rows, router, the experts those
+    tokens select, the shared expert).  Rows are independent, so the oracle's
+    tokens/s on the sample is its rate on the workload."""
+
+    def __init__(self, cfg, inputs_dev, n_tokens):
+        import torch
+        import oracle
+        self.cfg = cfg
+        T = cfg.T
+        n = max(1, min(n_tokens, T))
+        self.tokens = sorted(set(int(round(i * (T - 1) / max(n - 1, 1))) for i in range(n)))
+        sel = torch.tensor(self.tokens, device=inputs_dev["x"].device)
+        self.x = inputs_dev["x"].index_select(0, sel).cpu()
+        self.wr = inputs_dev["w_router"].cpu()
+        self.bias = inputs_dev["bias"].cpu()
+        self.threads = min(host_cores(), len(self.tokens))
+        # routing of a row depends on that row only
+        ridx, _, _ = oracle.route(self.x, self.wr, self.bias, cfg.k, cfg.scale, nthreads=self.threads)
+        self.need = sorted(set(ridx.reshape(-1).tolist()))
+        self.egu = [None] * cfg.E
+        self.edn = [None] * cfg.E
+        for e in self.need:
+            self.egu[e] = inputs_dev["w_gate_up"][e].cpu()
+            self.edn[e] = inputs_dev["w_down"][e].cpu()
+        self.sgu, self.sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
+
+    def run(self) -> float:
+        """Seconds for the oracle's full layer (routing + experts) on the sample."""
+        import oracle
+        t0 = time.perf_counter()
+        ridx, rw, _ = oracle.route(self.x, self.wr, self.bias, self.cfg.k, self.cfg.scale,
+                                   nthreads=self.threads)
+        oracle.moe_rows(self.x, ridx, rw, self.egu, self.edn, self.sgu, self.sdn,
+                        nthreads=self.threads)
+        return time.perf_counter() - t0
+
+    def describe(self) -> str:
+        return (f"{len(self.tokens)} of {self.cfg.T} tokens (evenly spaced), full routing + "
+                f"{len(self.need)} routed experts + shared expert, fp64")
 
 
 def default_cpu_sample(cfg):
@@ -322,12 +354,9 @@ def main(argv=None):
     if moe.moe_device_status() != 0:
         raise SystemExit("device status not clean after the timed region")
     clocks = clk.summary(t_wall0, t_wall1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1e3)
+    value = job_throughput(world, T, args.steps, ms_total)
 
     # ---------------------------------------------------------- end to end
     e2e = None
@@ -353,12 +382,8 @@ def main(argv=None):
             e2e_step()
         e2.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * T * args.steps / (ms_e2e / 1e3), "unit": UNIT,
+        ms_e2e = max_over_ranks(s2.elapsed_time(e2), world, dev)
+        e2e = {"value": job_throughput(world, T, args.steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
                "ms_per_step": ms_e2e / args.steps}
 
@@ -397,10 +422,10 @@ def main(argv=None):
     # ---------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = args.cpu_sample or default_cpu_sample(cfg)
-        dt, threads, nt, desc = run_oracle_sample(cfg, g, n)
-        cpu = {"value": nt / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc, "seconds": dt}
+        smp = OracleSample(cfg, g, args.cpu_sample or default_cpu_sample(cfg))
+        dt = smp.run()
+        cpu = {"value": len(smp.tokens) / dt, "unit": UNIT, "cores": smp.threads,
+               "kind": "oracle", "sample": smp.describe(), "seconds": dt}
 
     if rank == 0:
         line = {
@@ -423,22 +448,35 @@ def main(argv=None):
     return 0
 
 
+REFERENCE_BUDGET_S = 60.0      # target oracle seconds for all warm-up + timed steps
+
+
 def run_reference(args, cfg, world):
-    """The oracle on the host cores, --warmup + --steps bounded samples."""
+    """The fp64 oracle on the host cores: --warmup + --steps runs of one fixed
+    token sample.  The oracle runs one thread per token, so a run takes at
+    least one token's time; the sample is a whole number of waves of host
+    threads, as many as REFERENCE_BUDGET_S allows (at least one)."""
     import torch
     from moe_inputs import make_inputs
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     g = make_inputs(cfg, seed=0, device=dev)
-    n = args.cpu_sample or max(2, min(cfg.T, host_cores()))
-    # each step a bounded sample so the whole run stays within minutes
+    runs = args.warmup + args.steps
+    if args.cpu_sample:
+        n = args.cpu_sample
+    else:
+        probe = OracleSample(cfg, g, 1)        # one token measures the per-token cost
+        per_token = probe.run()
+        waves = max(1, int(REFERENCE_BUDGET_S / runs / per_token))
+        n = max(1, min(cfg.T, waves * host_cores()))
+    smp = OracleSample(cfg, g, n)
+    del g
     per_step = []
-    threads, nt, desc = 1, n, ""
-    for i in range(args.warmup + args.steps):
-        dt, threads, nt, desc = run_oracle_sample(cfg, g, n)
+    for i in range(runs):
+        dt = smp.run()
         if i >= args.warmup:
             per_step.append(dt)
     total = sum(per_step)
-    value = nt * len(per_step) / total
+    value = len(smp.tokens) * len(per_step) / total
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / len(per_step),
@@ -446,8 +484,8 @@ def run_reference(args, cfg, world):
         "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "inter": cfg.inter, "scale": cfg.scale, "bias": cfg.bias},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.threads, "kind": "oracle",
+                         "sample": smp.describe()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
