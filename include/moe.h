@@ -104,7 +104,9 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
  *   y         [T*k, d]      bf16   out, in row (permuted) order
  * bf16 x bf16 -> fp32 on tcgen05 tensor cores; the intermediate
  * silu(gate) * up is rounded to bf16.  The shared expert is the case E = 1,
- * k = 1, row_token = 0..T-1, offsets = {0, T}.
+ * k = 1, row_token = 0..T-1, offsets = {0, T}.  A row_token entry outside
+ * [0, T) is not read: it is recorded as MOE_ERR_INVALID_ARG in the device
+ * status, that row of y is unspecified, and every other row is unaffected.
  */
 int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* offsets,
                    const uint16_t* w_gate_up, const uint16_t* w_down, int T, int d, int E, int k,

@@ -88,8 +88,9 @@ bool all_ok(P... p) {
 
 // K splits of the router GEMM: more splits fill more SMs when T is small, but
 // every split adds one fp32 [T, E] partial that is written and read back.
-// Cost model in microseconds: ~0.3 us per 64-deep K step of a tile wave, and
-// the partials at ~4 TB/s.
+// Cost model in microseconds: ~0.9 us per 64-deep K step of a tile wave (the
+// measured pace of a single-slab router tile on B200), and the partials at
+// ~4 TB/s.
 int router_splits(int T, int d, int E) {
     const int nt = (T + kMaxN - 1) / kMaxN;
     const int mslabs = (E + kSlabRows - 1) / kSlabRows;
@@ -100,7 +101,7 @@ int router_splits(int T, int d, int E) {
     double best_cost = 1e30;
     for (int s = 1; s <= std::min(ks, kMaxSplits); ++s) {
         const int waves = (base * s + kTargetCtas - 1) / kTargetCtas;
-        const double cost = waves * static_cast<double>((ks + s - 1) / s) * 0.3 + s * partial_us;
+        const double cost = waves * static_cast<double>((ks + s - 1) / s) * 0.9 + s * partial_us;
         if (cost < best_cost) {
             best_cost = cost;
             best = s;

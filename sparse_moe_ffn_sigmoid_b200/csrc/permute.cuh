@@ -89,37 +89,34 @@ struct PlanArgs {
     int* ntiles;           // [0] = gate|up count, [1] = down count
 };
 
-__device__ __forceinline__ void plan_expert(const PlanArgs& p, int g, int c, int row0, int pos1,
-                                            int pos2) {
-    if (c <= 0) return;
+constexpr int kPlanMaxG = 1025;   // up to 1024 routed experts and the shared one
+
+// Writes tile `local` of expert g (c rows from row0): gate|up tiles (down =
+// false) or down tiles, at list position pos.  Within an expert the tiles run
+// feature tile by feature tile, token tile fastest: local = f * nt + tt.
+__device__ __forceinline__ void plan_tile(const PlanArgs& p, int g, int c, int row0, int local,
+                                          bool down, int pos) {
     const bool shared = (g == p.E);
     const int nt = (c + kTileN - 1) / kTileN;
     const int chunk = pad16((c + nt - 1) / nt);
-    const int ft1 = (p.inter + kSlabRows - 1) / kSlabRows;
-    const int ft2 = (p.d + 2 * kSlabRows - 1) / (2 * kSlabRows);
+    const int f = local / nt;
+    const int tt = local - f * nt;
+    const int n = min(chunk, c - tt * chunk);
     const int map = shared ? 1 : 0;
     const int e = shared ? 0 : g;
-    const int out_row = shared ? p.rows_routed : row0;
-    const int b_row = shared ? 0 : row0;
-    for (int f = 0; f < ft1; ++f)
-        for (int tt = 0; tt < nt; ++tt) {
-            const int n = min(chunk, c - tt * chunk);
-            const int a0 = e * 2 * p.inter + f * kSlabRows;
-            p.tiles1[2 * pos1] = make_int4(a0, a0 + p.inter, b_row + tt * chunk, n | (map << 16));
-            p.tiles1[2 * pos1 + 1] = make_int4(out_row + tt * chunk, f * kSlabRows, 0, p.d / kBK);
-            ++pos1;
-        }
-    for (int f = 0; f < ft2; ++f)
-        for (int tt = 0; tt < nt; ++tt) {
-            const int n = min(chunk, c - tt * chunk);
-            const int a0 = e * p.d + f * 2 * kSlabRows;
-            // down reads h rows where gate|up wrote them; both B map slots of the
-            // down launch point at h, the slot only picks routed / shared weights
-            p.tiles2[2 * pos2] = make_int4(a0, a0 + kSlabRows, out_row + tt * chunk, n | (map << 16));
-            p.tiles2[2 * pos2 + 1] = make_int4(out_row + tt * chunk, f * 2 * kSlabRows, 0,
-                                               p.inter / kBK);
-            ++pos2;
-        }
+    const int out_row = (shared ? p.rows_routed : row0) + tt * chunk;
+    const int b_row = (shared ? 0 : row0) + tt * chunk;
+    if (!down) {
+        const int a0 = e * 2 * p.inter + f * kSlabRows;
+        p.tiles1[2 * pos] = make_int4(a0, a0 + p.inter, b_row, n | (map << 16));
+        p.tiles1[2 * pos + 1] = make_int4(out_row, f * kSlabRows, 0, p.d / kBK);
+    } else {
+        const int a0 = e * p.d + f * 2 * kSlabRows;
+        // down reads h rows where gate|up wrote them; both B map slots of the
+        // down launch point at h, the slot only picks routed / shared weights
+        p.tiles2[2 * pos] = make_int4(a0, a0 + kSlabRows, out_row, n | (map << 16));
+        p.tiles2[2 * pos + 1] = make_int4(out_row, f * 2 * kSlabRows, 0, p.inter / kBK);
+    }
 }
 
 __device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, int* n2) {
@@ -132,8 +129,26 @@ __device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, i
     *n2 = nt * ((p.d + 2 * kSlabRows - 1) / (2 * kSlabRows));
 }
 
-// Plan over experts g = tid and g = tid + 1024 (G <= 2048).  offsets: [E+1].
+// Largest g in [0, n) with first[g] <= i, given first[0] == 0 <= i and first
+// non-decreasing: the expert that owns list position i (an expert with no
+// tiles shares its first position with the next one and is skipped).
+__device__ __forceinline__ int owner_of(const int* first, int n, int i) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (first[mid] <= i)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Plan over experts g = tid and g = tid + 1024 (G <= kPlanMaxG).  offsets: [E+1].
+// Tile counts per expert are scanned into first positions; then the whole
+// block writes the lists, consecutive threads taking consecutive tiles.
 __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) {
+    __shared__ int s_c[kPlanMaxG], s_row0[kPlanMaxG], s_first1[kPlanMaxG], s_first2[kPlanMaxG];
     const int G = p.E + p.has_shared;
     int c[2], r0[2], n1[2], n2[2];
     for (int h = 0; h < 2; ++h) {
@@ -159,11 +174,30 @@ __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) 
     const int s2a = block_exclusive_scan(n2[0], &tot2a, scratch);
     const int s1b = block_exclusive_scan(n1[1], &tot1b, scratch);
     const int s2b = block_exclusive_scan(n2[1], &tot2b, scratch);
-    plan_expert(p, threadIdx.x, c[0], r0[0], s1a, s2a);
-    if (threadIdx.x + 1024 < G) plan_expert(p, threadIdx.x + 1024, c[1], r0[1], tot1a + s1b, tot2a + s2b);
+    const int first1[2] = {s1a, tot1a + s1b};
+    const int first2[2] = {s2a, tot2a + s2b};
+    for (int h = 0; h < 2; ++h) {
+        const int g = threadIdx.x + h * 1024;
+        if (g < G) {
+            s_c[g] = c[h];
+            s_row0[g] = r0[h];
+            s_first1[g] = first1[h];
+            s_first2[g] = first2[h];
+        }
+    }
+    const int tot1 = tot1a + tot1b, tot2 = tot2a + tot2b;
     if (threadIdx.x == 0) {
-        p.ntiles[0] = tot1a + tot1b;
-        p.ntiles[1] = tot2a + tot2b;
+        p.ntiles[0] = tot1;
+        p.ntiles[1] = tot2;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < tot1; i += blockDim.x) {
+        const int g = owner_of(s_first1, G, i);
+        plan_tile(p, g, s_c[g], s_row0[g], i - s_first1[g], false, i);
+    }
+    for (int i = threadIdx.x; i < tot2; i += blockDim.x) {
+        const int g = owner_of(s_first2, G, i);
+        plan_tile(p, g, s_c[g], s_row0[g], i - s_first2[g], true, i);
     }
 }
 

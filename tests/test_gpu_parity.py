@@ -178,6 +178,28 @@ def test_expert_ffn_parity(moe, cfg):
     PR.check_output(PR.bf16_np(y), ref)
 
 
+def test_expert_ffn_bad_row_token(moe):
+    """Out-of-range token indices are reported and skipped; other rows are exact."""
+    cfg = MoEConfig("bad_rows", T=40, d=256, E=4, k=2, inter=128, scale=1.0)
+    inp = make_inputs(cfg, seed=21)
+    idx = make_topk_idx(cfg.T, cfg.E, cfg.k, seed=22)
+    counts, offsets, row_token, _ = oracle.permute(idx.numpy(), cfg.E)
+    bad = row_token.copy()
+    bad_rows = [3, 41, 70]
+    bad[3], bad[41], bad[70] = cfg.T, -1, 1 << 30
+    g = _cuda(inp)
+    y = torch.empty((cfg.T * cfg.k, cfg.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(g["x"], torch.from_numpy(bad).cuda(), torch.from_numpy(offsets).cuda(),
+                       g["w_gate_up"], g["w_down"], cfg.k, y,
+                       _ws(moe, cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter))
+    assert moe.moe_device_status() == -1          # MOE_ERR_INVALID_ARG
+    expert_of_row = np.repeat(np.arange(cfg.E), counts)
+    keep = [r for r in range(cfg.T * cfg.k) if r not in bad_rows]
+    ref = np.stack([oracle.swiglu_row(inp["x"][row_token[r]], inp["w_gate_up"][expert_of_row[r]],
+                                      inp["w_down"][expert_of_row[r]]) for r in keep])
+    PR.check_output(PR.bf16_np(y)[keep], ref)
+
+
 # -------------------------------------------------------------------- layer
 
 LAYER_CASES = [
