@@ -12,6 +12,8 @@
 
 namespace moe {
 
+constexpr int kCombineThreads = 128;
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -30,20 +32,22 @@ __device__ __forceinline__ uint4 f32_to_bf16x8(const float (&f)[8]) {
     return v;
 }
 
-// One block per token; threads stride over 8-element vectors of the row.
-__global__ void __launch_bounds__(128) combine_kernel(const bf16* __restrict__ y,
-                                                      const bf16* __restrict__ y_shared,
-                                                      const float* __restrict__ topk_w,
-                                                      const int* __restrict__ slot_row, int T,
-                                                      int d, int k, long long y_rows,
-                                                      bf16* __restrict__ out) {
+// Block (t, c) combines the 8-element vectors v = c * blockDim.x + threadIdx.x
+// (+ gridDim.y * blockDim.x ...) of token t's row.  Each thread issues the
+// loads of up to 8 routed rows before it accumulates them (in slot order), so
+// it waits on memory once per 8 rows; at small T the row is split over
+// several blocks (gridDim.y > 1) to keep enough loads in flight.
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const bf16* __restrict__ y, const bf16* __restrict__ y_shared, const float* __restrict__ topk_w,
+    const int* __restrict__ slot_row, int T, int d, int k, long long y_rows,
+    bf16* __restrict__ out) {
     __shared__ int s_row[32];
     __shared__ float s_w[32];
     const int t = blockIdx.x;
     if (threadIdx.x < k) {
         int r = slot_row[(long long)t * k + threadIdx.x];
         if (r < 0 || r >= y_rows) {
-            record_status(kStatusInvalidArg);
+            if (blockIdx.y == 0) record_status(kStatusInvalidArg);
             r = -1;
         }
         s_row[threadIdx.x] = r;
@@ -51,22 +55,33 @@ __global__ void __launch_bounds__(128) combine_kernel(const bf16* __restrict__ y
     }
     __syncthreads();
     const int nv = d / 8;
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nv; v += gridDim.y * blockDim.x) {
         float acc[8];
         if (y_shared != nullptr) {
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(y_shared + (long long)t * d) + v), acc);
+            const uint4* ys = reinterpret_cast<const uint4*>(y_shared + (long long)t * d);
+            bf16x8_to_f32(__ldg(ys + v), acc);
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
         }
-        for (int j = 0; j < k; ++j) {
-            const int r = s_row[j];
-            if (r < 0) continue;
-            float f[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(y + (long long)r * d) + v), f);
-            const float wj = s_w[j];
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 raw[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+            for (int u = 0; u < 8; ++u) {
+                const int r = (j0 + u < k) ? s_row[j0 + u] : -1;
+                raw[u] = r >= 0 ? __ldg(reinterpret_cast<const uint4*>(y + (long long)r * d) + v)
+                                : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u;
+                if (j >= k || s_row[j] < 0) continue;
+                float f[8];
+                bf16x8_to_f32(raw[u], f);
+                const float wj = s_w[j];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+            }
         }
         reinterpret_cast<uint4*>(out + (long long)t * d)[v] = f32_to_bf16x8(acc);
     }

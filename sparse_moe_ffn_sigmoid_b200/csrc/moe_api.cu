@@ -33,6 +33,7 @@ constexpr int kTargetCtas = 148;          // SMs of a B200: the router's split h
 constexpr int kMaxSplits = 64;
 constexpr size_t kMaxDynSmem = 232448;    // 227 KB opt-in per block on sm_100
 constexpr size_t kScanSmem = 200 * 1024;  // shared memory for the scan's block counts
+constexpr int kTopkBlockTokens = 512;      // top-k launch shape switch (tokens per call)
 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 std::atomic<int> g_last_launches{0};
@@ -281,11 +282,19 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
     if (rc != MOE_OK) return rc;
     rec.mark(st);
     const int npl = (E + 31) / 32;
-    const dim3 grid((T + 7) / 8), block(256);
     const long long sstride = static_cast<long long>(T) * E;
-#define MOE_TOPK(N)                                                                          \
-    topk_kernel<N><<<grid, block, 0, st>>>(partials, splits, sstride, T, E, k, bias, scale, idx, \
-                                           w)
+    // a block per token while the batch is small (the partial sums then wait
+    // on memory, not on selection throughput); a warp per token otherwise
+    const bool per_block = T <= kTopkBlockTokens;
+#define MOE_TOPK(N)                                                                              \
+    do {                                                                                         \
+        if (per_block)                                                                           \
+            topk_block_kernel<N><<<T, 32 * (N), 0, st>>>(partials, splits, sstride, T, E, k,     \
+                                                         bias, scale, idx, w);                   \
+        else                                                                                     \
+            topk_warp_kernel<N><<<(T + 7) / 8, 256, 0, st>>>(partials, splits, sstride, T, E, k, \
+                                                             bias, scale, idx, w);               \
+    } while (0)
     if (npl <= 1) MOE_TOPK(1);
     else if (npl <= 2) MOE_TOPK(2);
     else if (npl <= 4) MOE_TOPK(4);
@@ -385,8 +394,11 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
 
 int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* slot_row, int T,
                    int d, int k, bf16* out, cudaStream_t st, Recorder& rec) {
-    combine_kernel<<<T, 128, 0, st>>>(y, ysh, w, slot_row, T, d, k,
-                                      static_cast<long long>(T) * k, out);
+    // split each row over several blocks only while the batch is small
+    const int chunks = (d / 8 + kCombineThreads - 1) / kCombineThreads;
+    const dim3 grid(T, std::max(1, std::min(chunks, (2048 + T - 1) / T)));
+    combine_kernel<<<grid, kCombineThreads, 0, st>>>(y, ysh, w, slot_row, T, d, k,
+                                                     static_cast<long long>(T) * k, out);
     rec.mark(st);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -91,15 +91,14 @@ struct PlanArgs {
 
 constexpr int kPlanMaxG = 1025;   // up to 1024 routed experts and the shared one
 
-// Writes tile `local` of expert g (c rows from row0): gate|up tiles (down =
-// false) or down tiles, at list position pos.  Within an expert the tiles run
-// feature tile by feature tile, token tile fastest: local = f * nt + tt.
-__device__ __forceinline__ void plan_tile(const PlanArgs& p, int g, int c, int row0, int local,
-                                          bool down, int pos) {
+// Writes tile `local` of expert g (c rows from row0, cut into nt token tiles
+// of `chunk` rows): gate|up tiles (down = false) or down tiles, at list
+// position pos.  Within an expert the tiles run feature tile by feature tile,
+// token tile fastest: local = f * nt + tt.
+__device__ __forceinline__ void plan_tile(const PlanArgs& p, int g, int c, int row0, int nt,
+                                          int chunk, int local, bool down, int pos) {
     const bool shared = (g == p.E);
-    const int nt = (c + kTileN - 1) / kTileN;
-    const int chunk = pad16((c + nt - 1) / nt);
-    const int f = local / nt;
+    const int f = nt == 1 ? local : local / nt;
     const int tt = local - f * nt;
     const int n = min(chunk, c - tt * chunk);
     const int map = shared ? 1 : 0;
@@ -129,24 +128,9 @@ __device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, i
     *n2 = nt * ((p.d + 2 * kSlabRows - 1) / (2 * kSlabRows));
 }
 
-// Largest g in [0, n) with first[g] <= i, given first[0] == 0 <= i and first
-// non-decreasing: the expert that owns list position i (an expert with no
-// tiles shares its first position with the next one and is skipped).
-__device__ __forceinline__ int owner_of(const int* first, int n, int i) {
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (first[mid] <= i)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    return lo;
-}
-
 // Plan over experts g = tid and g = tid + 1024 (G <= kPlanMaxG).  offsets: [E+1].
-// Tile counts per expert are scanned into first positions; then the whole
-// block writes the lists, consecutive threads taking consecutive tiles.
+// Tile counts per expert are scanned into first positions; then each warp
+// writes whole experts' tiles, its lanes taking consecutive list positions.
 __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) {
     __shared__ int s_c[kPlanMaxG], s_row0[kPlanMaxG], s_first1[kPlanMaxG], s_first2[kPlanMaxG];
     const int G = p.E + p.has_shared;
@@ -185,19 +169,24 @@ __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) 
             s_first2[g] = first2[h];
         }
     }
-    const int tot1 = tot1a + tot1b, tot2 = tot2a + tot2b;
     if (threadIdx.x == 0) {
-        p.ntiles[0] = tot1;
-        p.ntiles[1] = tot2;
+        p.ntiles[0] = tot1a + tot1b;
+        p.ntiles[1] = tot2a + tot2b;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < tot1; i += blockDim.x) {
-        const int g = owner_of(s_first1, G, i);
-        plan_tile(p, g, s_c[g], s_row0[g], i - s_first1[g], false, i);
-    }
-    for (int i = threadIdx.x; i < tot2; i += blockDim.x) {
-        const int g = owner_of(s_first2, G, i);
-        plan_tile(p, g, s_c[g], s_row0[g], i - s_first2[g], true, i);
+    const int ft1 = (p.inter + kSlabRows - 1) / kSlabRows;
+    const int ft2 = (p.d + 2 * kSlabRows - 1) / (2 * kSlabRows);
+    const int lane = threadIdx.x & 31;
+    for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
+        const int cg = s_c[g];
+        if (cg <= 0) continue;
+        const int nt = (cg + kTileN - 1) / kTileN;
+        const int chunk = pad16((cg + nt - 1) / nt);
+        const int row0 = s_row0[g];
+        for (int l = lane; l < nt * ft1; l += 32)
+            plan_tile(p, g, cg, row0, nt, chunk, l, false, s_first1[g] + l);
+        for (int l = lane; l < nt * ft2; l += 32)
+            plan_tile(p, g, cg, row0, nt, chunk, l, true, s_first2[g] + l);
     }
 }
 
