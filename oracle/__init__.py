@@ -71,6 +71,17 @@ def _bind(L):
     L.oracle_moe_rows.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, i32, P,
                                   i32]
     L.oracle_moe_rows.restype = i32
+    i64 = ctypes.c_int64
+    L.oracle_e4m3_encode.argtypes = [f64]
+    L.oracle_e4m3_encode.restype = ctypes.c_uint8
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_decode.restype = f64
+    L.oracle_fp8_block_exponent.argtypes = [f64]
+    L.oracle_fp8_block_exponent.restype = i32
+    L.oracle_quantize_fp8.argtypes = [P, i64, i64, P, P]
+    L.oracle_quantize_fp8.restype = i32
+    L.oracle_dequantize_fp8.argtypes = [P, P, i64, i64, P]
+    L.oracle_dequantize_fp8.restype = i32
     return L
 
 
@@ -112,6 +123,46 @@ def f64_to_bf16(a) -> np.ndarray:
     a = np.ascontiguousarray(a, dtype=np.float64)
     out = np.empty(a.shape, dtype=np.uint16)
     lib().oracle_round_bf16(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def e4m3_encode(v: float) -> int:
+    """E4M3 code of v (nearest, ties to even; saturating)."""
+    return int(lib().oracle_e4m3_encode(float(v)))
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().oracle_e4m3_decode(int(code) & 0xFF)
+
+
+def fp8_block_exponent(amax: float) -> int:
+    return int(lib().oracle_fp8_block_exponent(float(amax)))
+
+
+def quantize_fp8(w):
+    """bf16 matrix [rows, cols] (rows, cols multiples of 128) -> (codes uint8
+    [rows, cols], block exponents int8 [rows/128, cols/128])."""
+    u = _u16(w)
+    cols = u.shape[-1]
+    rows = u.size // cols
+    q = np.empty(u.shape, dtype=np.uint8)
+    sexp = np.empty(u.shape[:-2] + (u.shape[-2] // 128, cols // 128), dtype=np.int8)
+    rc = lib().oracle_quantize_fp8(_ptr(u), rows, cols, _ptr(q), _ptr(sexp))
+    if rc != 0:
+        raise ValueError("oracle_quantize_fp8: rows and cols must be multiples of 128")
+    return q, sexp
+
+
+def dequantize_fp8(q, sexp):
+    """codes [.., rows, cols] + block exponents -> the exact bf16 weights (uint16)."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sexp = np.ascontiguousarray(sexp, dtype=np.int8)
+    cols = q.shape[-1]
+    rows = q.size // cols
+    out = np.empty(q.shape, dtype=np.uint16)
+    rc = lib().oracle_dequantize_fp8(_ptr(q), _ptr(sexp), rows, cols, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_dequantize_fp8: rows and cols must be multiples of 128")
     return out
 
 

@@ -292,3 +292,72 @@ int oracle_moe_rows(const uint16_t* x, int T, int d, int E, int k, int inter,
     oracle_parallel_for(n_tokens, nthreads, rows_tokens, &c);
     return 0;
 }
+
+/* ------------------------------------------------------- FP8 (E4M3) storage */
+
+uint8_t oracle_e4m3_encode(double v) {
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;                 /* largest finite: 1.75 * 2^8 */
+    if (a < 0x1p-6) {                                   /* subnormal range: step 2^-9 */
+        const double m = rint(a * 0x1p9);               /* 0 .. 8, ties to even */
+        return sign | (uint8_t)m;                       /* m == 8 is the code of 2^-6 */
+    }
+    int e = ilogb(a);                                   /* 2^e <= a < 2^(e+1), -6 <= e <= 8 */
+    double m = rint(ldexp(a, 3 - e));                   /* 8 .. 16: 1.mmm scaled by 8 */
+    if (m == 16.0) {
+        m = 8.0;
+        e += 1;
+    }
+    if (e > 8 || (e == 8 && m > 14.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)m - 8));
+}
+
+double oracle_e4m3_decode(uint8_t code) {
+    const int ex = (code >> 3) & 0xF, man = code & 0x7;
+    if (ex == 0xF && man == 0x7) return NAN;
+    const double mag = ex == 0 ? ldexp((double)man, -9) : ldexp(1.0 + man / 8.0, ex - 7);
+    return (code & 0x80) ? -mag : mag;
+}
+
+int oracle_fp8_block_exponent(double amax) {
+    if (!(amax > 0.0)) return 0;
+    int s = ilogb(amax) - 8;                            /* amax < 2^(s+9) */
+    if (amax > ldexp(448.0, s)) s += 1;                 /* now amax <= 448 * 2^s */
+    while (s > -1000 && amax <= ldexp(448.0, s - 1)) s -= 1;   /* smallest such s */
+    if (s < -124) s = -124;
+    if (s > 127) s = 127;
+    return s;
+}
+
+int oracle_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, int8_t* sexp) {
+    if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128) return -1;
+    const int64_t bc = cols / 128;
+    for (int64_t br = 0; br < rows / 128; ++br)
+        for (int64_t bk = 0; bk < bc; ++bk) {
+            double amax = 0.0;
+            for (int64_t r = br * 128; r < br * 128 + 128; ++r)
+                for (int64_t c = bk * 128; c < bk * 128 + 128; ++c) {
+                    const double a = fabs(oracle_bf16_to_f64(w[r * cols + c]));
+                    if (a > amax) amax = a;
+                }
+            const int s = oracle_fp8_block_exponent(amax);
+            sexp[br * bc + bk] = (int8_t)s;
+            for (int64_t r = br * 128; r < br * 128 + 128; ++r)
+                for (int64_t c = bk * 128; c < bk * 128 + 128; ++c)
+                    q[r * cols + c] = oracle_e4m3_encode(ldexp(oracle_bf16_to_f64(w[r * cols + c]), -s));
+        }
+    return 0;
+}
+
+int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, int64_t cols,
+                          uint16_t* w_out) {
+    if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128) return -1;
+    const int64_t bc = cols / 128;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            w_out[r * cols + c] = oracle_f64_to_bf16(
+                ldexp(oracle_e4m3_decode(q[r * cols + c]), sexp[(r / 128) * bc + c / 128]));
+    return 0;
+}

@@ -107,6 +107,44 @@ int oracle_moe_rows(const uint16_t* x, int T, int d, int E, int k, int inter,
                     const uint16_t* shared_gate_up, const uint16_t* shared_down,
                     const int32_t* tokens, int n_tokens, double* out, int nthreads);
 
+/*
+ * FP8 storage of the routed experts' weights.
+ *
+ * "Kimi K2.5 Q&A", Q7.1: what the deployment quantizes is the routed experts'
+ * weight storage, while compute stays in BF16 ("storage quantization + high-
+ * precision compute"); the shared experts are exempt and stay BF16.  The
+ * pages name FP8 as the other storage option ("Kimi K2 deep dive", 3.2:
+ * FP8 halves the memory) but give no format.  The format taken here:
+ *   - element: FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ *     exponent 0 holds subnormals m * 2^-9; code 0x7F / 0xFF is NaN; largest
+ *     finite value 448; no infinities);
+ *   - one scale per block of 128 rows x 128 columns (K), a power of two 2^s
+ *     with s an int8, so dequantization q * 2^s is exact in bf16;
+ *   - s = the smallest integer with amax <= 448 * 2^s (amax = largest |w| of
+ *     the block), clamped to [-124, 127]; s = 0 for an all-zero block;
+ *   - q = the E4M3 value nearest to w * 2^-s (ties to even; w * 2^-s is exact).
+ */
+
+/* E4M3 code of v, nearest value, ties to even; |v| > 448 saturates to +-448,
+ * NaN -> 0x7F. */
+uint8_t oracle_e4m3_encode(double v);
+/* Value of an E4M3 code (NaN for 0x7F / 0xFF). */
+double oracle_e4m3_decode(uint8_t code);
+/* Block exponent s for a block whose largest magnitude is amax (rule above). */
+int oracle_fp8_block_exponent(double amax);
+/*
+ * Quantize a bf16 matrix w [rows, cols] (row-major; rows and cols multiples of
+ * 128) into codes q [rows, cols] and block exponents sexp [rows/128, cols/128].
+ * Returns 0, or -1 if a dimension is not a multiple of 128.
+ */
+int oracle_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, int8_t* sexp);
+/*
+ * Dequantize: w_out[r, c] = bf16( decode(q[r, c]) * 2^sexp[r/128, c/128] ), a
+ * value that bf16 holds exactly whenever it is finite.  Returns 0 or -1 as above.
+ */
+int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, int64_t cols,
+                          uint16_t* w_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -310,11 +310,100 @@ def pin_combine():
     assert np.array_equal(out1, y[slot_row.reshape(T, k)[:, 1]])
 
 
+
+# ------------------------------------------------------------ FP8 storage
+# "Kimi K2.5 Q&A", Q7.1: routed-expert weights are stored quantized and
+# computed in BF16; the element format is OCP FP8 E4M3 and the scale is one
+# power of two per 128 x 128 block (the rule in the oracle header).
+
+def _torch_e4m3(v):
+    return torch.from_numpy(np.asarray(v, dtype=np.float32)).to(torch.float8_e4m3fn).view(
+        torch.uint8).numpy()
+
+
+def pin_fp8_decode_library():
+    """Every code decodes to torch's float8_e4m3fn value (NaN only at 0x7F/0xFF)."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = np.array([oracle.e4m3_decode(c) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def pin_fp8_anchor_values():
+    """Published values of the format: 448 max, 2^-6 smallest normal, 2^-9 smallest subnormal."""
+    assert oracle.e4m3_encode(448.0) == 0x7E and oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_encode(2.0 ** -6) == 0x08
+    assert oracle.e4m3_encode(2.0 ** -9) == 0x01
+    assert oracle.e4m3_encode(1.0) == 0x38 and oracle.e4m3_encode(-2.0) == 0xC0
+    assert oracle.e4m3_encode(0.0) == 0x00
+    assert oracle.e4m3_encode(1000.0) == 0x7E and oracle.e4m3_encode(-1000.0) == 0xFE
+
+
+def pin_fp8_encode_library():
+    """Encoding matches torch's float -> float8_e4m3fn cast on random values and
+    on every midpoint between adjacent codes (ties to the even code)."""
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.uniform(-448, 448, 3000), rng.normal(0, 1, 3000),
+                        rng.normal(0, 0.01, 3000), rng.uniform(-2.0 ** -6, 2.0 ** -6, 1000)])
+    v = v.astype(np.float32).astype(np.float64)
+    assert np.array_equal(np.array([oracle.e4m3_encode(x) for x in v], dtype=np.uint8),
+                          _torch_e4m3(v))
+    vals = np.array([oracle.e4m3_decode(c) for c in range(0x7F)])     # 0 .. 448 ascending
+    mids = (vals[:-1] + vals[1:]) / 2.0
+    ours = np.array([oracle.e4m3_encode(m) for m in mids])
+    assert np.all(ours % 2 == 0)
+    assert np.array_equal(ours, _torch_e4m3(mids))
+    assert np.array_equal(np.array([oracle.e4m3_encode(-m) for m in mids]), ours | 0x80)
+
+
+def pin_fp8_block_exponent_brute_force():
+    """s is the smallest integer with amax <= 448 * 2^s, clamped to [-124, 127]."""
+    rng = np.random.default_rng(2)
+    cases = [0.05, 1.0, 448.0, 449.0, 3.0e-3, 7.0, 224.0, 224.5, 1e-30, 3e38]
+    cases += list(np.exp(rng.uniform(-20, 20, 40)))
+    for amax in cases:
+        brute = next(t for t in range(-300, 300) if amax <= 448.0 * 2.0 ** t)
+        assert oracle.fp8_block_exponent(amax) == min(max(brute, -124), 127), amax
+    assert oracle.fp8_block_exponent(0.0) == 0
+
+
+def pin_fp8_quantize_bounds():
+    """Per-element error within half a step of the format, each block's exponent
+    from its own amax and on its own block, the block maximum in the top binade."""
+    rng = np.random.default_rng(1)
+    rows, cols = 256, 384
+    w = rng.normal(0, 0.02, (rows, cols))
+    for i in range(rows // 128):
+        for j in range(cols // 128):
+            w[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128] *= 2.0 ** (i + 3 * j)
+    wb = _bf16(w).view(torch.int16).numpy().view(np.uint16)
+    wf = oracle.bf16_to_f64(wb)
+    q, sexp = oracle.quantize_fp8(wb)
+    assert sexp.shape == (rows // 128, cols // 128)
+    for i in range(rows // 128):
+        for j in range(cols // 128):
+            blk = wf[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]
+            brute = next(t for t in range(-300, 300) if np.abs(blk).max() <= 448.0 * 2.0 ** t)
+            assert sexp[i, j] == brute
+    wq = oracle.bf16_to_f64(oracle.dequantize_fp8(q, sexp))
+    scale = np.repeat(np.repeat(2.0 ** sexp.astype(float), 128, 0), 128, 1)
+    y = np.abs(wf) / scale
+    bound = np.where(y >= 2.0 ** -6, 2.0 ** -4 * np.abs(wf), 2.0 ** -10 * scale)
+    assert np.all(np.abs(wq - wf) <= bound)
+    assert np.all(np.sign(wq) * np.sign(wf) >= 0)
+    for i in range(rows // 128):
+        for j in range(cols // 128):
+            top = np.abs(wq[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]).max()
+            assert 224.0 <= top / 2.0 ** sexp[i, j] <= 448.0
+
 ALL_PINS = [pin_bf16_rounding, pin_sigmoid_silu, pin_route_worked_example,
             pin_router_scores_library, pin_topk_brute_force, pin_exact_ties,
             pin_weights_closed_form, pin_bias_selection_only, pin_permute_brute_force,
             pin_swiglu_textbook, pin_dense_vs_sparse, pin_special_cases,
-            pin_row_independence, pin_combine]
+            pin_row_independence, pin_combine, pin_fp8_decode_library, pin_fp8_anchor_values,
+            pin_fp8_encode_library, pin_fp8_block_exponent_brute_force, pin_fp8_quantize_bounds]
 
 
 def failing_pins():

@@ -53,6 +53,16 @@ MUTANTS = [
     ("combine_drops_shared", "o[i] = y_shared ? y_shared[(size_t)t * d + i] : 0.0;", "o[i] = 0.0;"),
     ("bf16_truncates", "r = ldexp(rint(ldexp(m, 8)), e - 8);",
      "r = ldexp(trunc(ldexp(m, 8)), e - 8);"),
+    ("e4m3_truncates", "double m = rint(ldexp(a, 3 - e));", "double m = trunc(ldexp(a, 3 - e));"),
+    ("e4m3_bias_off_by_one", "ldexp(1.0 + man / 8.0, ex - 7)", "ldexp(1.0 + man / 8.0, ex - 8)"),
+    ("e4m3_subnormal_step", "const double m = rint(a * 0x1p9);", "const double m = rint(a * 0x1p8);"),
+    ("fp8_exponent_one_low", "if (amax > ldexp(448.0, s)) s += 1;",
+     "if (amax > ldexp(448.0, s)) s += 0;"),
+    ("fp8_scale_applied_twice",
+     "q[r * cols + c] = oracle_e4m3_encode(ldexp(oracle_bf16_to_f64(w[r * cols + c]), -s));",
+     "q[r * cols + c] = oracle_e4m3_encode(ldexp(oracle_bf16_to_f64(w[r * cols + c]), -2 * s));"),
+    ("fp8_dequant_block_transposed", "sexp[(r / 128) * bc + c / 128]",
+     "sexp[(r / 128) + (c / 128) * (rows / 128)]"),
 ]
 
 
