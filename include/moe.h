@@ -198,6 +198,56 @@ int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const
                               int E, int k, int inter, float scale, uint16_t* out, void* stream);
 
 /*
+ * FP8 storage of the routed experts' weights ("Kimi K2.5 Q&A", Q7.1: the
+ * routed experts' weight storage is quantized while compute stays in BF16;
+ * the shared experts are exempt).  The pages give no format; this library
+ * uses E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * largest finite 448, NaN at 0x7F/0xFF, no infinities) with one power-of-two
+ * scale 2^s per block of 128 rows x 128 columns, s an int8:
+ *     s = smallest integer with max|w| <= 448 * 2^s over the block, clamped to
+ *         [-124, 127] (0 for an all-zero block);
+ *     q = the E4M3 value nearest to w * 2^-s, ties to even.
+ * q * 2^s is exactly representable in bf16, so the FP8 layer computes with
+ * exactly the weights the codes stand for (bf16 tensor-core math, as in
+ * moe_layer_forward).  Weights must be finite with |w| < 2^120.
+ *
+ * moe_quantize_fp8: w [rows, cols] bf16 row-major (rows and cols multiples of
+ * 128, cols / 128 <= 65535) -> q [rows, cols] uint8 codes and
+ * exps [rows/128, cols/128] int8 exponents, all device memory owned by the
+ * caller, asynchronous on `stream`.  Stacked expert weights quantize in one
+ * call: [E, 2*inter, d] as rows = E*2*inter, cols = d (exps [E, 2*inter/128,
+ * d/128]); [E, d, inter] as rows = E*d, cols = inter.
+ * Returns MOE_ERR_UNSUPPORTED_SHAPE for other shapes, MOE_ERR_INVALID_ARG for
+ * null or unaligned (16-byte) pointers.
+ */
+int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, int8_t* exps,
+                     void* stream);
+
+/*
+ * The layer of moe_layer_forward with the routed experts' weights in FP8
+ * (codes and exponents from moe_quantize_fp8):
+ *   wq_gate_up [E, 2*inter, d] uint8, wq_gate_up_exp [E, 2*inter/128, d/128] int8
+ *   wq_down    [E, d, inter]   uint8, wq_down_exp    [E, d/128, inter/128]   int8
+ * Everything else (router, shared expert, activations, output) is as in
+ * moe_layer_forward, bf16.  d and inter must be multiples of 128.  The
+ * routed weights are dequantized in shared memory just before the tensor
+ * cores read them; nothing in HBM holds a bf16 copy.  Errors as in
+ * moe_layer_forward.  The _ws form takes a caller-owned workspace of
+ * moe_workspace_size(T, d, E, k, inter) bytes, like moe_layer_forward_ws.
+ */
+int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                          const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                          const uint8_t* wq_down, const int8_t* wq_down_exp,
+                          const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                          int E, int k, int inter, float scale, uint16_t* out, void* stream);
+int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                             const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                             const uint8_t* wq_down, const int8_t* wq_down_exp,
+                             const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                             int E, int k, int inter, float scale, uint16_t* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word:
  * *device_status = MOE_OK, or the first problem a kernel recorded since the
  * last read (MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT).  Returns MOE_OK or

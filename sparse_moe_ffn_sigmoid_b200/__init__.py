@@ -20,7 +20,8 @@ __all__ = [
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_ws",
     "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
-    "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "moe_layer_forward_noalloc", "moe_quantize_fp8", "moe_layer_forward_fp8",
+    "moe_layer_forward_fp8_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
@@ -29,6 +30,7 @@ EXPORTED_SYMBOLS = [
     "moe_combine", "moe_layer_forward", "moe_layer_forward_ws", "moe_device_status",
     "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
+    "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
 ]
 
 MOE_OK = 0
@@ -45,7 +47,7 @@ def _load():
     path = _build.build()
     L = ctypes.CDLL(path)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    SZ, U64 = ctypes.c_size_t, ctypes.c_uint64
+    SZ, U64, I64 = ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int64
     sig = {
         "moe_status_string": ([I], ctypes.c_char_p),
         "moe_workspace_size": ([I, I, I, I, I], SZ),
@@ -63,6 +65,10 @@ def _load():
         "moe_profile_end": ([ctypes.POINTER(F), I, ctypes.POINTER(I)], I),
         "moe_kernel_name": ([I], ctypes.c_char_p),
         "moe_layer_forward_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, I, F, P, P], I),
+        "moe_quantize_fp8": ([P, I64, I64, P, P, P], I),
+        "moe_layer_forward_fp8": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P], I),
+        "moe_layer_forward_fp8_ws": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, SZ, P],
+                                     I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -197,6 +203,59 @@ def moe_layer_forward_noalloc(x, w_router, bias, w_gate_up, w_down, ws_gate_up, 
     rc = _LIB.moe_layer_forward_noalloc(*ptrs, T, d, E, k, inter, float(scale),
                                         _ptr(out, BF16, "out"), _stream(stream))
     _check("moe_layer_forward_noalloc", rc)
+
+
+def moe_quantize_fp8(w, stream=None):
+    """bf16 weights [..., rows, cols] (rows and cols multiples of 128) ->
+    (E4M3 codes uint8 [..., rows, cols], int8 block exponents
+    [..., rows/128, cols/128]), new tensors on w's device."""
+    if w.dim() < 2:
+        raise ValueError("w must have at least 2 dimensions")
+    rows, cols = w.shape[-2], w.shape[-1]
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    exps = torch.empty(tuple(w.shape[:-2]) + (rows // 128, cols // 128), dtype=torch.int8,
+                       device=w.device)
+    rc = _LIB.moe_quantize_fp8(_ptr(w, BF16, "w"), w.numel() // cols, cols,
+                               _ptr(q, torch.uint8, "q"), _ptr(exps, torch.int8, "exps"),
+                               _stream(stream))
+    _check("moe_quantize_fp8", rc)
+    return q, exps
+
+
+def _layer_fp8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                    ws_gate_up, ws_down):
+    T, d = x.shape
+    E = w_router.shape[0]
+    inter = wq_gate_up.shape[1] // 2
+    return ([_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"), _ptr(bias, F32, "bias"),
+             _ptr(wq_gate_up, torch.uint8, "wq_gate_up"),
+             _ptr(wq_gate_up_exp, torch.int8, "wq_gate_up_exp"),
+             _ptr(wq_down, torch.uint8, "wq_down"), _ptr(wq_down_exp, torch.int8, "wq_down_exp"),
+             _ptr(ws_gate_up, BF16, "ws_gate_up"), _ptr(ws_down, BF16, "ws_down")],
+            T, d, E, inter)
+
+
+def moe_layer_forward_fp8(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                          ws_gate_up, ws_down, k: int, scale: float, out, stream=None):
+    """moe_layer_forward with the routed experts' weights as FP8 codes + block
+    exponents (from moe_quantize_fp8); router and shared expert stay bf16."""
+    ptrs, T, d, E, inter = _layer_fp8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp,
+                                           wq_down, wq_down_exp, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_fp8(*ptrs, T, d, E, k, inter, float(scale),
+                                    _ptr(out, BF16, "out"), _stream(stream))
+    _check("moe_layer_forward_fp8", rc)
+
+
+def moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                             ws_gate_up, ws_down, k: int, scale: float, out, workspace,
+                             stream=None):
+    ptrs, T, d, E, inter = _layer_fp8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp,
+                                           wq_down, wq_down_exp, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_fp8_ws(*ptrs, T, d, E, k, inter, float(scale),
+                                       _ptr(out, BF16, "out"),
+                                       _ptr(workspace, torch.uint8, "workspace"),
+                                       workspace.numel(), _stream(stream))
+    _check("moe_layer_forward_fp8_ws", rc)
 
 
 def moe_device_status(stream=None) -> int:

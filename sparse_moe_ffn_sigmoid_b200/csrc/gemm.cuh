@@ -33,6 +33,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace moe {
 
@@ -50,6 +51,11 @@ constexpr int kMaxN = 256;                    // MMA N limit (router tiles)
 constexpr int kTileN = 256;
 constexpr int kGemmThreads = 352;             // 11 warps: roles below
 constexpr int kTokenWarp = 10;
+// FP8-weight mode: four more warps dequantize the weight codes into the bf16 ring
+constexpr int kConvWarps = 4;
+constexpr int kConvWarp0 = 11;
+constexpr int kGemmThreadsFP8 = kGemmThreads + 32 * kConvWarps;
+constexpr int kSlabBytes8 = kSlabRows * kBK;  // one FP8 slab per K step (128 rows x 64 codes)
 constexpr int kTmemCols = 512;
 
 enum GemmEpilogue : int {
@@ -84,6 +90,13 @@ struct __align__(64) GemmArgs {
     int acc_bufs;             // accumulator buffers in TMEM (1 or 2)
     int acc_stride;           // TMEM columns per accumulator buffer
     unsigned long long timeout_ns;
+    // FP8-weight mode only: routed tiles (map 0) read E4M3 codes through a8_map
+    // ([rows, K] uint8, 64 x 128 boxes) and one int8 exponent per 128 x 128 block
+    // (a8_scale[(row / 128) * a8_kblocks + k / 128]); shared tiles (map 1) stay bf16
+    CUtensorMap a8_map;
+    const int8_t* a8_scale;
+    int a8_kblocks;
+    int stages_a8;            // FP8 code ring depth
 };
 
 __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int i) {
@@ -156,8 +169,124 @@ __device__ __forceinline__ void store_block_bf16(bf16* stg, const float (&v)[kSt
     __syncwarp();
 }
 
-template <int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_constant__ GemmArgs args) {
+// Lane 0 waits (bounded) and the warp shares the outcome; after a completed
+// wait every lane observes the phase itself (one try_wait, which cannot fail
+// then: the barrier cannot complete its next phase before this warp acts), so
+// each lane acquires what the phase publishes.
+__device__ __forceinline__ bool wait_lane0(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           uint64_t tmo, int lane) {
+    bool ok = true;
+    if (lane == 0) ok = wait_bounded(bar, parity, abort_flag, tmo);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) (void)ptx::mbar_try_wait(bar, parity);
+    return ok;
+}
+
+// FP8-weight mode: the kConvWarps converter warps (thread ct = 0..127) fill
+// the bf16 weight ring for every K step, in step order, all four warps
+// together: at every step each warp waits for the bf16 slot (empty: the MMAs
+// of step q - SA done), and for a routed step also for its codes (full8).
+// Parity waits only tell a phase from the one before it, so every warp waits
+// at every step and the warps meet on a named barrier once per step: none can
+// run a lap ahead of the slot's barrier (and write a slot the MMA still
+// reads) or fall a lap behind it.
+// Routed step: thread ct converts eight codes at a time, units u = ct + 128 i
+// (slab u / 1024, row (u / 8) % 128, chunk u % 8), into the 128-byte-swizzled
+// layout a TMA box would have produced (row r at byte 128 r, 16-byte chunk c
+// at position c ^ (r % 8)); each code times the block's 2^s is exact in bf16.
+// Every thread fences its stores towards the async proxy before the barrier,
+// and thread 0 then publishes the slot (full) and frees the codes (empty8).
+// Shared-expert step (bf16 in HBM): after the barrier thread 0 loads the bf16
+// weights into the slot with TMA (arrive.expect_tx on full).  The weight
+// producer, which runs up to SA8 routed steps ahead, never touches the bf16
+// ring in this mode.
+template <int nslab>
+__device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint8_t* ring8,
+                                                uint8_t* ring_a, int SA, int SA8, uint64_t* full,
+                                                uint64_t* empty, uint64_t* full8,
+                                                uint64_t* empty8, volatile int* abort_flag,
+                                                uint64_t tmo, int ntiles, int ct) {
+    constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
+    constexpr uint32_t a_bytes = nslab * kSlabBytes;
+    constexpr int kUnits = nslab * kSlabRows * (kBK / 8) / (32 * kConvWarps);   // per thread
+    const int lane = ct & 31;
+    const uint64_t pol = ptx::policy_evict_first();
+    Ring rq{0, 0, SA};          // bf16 slot of step q
+    Ring r8{0, 0, SA8};         // code slot of the routed steps
+    bool ok = true;
+    uint32_t issued = 0, issued_parity = 0;   // thread 0's bf16 loads, for draining
+    for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
+        const Tile t = load_tile(args, i);
+        const bool routed = (t.map == 0);
+        const int8_t* sc0 = args.a8_scale + (t.a_row0 / kQuantBlock) * args.a8_kblocks;
+        const int8_t* sc1 = args.a8_scale + (t.a_row1 / kQuantBlock) * args.a8_kblocks;
+        for (int ks = t.ks0; ks < t.ks1; ++ks) {
+            bool w_ok = (!routed || wait_lane0(&full8[r8.stage], r8.phase, abort_flag, tmo, lane)) &&
+                        wait_lane0(&empty[rq.stage], rq.phase ^ 1, abort_flag, tmo, lane);
+            if (routed && w_ok) {
+                const Fp8Scale s0 = fp8_scale(__ldg(sc0 + ks * kBK / kQuantBlock));
+                const Fp8Scale s1 = nslab == 2 ? fp8_scale(__ldg(sc1 + ks * kBK / kQuantBlock)) : s0;
+                const uint8_t* src = ring8 + r8.stage * a8_bytes;
+                uint8_t* dst = ring_a + rq.stage * a_bytes;
+                // all of this thread's code loads first, then the conversions:
+                // the kUnits chains are independent, so their latencies overlap
+                uint2 codes[kUnits];
+#pragma unroll
+                for (int j = 0; j < kUnits; ++j) {
+                    const int u = ct + 32 * kConvWarps * j;
+                    const int slab = u / (kSlabRows * 8);
+                    const int r = (u >> 3) & (kSlabRows - 1);
+                    codes[j] = *reinterpret_cast<const uint2*>(src + slab * kSlabBytes8 + r * kBK +
+                                                               (u & 7) * 8);
+                }
+#pragma unroll
+                for (int j = 0; j < kUnits; ++j) {
+                    const int u = ct + 32 * kConvWarps * j;
+                    const int slab = u / (kSlabRows * 8);
+                    const int r = (u >> 3) & (kSlabRows - 1);
+                    const int c = u & 7;
+                    *reinterpret_cast<uint4*>(dst + slab * kSlabBytes + r * (kBK * 2) +
+                                              ((c ^ (r & 7)) << 4)) =
+                        fp8x8_to_bf16x8(codes[j], slab == 0 ? s0 : s1);
+                }
+                ptx::fence_proxy_async_smem();
+            }
+            // every converter thread reaches this barrier once per step
+            ok = ptx::bar_red_and(1, 32 * kConvWarps, w_ok);
+            if (!ok) break;
+            if (ct == 0) {
+                if (routed) {
+                    ptx::mbar_arrive(&full[rq.stage]);
+                    ptx::mbar_arrive(&empty8[r8.stage]);
+                } else {
+                    uint64_t* bar = &full[rq.stage];
+                    uint8_t* sa = ring_a + rq.stage * a_bytes;
+                    ptx::mbar_arrive_expect_tx(bar, a_bytes);
+                    ptx::tma_load_2d_hint(sa, &args.a_map[1], bar, ks * kBK, t.a_row0, pol);
+                    if (nslab == 2)
+                        ptx::tma_load_2d_hint(sa + kSlabBytes, &args.a_map[1], bar, ks * kBK,
+                                              t.a_row1, pol);
+                    issued |= 1u << rq.stage;
+                    issued_parity = (issued_parity & ~(1u << rq.stage)) | (rq.phase << rq.stage);
+                }
+            }
+            if (routed) r8.next();
+            rq.next();
+        }
+    }
+    if (ct == 0 && !ok) {
+        // the bf16 loads this thread started land before the CTA exits
+        for (int s = 0; s < SA; ++s)
+            if (issued & (1u << s)) wait_bounded(&full[s], (issued_parity >> s) & 1, nullptr, tmo);
+    }
+}
+
+// FP8A: routed weights arrive as E4M3 codes and are dequantized in shared
+// memory by the converter warps (kGemmThreadsFP8 threads); FP8A = false is the
+// all-bf16 kernel (kGemmThreads threads).
+template <int EPI, bool FP8A>
+__global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -169,15 +298,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
     constexpr int nslab = (EPI == kEpiStoreF32) ? 1 : 2;
     const uint32_t a_bytes = nslab * kSlabBytes;
     const uint32_t b_bytes = args.n_max * kBK * 2;
+    static_assert(!FP8A || nslab == 2, "FP8 weights are for the expert GEMMs");
+    const int SA8 = FP8A ? args.stages_a8 : 0;
+    constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
     uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
     uint8_t* ring_b = ring_a + SA * a_bytes;                 // [SB][n_max x 64] bf16
-    bf16* staging = reinterpret_cast<bf16*>(ring_b + SB * b_bytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(ring_b + SB * b_bytes + kStagingBytes);
+    uint8_t* ring8 = ring_b + SB * b_bytes;                  // [SA8][nslab][128 x 64] E4M3
+    bf16* staging = reinterpret_cast<bf16*>(ring8 + SA8 * a8_bytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring8 + SA8 * a8_bytes + kStagingBytes);
     uint64_t* empty = full + SA;
     uint64_t* acc_full = empty + SA;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* full8 = drain + 1;                             // [SA8] codes landed
+    uint64_t* empty8 = full8 + SA8;                          // [SA8] codes converted
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(empty8 + SA8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -193,6 +328,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
             ptx::mbar_init(&acc_empty[b], kEpiWarps);
         }
         ptx::mbar_init(drain, 1);
+        for (int s = 0; s < SA8; ++s) {
+            ptx::mbar_init(&full8[s], 1);    // the weight producer's codes
+            ptx::mbar_init(&empty8[s], 1);   // converter thread 0, after all converted
+        }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -203,6 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
         ptx::prefetch_tensormap(&args.b_map[1]);
         ptx::prefetch_tensormap(&args.b_map64[0]);
         ptx::prefetch_tensormap(&args.b_map64[1]);
+        if (FP8A) ptx::prefetch_tensormap(&args.a8_map);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_holder, kTmemCols);
@@ -225,14 +365,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
             Ring rq{0, 0, SA};          // K step q: its full barrier / weight slot
             Ring rb{0, 0, SB};          // token slot of step q
             Ring rp{0, 0, SA};          // step q - SB, whose MMAs free token slot q % SB
+            Ring r8{0, 0, SA8};         // FP8 code slot of the routed steps
             uint32_t q = 0;
             uint32_t issued = 0, issued_parity = 0;             // per-barrier bits, for draining
+            uint32_t issued8 = 0, issued8_parity = 0;
             bool ok = true;
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
                 const Tile t = load_tile(args, i);
                 const int npad = pad16(t.n);
                 const uint32_t tx = weights ? a_bytes : npad * kBK * 2;
                 for (int ks = t.ks0; ks < t.ks1; ++ks, ++q) {
+                    if (FP8A && weights && t.map != 0) {
+                        // shared-expert step: the converter warps load its bf16
+                        // weights (they track the bf16 ring step by step; this
+                        // thread runs up to SA8 routed steps ahead of it and must
+                        // not wait on its barriers)
+                        rq.next();
+                        rb.next();
+                        continue;
+                    }
+                    if (FP8A && weights) {
+                        // routed step: E4M3 codes into the code ring; the converter
+                        // warps fill and publish the bf16 slot
+                        if (!wait_bounded(&empty8[r8.stage], r8.phase ^ 1, abort_flag, tmo)) {
+                            ok = false;
+                            break;
+                        }
+                        uint64_t* bar8 = &full8[r8.stage];
+                        ptx::mbar_arrive_expect_tx(bar8, a8_bytes);
+                        uint8_t* s8 = ring8 + r8.stage * a8_bytes;
+                        ptx::tma_load_2d_hint(s8, &args.a8_map, bar8, ks * kBK, t.a_row0, pol);
+                        ptx::tma_load_2d_hint(s8 + kSlabBytes8, &args.a8_map, bar8, ks * kBK,
+                                              t.a_row1, pol);
+                        issued8 |= 1u << r8.stage;
+                        issued8_parity = (issued8_parity & ~(1u << r8.stage)) | (r8.phase << r8.stage);
+                        r8.next();
+                        rq.next();
+                        rb.next();
+                        continue;
+                    }
                     bool free_ok;
                     if (weights) {
                         // weight slot is free once the MMAs of step q - SA are done
@@ -277,6 +448,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 for (int s = 0; s < SA; ++s)
                     if (issued & (1u << s))
                         wait_bounded(&full[s], (issued_parity >> s) & 1, nullptr, tmo);
+                for (int s = 0; s < SA8; ++s)
+                    if (issued8 & (1u << s))
+                        wait_bounded(&full8[s], (issued8_parity >> s) & 1, nullptr, tmo);
             }
         }
     } else if (warp == 1) {
@@ -349,6 +523,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
                 wait_bounded(drain, 0, nullptr, tmo);
             }
         }
+    } else if (FP8A && warp >= kConvWarp0) {
+        // ---------------------------------------------------------- converters
+        convert_weights<nslab>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
+                               abort_flag, tmo, ntiles, threadIdx.x - 32 * kConvWarp0);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
@@ -437,11 +615,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_gemm_kernel(const __grid_
 }
 
 // Dynamic shared memory the kernel needs for a configuration.
-inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max) {
+inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max, int stages_a8 = 0) {
     const size_t a = static_cast<size_t>(nslab) * kSlabBytes;
     const size_t b = static_cast<size_t>(n_max) * kBK * 2;
-    return 1024 /* alignment slack */ + stages_a * a + stages_b * b + kStagingBytes +
-           (2 * stages_a + 5) * 8 + 16;
+    const size_t a8 = static_cast<size_t>(nslab) * kSlabBytes8;
+    return 1024 /* alignment slack */ + stages_a * a + stages_b * b + stages_a8 * a8 +
+           kStagingBytes + (2 * stages_a + 2 * stages_a8 + 5) * 8 + 16;
 }
 
 }  // namespace moe

@@ -171,15 +171,13 @@ int device_info(DeviceInfo* out) {
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
-        if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kMaxDynSmem)) != cudaSuccess ||
+        const int smem = static_cast<int>(kMaxDynSmem);
+        const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, false>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, false>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32, false>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, true>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, true>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(scan_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kScanSmem)) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -208,6 +206,21 @@ EncodeTiledFn encode_fn() {
             fn = reinterpret_cast<EncodeTiledFn>(p);
     });
     return fn;
+}
+
+// Row-major E4M3 code matrix [rows, cols] (uint8) read in boxes of 128 rows x
+// 64 codes, unswizzled (the converter warps read it, not the tensor core).
+bool make_map8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kSlabRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Row-major bf16 matrix [rows, cols] read in boxes of box_rows x 64 columns,
@@ -245,11 +258,27 @@ void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
     a.timeout_ns = g_timeout_ns.load();
 }
 
-template <int EPI>
+// FP8-weight expert GEMMs: a shallow bf16 ring between the converter warps
+// and the MMAs, a deep code ring for the weight stream (half the bytes per
+// slot), the token ring as in the bf16 kernel.
+void fill_pipeline_fp8(GemmArgs& a, int n_max) {
+    fill_pipeline(a, 2, n_max);
+    const size_t a_bytes = 2 * static_cast<size_t>(kSlabBytes);
+    const size_t a8_bytes = 2 * static_cast<size_t>(kSlabBytes8);
+    const size_t b_bytes = static_cast<size_t>(n_max) * kBK * 2;
+    const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 1024;
+    a.stages_b = (n_max <= 64 || n_max > 128) ? 2 : 3;
+    a.stages_a = std::max(a.stages_b, n_max <= 128 ? 3 : 2);
+    const size_t left = budget - a.stages_a * a_bytes - a.stages_b * b_bytes;
+    a.stages_a8 = static_cast<int>(std::min<size_t>(12, left / a8_bytes));
+}
+
+template <int EPI, bool FP8A = false>
 int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
-    const size_t smem = gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max);
-    if (smem > kMaxDynSmem) return MOE_ERR_UNSUPPORTED_SHAPE;
-    moe_gemm_kernel<EPI><<<grid, kGemmThreads, smem, st>>>(a);
+    const size_t smem =
+        gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max, FP8A ? a.stages_a8 : 0);
+    if (smem > kMaxDynSmem || (FP8A && a.stages_a8 < 2)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    moe_gemm_kernel<EPI, FP8A><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -278,7 +307,7 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
     a.out_ld = E;
     a.col_limit = E;
     fill_pipeline(a, 1, chunk);
-    int rc = launch_gemm<kEpiStoreF32>(a, std::min(a.ntiles_host, di.sms), st);
+    int rc = launch_gemm<kEpiStoreF32, false>(a, std::min(a.ntiles_host, di.sms), st);
     if (rc != MOE_OK) return rc;
     rec.mark(st);
     const int npl = (E + 31) / 32;
@@ -325,13 +354,26 @@ int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offset
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Routed experts' weights stored as E4M3 codes with one int8 exponent per
+// 128 x 128 block (quant.cuh): gate|up codes [E, 2I, d] + [E, 2I/128, d/128],
+// down codes [E, d, I] + [E, d/128, I/128].
+struct Fp8Experts {
+    const uint8_t* gate_up;
+    const int8_t* gate_up_exp;
+    const uint8_t* down;
+    const int8_t* down_exp;
+};
+
 // gather + gate|up + down over a planned tile list.
 //   rows_b0: rows of the permuted token matrix (T*k); h_rows / y rows: rows_b0 (+ T if shared)
+//   f8: routed weights in FP8 (then w_gate_up / w_down are unused), or null for bf16
 int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T, int d, int E,
                int k, int inter, const bf16* w_gate_up, const bf16* w_down,
                const bf16* ws_gate_up, const bf16* ws_down, bool shared, bf16* xperm, bf16* h,
                bf16* y, const int4* tiles1, const int4* tiles2, const int* ntiles,
-               int max_tiles1, int max_tiles2, cudaStream_t st, Recorder& rec) {
+               int max_tiles1, int max_tiles2, cudaStream_t st, Recorder& rec,
+               const Fp8Experts* f8 = nullptr) {
+    if (f8 != nullptr && !shared) return MOE_ERR_INVALID_ARG;
     const int rows_routed = T * k;
     const int rows_all = rows_routed + (shared ? T : 0);
     if (rows_routed > 0) {
@@ -346,8 +388,18 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     GemmArgs g1;
     std::memset(&g1, 0, sizeof(g1));
     const bf16* xp = rows_routed > 0 ? xperm : x;
-    if (!make_map(&g1.a_map[0], w_gate_up, static_cast<uint64_t>(E) * 2 * inter, d, kSlabRows) ||
-        !make_map(&g1.b_map[0], xp, std::max(rows_routed, 1), d, kBoxRows) ||
+    if (f8 != nullptr) {
+        // routed tiles read codes; slot 0 of the bf16 maps is never used
+        if (!make_map8(&g1.a8_map, f8->gate_up, static_cast<uint64_t>(E) * 2 * inter, d) ||
+            !make_map(&g1.a_map[0], ws_gate_up, 2ull * inter, d, kSlabRows))
+            return MOE_ERR_CUDA;
+        g1.a8_scale = f8->gate_up_exp;
+        g1.a8_kblocks = d / kQuantBlock;
+    } else if (!make_map(&g1.a_map[0], w_gate_up, static_cast<uint64_t>(E) * 2 * inter, d,
+                         kSlabRows)) {
+        return MOE_ERR_CUDA;
+    }
+    if (!make_map(&g1.b_map[0], xp, std::max(rows_routed, 1), d, kBoxRows) ||
         !make_map(&g1.b_map[1], x, T, d, kBoxRows) ||
         !make_map(&g1.b_map64[0], xp, std::max(rows_routed, 1), d, kBoxRowsBig) ||
         !make_map(&g1.b_map64[1], x, T, d, kBoxRowsBig))
@@ -362,15 +414,29 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     g1.out = h;
     g1.out_ld = inter;
     g1.col_limit = inter;
-    fill_pipeline(g1, 2, n_max);
-    int rc = launch_gemm<kEpiSwiGLU>(g1, std::min(max_tiles1, di.sms), st);
+    int rc;
+    if (f8 != nullptr) {
+        fill_pipeline_fp8(g1, n_max);
+        rc = launch_gemm<kEpiSwiGLU, true>(g1, std::min(max_tiles1, di.sms), st);
+    } else {
+        fill_pipeline(g1, 2, n_max);
+        rc = launch_gemm<kEpiSwiGLU>(g1, std::min(max_tiles1, di.sms), st);
+    }
     if (rc != MOE_OK) return rc;
     rec.mark(st);
 
     GemmArgs g2;
     std::memset(&g2, 0, sizeof(g2));
-    if (!make_map(&g2.a_map[0], w_down, static_cast<uint64_t>(E) * d, inter, kSlabRows) ||
-        !make_map(&g2.b_map[0], h, rows_all, inter, kBoxRows) ||
+    if (f8 != nullptr) {
+        if (!make_map8(&g2.a8_map, f8->down, static_cast<uint64_t>(E) * d, inter) ||
+            !make_map(&g2.a_map[0], ws_down, d, inter, kSlabRows))
+            return MOE_ERR_CUDA;
+        g2.a8_scale = f8->down_exp;
+        g2.a8_kblocks = inter / kQuantBlock;
+    } else if (!make_map(&g2.a_map[0], w_down, static_cast<uint64_t>(E) * d, inter, kSlabRows)) {
+        return MOE_ERR_CUDA;
+    }
+    if (!make_map(&g2.b_map[0], h, rows_all, inter, kBoxRows) ||
         !make_map(&g2.b_map64[0], h, rows_all, inter, kBoxRowsBig))
         return MOE_ERR_CUDA;
     if (shared) {
@@ -385,8 +451,13 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     g2.out = y;
     g2.out_ld = d;
     g2.col_limit = d;
-    fill_pipeline(g2, 2, n_max);
-    rc = launch_gemm<kEpiStoreBF16>(g2, std::min(max_tiles2, di.sms), st);
+    if (f8 != nullptr) {
+        fill_pipeline_fp8(g2, n_max);
+        rc = launch_gemm<kEpiStoreBF16, true>(g2, std::min(max_tiles2, di.sms), st);
+    } else {
+        fill_pipeline(g2, 2, n_max);
+        rc = launch_gemm<kEpiStoreBF16>(g2, std::min(max_tiles2, di.sms), st);
+    }
     if (rc != MOE_OK) return rc;
     rec.mark(st);
     return MOE_OK;
@@ -415,7 +486,8 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
 
 int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* wgu,
                   const bf16* wdn, const bf16* sgu, const bf16* sdn, int T, int d, int E, int k,
-                  int inter, float scale, bf16* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+                  int inter, float scale, bf16* out, void* ws, size_t ws_bytes, cudaStream_t st,
+                  const Fp8Experts* f8 = nullptr) {
     const Layout L = make_layout(T, d, E, k, inter);
     if (ws == nullptr || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
     DeviceInfo di;
@@ -452,7 +524,7 @@ int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* 
                         reinterpret_cast<int*>(P(L.blk)), plan, st, rec);
     if (rc != MOE_OK) return rc;
     rc = launch_ffn(di, x, row_token, T, d, E, k, inter, wgu, wdn, sgu, sdn, true, xperm, h, y,
-                    tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec);
+                    tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8);
     if (rc != MOE_OK) return rc;
     rc = launch_combine(y, y + static_cast<size_t>(T) * k * d, w, slot_row, T, d, k, out, st, rec);
     g_last_launches.store(rec.n);
@@ -686,6 +758,62 @@ int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const
                          reinterpret_cast<const bf16*>(ws_down), T, d, E, k, inter, scale,
                          reinterpret_cast<bf16*>(out), ws, MOE_NOALLOC_SCRATCH_BYTES,
                          static_cast<cudaStream_t>(stream));
+}
+
+int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, int8_t* exps,
+                     void* stream) {
+    if (rows < 0 || cols < 0 || rows % kQuantBlock != 0 || cols % kQuantBlock != 0 ||
+        rows / kQuantBlock > 0x7FFFFFFF || cols / kQuantBlock > 65535)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!all_ok(w, q) || exps == nullptr) return MOE_ERR_INVALID_ARG;
+    const dim3 grid(static_cast<unsigned>(rows / kQuantBlock), static_cast<unsigned>(cols / kQuantBlock));
+    fp8_quantize_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const bf16*>(w), cols, q, exps);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                             const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                             const uint8_t* wq_down, const int8_t* wq_down_exp,
+                             const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                             int E, int k, int inter, float scale, uint16_t* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (d % kQuantBlock != 0 || inter % kQuantBlock != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_down, ws_gate_up, ws_down, out, workspace) ||
+        wq_gate_up_exp == nullptr || wq_down_exp == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    const Fp8Experts f8{wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp};
+    return layer_forward(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                         bias, nullptr, nullptr, reinterpret_cast<const bf16*>(ws_gate_up),
+                         reinterpret_cast<const bf16*>(ws_down), T, d, E, k, inter, scale,
+                         reinterpret_cast<bf16*>(out), workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream), &f8);
+}
+
+int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                          const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                          const uint8_t* wq_down, const int8_t* wq_down_exp,
+                          const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                          int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (d % kQuantBlock != 0 || inter % kQuantBlock != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_down, ws_gate_up, ws_down, out) ||
+        wq_gate_up_exp == nullptr || wq_down_exp == nullptr || !(scale == scale))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = make_layout(T, d, E, k, inter).total;
+    void* ws = nullptr;
+    rc = owned_workspace(static_cast<cudaStream_t>(stream), need, &ws);
+    if (rc != MOE_OK) return rc;
+    return moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
+                                    wq_down_exp, ws_gate_up, ws_down, T, d, E, k, inter, scale,
+                                    out, ws, need, stream);
 }
 
 int moe_device_status(void* stream, int* device_status) {

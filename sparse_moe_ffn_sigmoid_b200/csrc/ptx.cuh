@@ -57,6 +57,27 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Named barrier `id` (not 0, which __syncthreads uses) over `nthreads` threads
+// (a multiple of 32); returns whether `pred` held in every one of them.
+__device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes on

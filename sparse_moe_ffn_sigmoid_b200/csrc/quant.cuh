@@ -1,0 +1,142 @@
+// quant.cuh -- FP8 (E4M3) storage of the routed experts' weights.
+//
+// "Kimi K2.5 Q&A", Q7.1: the deployment quantizes the routed experts' weight
+// storage while compute stays in BF16, and the shared experts stay BF16.  The
+// pages give no FP8 format; the one used here is OCP E4M3 elements with one
+// power-of-two scale 2^s per block of 128 rows x 128 columns (K), s an int8:
+//   s = the smallest integer with amax <= 448 * 2^s, clamped to [-124, 127]
+//       (s = 0 for an all-zero block), amax = the block's largest |w|;
+//   q = E4M3 nearest to w * 2^-s (ties to even; the scaling is exact).
+// Dequantization q * 2^s is then exact in bf16, so the expert GEMMs compute
+// with exactly the weights the codes stand for.
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kQuantBlock = 128;          // rows and columns per scale block
+constexpr int kQuantThreads = 256;
+
+// 2^e as a float, e in [-126, 127] (a normal number, built from its bits).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
+// Block exponent from the block's largest magnitude (rule above), from the
+// bits of amax: amax = 1.f * 2^E lies within 448 * 2^(E-8) = 1.75 * 2^E exactly
+// when 1.f <= 1.75.
+__device__ __forceinline__ int fp8_block_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    const uint32_t bits = __float_as_uint(amax);
+    const int ef = static_cast<int>(bits >> 23) & 0xFF;
+    if (ef == 0) return -124;                               // below 2^-126: clamped
+    int s = ef - 127 - 8 + ((bits & 0x7FFFFF) > 0x600000 ? 1 : 0);
+    return max(-124, min(127, s));
+}
+
+// One block of kQuantThreads threads per 128 x 128 block (blockIdx.x = row
+// block, blockIdx.y = column block) of w [rows, cols] bf16 row-major.
+__global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(const bf16* __restrict__ w,
+                                                                     long long cols,
+                                                                     uint8_t* __restrict__ q,
+                                                                     int8_t* __restrict__ sexp) {
+    __shared__ float s_max[kQuantThreads / 32];
+    const long long r0 = static_cast<long long>(blockIdx.x) * kQuantBlock;
+    const long long c0 = static_cast<long long>(blockIdx.y) * kQuantBlock;
+    // thread -> 8 consecutive columns of rows r = tid / 16 + 16 i
+    const int cc = (threadIdx.x & 15) * 8;
+    const int rr = threadIdx.x >> 4;
+    float amax = 0.0f;
+    for (int i = 0; i < kQuantBlock / 16; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4*>(w + (r0 + rr + 16 * i) * cols + c0 + cc);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = s_max[0];
+#pragma unroll
+    for (int i = 1; i < kQuantThreads / 32; ++i) amax = fmaxf(amax, s_max[i]);
+    const int s = fp8_block_exponent(amax);
+    if (threadIdx.x == 0)
+        sexp[static_cast<long long>(blockIdx.x) * gridDim.y + blockIdx.y] = static_cast<int8_t>(s);
+    // w * 2^-s in two exact steps (2^-s alone may be below the normal range)
+    const float m1 = pow2f(-(s / 2));
+    const float m2 = pow2f(-(s - s / 2));
+    for (int i = 0; i < kQuantBlock / 16; ++i) {
+        const long long off = (r0 + rr + 16 * i) * cols + c0 + cc;
+        const uint4 v = *reinterpret_cast<const uint4*>(w + off);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+        uint2 out;
+        uint8_t* o = reinterpret_cast<uint8_t*>(&out);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            o[2 * j] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.x, m1), m2), __NV_SATFINITE,
+                                             __NV_E4M3);
+            o[2 * j + 1] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.y, m1), m2),
+                                                 __NV_SATFINITE, __NV_E4M3);
+        }
+        *reinterpret_cast<uint2*>(q + off) = out;
+    }
+}
+
+// Four E4M3 codes (the bytes of v, little-endian) -> two bf16x2 words whose
+// values are code * 2^-120, bit for bit: each code's sign moves from bit 7 to
+// bit 15 of its 16-bit lane and its seven magnitude bits eeeemmm from [6:0]
+// to [10:4].  A bf16 with exponent field 0000eeee and mantissa mmm0000 is
+// 2^(eeee-127) * 1.mmm for eeee > 0, and 2^-126 * 0.mmm (a subnormal) for
+// eeee = 0, which is the E4M3 value (2^(eeee-7) * 1.mmm, or 2^-6 * 0.mmm)
+// times 2^-120 in both cases.
+__device__ __forceinline__ void fp8x4_to_bf16x4_pow2m120(uint32_t v, uint32_t& lo, uint32_t& hi) {
+    const uint32_t mag = v & 0x7F7F7F7Fu;
+    const uint32_t sgn = v & 0x80808080u;
+    // byte_perm 0x1404: [0, byte0, 0, byte1]; 0x3424: [0, byte2, 0, byte3]
+    lo = (__byte_perm(mag, 0u, 0x1404) >> 4) | __byte_perm(sgn, 0u, 0x1404);
+    hi = (__byte_perm(mag, 0u, 0x3424) >> 4) | __byte_perm(sgn, 0u, 0x3424);
+}
+
+// Multipliers for a block exponent s: code * 2^-120 * m1 * m2 = code * 2^s,
+// with m1 = 2^(120 + min(s, 7)) and m2 = 2^(s - min(s, 7)), both normal bf16
+// numbers for s in [-124, 127]; each product is exact (a power-of-two scaling
+// of a value with at most four significant bits inside bf16's range).
+struct Fp8Scale {
+    __nv_bfloat162 m1, m2;
+};
+
+__device__ __forceinline__ __nv_bfloat162 bf16x2_pow2(int e) {
+    // 2^e, -126 <= e <= 127: exponent field e + 127, zero mantissa, both lanes
+    const uint32_t b = static_cast<uint32_t>(e + 127) << 7;
+    const uint32_t w = b | (b << 16);
+    return *reinterpret_cast<const __nv_bfloat162*>(&w);
+}
+
+__device__ __forceinline__ Fp8Scale fp8_scale(int s) {
+    const int a = min(s, 7);
+    return Fp8Scale{bf16x2_pow2(120 + a), bf16x2_pow2(s - a)};
+}
+
+// Eight E4M3 codes (little-endian in `v`) -> eight bf16 values code * 2^s, exact.
+__device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 v, const Fp8Scale& sc) {
+    uint32_t w[4];
+    fp8x4_to_bf16x4_pow2m120(v.x, w[0], w[1]);
+    fp8x4_to_bf16x4_pow2m120(v.y, w[2], w[3]);
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        const __nv_bfloat162 y = __hmul2(__hmul2(x, sc.m1), sc.m2);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+    }
+    return out;
+}
+
+}  // namespace moe

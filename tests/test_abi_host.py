@@ -103,3 +103,44 @@ def test_combine_rejects_bad_shapes():
     assert L.moe_combine(FAKE, NULL, FAKE, FAKE, 4, 12, 4, FAKE, NULL) == SHAPE
     assert L.moe_combine(FAKE, NULL, FAKE, FAKE, 4, 512, 33, FAKE, NULL) == SHAPE
     assert L.moe_combine(NULL, NULL, FAKE, FAKE, 4, 512, 4, FAKE, NULL) == INVALID
+
+
+# ------------------------------------------------------------ FP8 weights
+
+def _layer_fp8(T=64, d=7168, E=384, k=8, inter=2048, scale=2.827, ptrs=None, out=FAKE, ws=None):
+    p = ptrs if ptrs is not None else [FAKE] * 9
+    L = moe.lib()
+    if ws is None:
+        return L.moe_layer_forward_fp8(*p, T, d, E, k, inter, ctypes.c_float(scale), out, NULL)
+    return L.moe_layer_forward_fp8_ws(*p, T, d, E, k, inter, ctypes.c_float(scale), out, FAKE, ws,
+                                      NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=7104), SHAPE), (dict(inter=2112), SHAPE), (dict(d=7100), SHAPE), (dict(E=0), SHAPE),
+    (dict(k=9, E=8), SHAPE), (dict(T=-1), INVALID), (dict(scale=float("nan")), INVALID),
+])
+def test_fp8_layer_rejects_bad_shapes(kw, code):
+    # FP8 blocks are 128 x 128: d and inter must be multiples of 128, not just 64
+    assert _layer_fp8(**kw) == code
+
+
+def test_fp8_layer_rejects_null_pointers_and_small_workspace():
+    for i in range(9):
+        p = [FAKE] * 9
+        p[i] = NULL
+        assert _layer_fp8(ptrs=p) == INVALID
+    assert _layer_fp8(out=NULL) == INVALID
+    need = moe.moe_workspace_size(64, 7168, 384, 8, 2048)
+    assert _layer_fp8(ws=need - 1) == INVALID
+    assert _layer_fp8(T=0) == OK
+
+
+def test_quantize_fp8_rejects_bad_shapes():
+    L = moe.lib()
+    assert L.moe_quantize_fp8(FAKE, 100, 128, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_fp8(FAKE, 128, 100, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_fp8(FAKE, 128, 128 * 65536, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_fp8(FAKE, 0, 128, FAKE, FAKE, NULL) == OK
+    assert L.moe_quantize_fp8(NULL, 128, 128, FAKE, FAKE, NULL) == INVALID
+    assert L.moe_quantize_fp8(FAKE, 128, 128, FAKE, NULL, NULL) == INVALID
