@@ -20,6 +20,9 @@
 //   warps 2..9  epilogue: two warps per TMEM lane quarter, each taking every
 //               other 32-column chunk; tcgen05.ld 32 lanes x 32 columns,
 //               convert, store
+// FP8-weight mode (480 threads): warps 2..5 are the epilogue (one per lane
+// quarter, every chunk), warps 6..9 and 11..14 dequantize E4M3 weight codes
+// into the bf16 weight ring (convert_weights).
 // Weights come from HBM and tokens mostly from L2, so the two operands have
 // separate rings: a deep one for weights (their HBM latency needs many bytes
 // in flight) and a short one for tokens.  K step q uses weight slot q % SA and
@@ -51,10 +54,13 @@ constexpr int kMaxN = 256;                    // MMA N limit (router tiles)
 constexpr int kTileN = 256;
 constexpr int kGemmThreads = 352;             // 11 warps: roles below
 constexpr int kTokenWarp = 10;
-// FP8-weight mode: four more warps dequantize the weight codes into the bf16 ring
-constexpr int kConvWarps = 4;
-constexpr int kConvWarp0 = 11;
-constexpr int kGemmThreadsFP8 = kGemmThreads + 32 * kConvWarps;
+// FP8-weight mode: 15 warps.  Warps 2..5 are the epilogue (one per TMEM lane
+// quarter, 4 instead of 8) and warps 6..9 and 11..14 dequantize the weight
+// codes into the bf16 ring (two converter warps per SM sub-partition).
+constexpr int kEpiWarpsFP8 = 4;
+constexpr int kConvWarps = 8;
+constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kGemmThreadsFP8 = 480;
 constexpr int kSlabBytes8 = kSlabRows * kBK;  // one FP8 slab per K step (128 rows x 64 codes)
 constexpr int kTmemCols = 512;
 
@@ -208,7 +214,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                                                 uint64_t tmo, int ntiles, int ct) {
     constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
     constexpr uint32_t a_bytes = nslab * kSlabBytes;
-    constexpr int kUnits = nslab * kSlabRows * (kBK / 8) / (32 * kConvWarps);   // per thread
+    constexpr int kUnits = nslab * kSlabRows * (kBK / 8) / kConvThreads;   // per thread
     const int lane = ct & 31;
     const uint64_t pol = ptx::policy_evict_first();
     Ring rq{0, 0, SA};          // bf16 slot of step q
@@ -233,7 +239,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 uint2 codes[kUnits];
 #pragma unroll
                 for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + 32 * kConvWarps * j;
+                    const int u = ct + kConvThreads * j;
                     const int slab = u / (kSlabRows * 8);
                     const int r = (u >> 3) & (kSlabRows - 1);
                     codes[j] = *reinterpret_cast<const uint2*>(src + slab * kSlabBytes8 + r * kBK +
@@ -241,7 +247,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 }
 #pragma unroll
                 for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + 32 * kConvWarps * j;
+                    const int u = ct + kConvThreads * j;
                     const int slab = u / (kSlabRows * 8);
                     const int r = (u >> 3) & (kSlabRows - 1);
                     const int c = u & 7;
@@ -252,7 +258,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 ptx::fence_proxy_async_smem();
             }
             // every converter thread reaches this barrier once per step
-            ok = ptx::bar_red_and(1, 32 * kConvWarps, w_ok);
+            ok = ptx::bar_red_and(1, kConvThreads, w_ok);
             if (!ok) break;
             if (ct == 0) {
                 if (routed) {
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
-            ptx::mbar_init(&acc_empty[b], kEpiWarps);
+            ptx::mbar_init(&acc_empty[b], FP8A ? kEpiWarpsFP8 : kEpiWarps);
         }
         ptx::mbar_init(drain, 1);
         for (int s = 0; s < SA8; ++s) {
@@ -523,14 +529,18 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                 wait_bounded(drain, 0, nullptr, tmo);
             }
         }
-    } else if (FP8A && warp >= kConvWarp0) {
+    } else if (FP8A && warp >= 2 + kEpiWarpsFP8) {
         // ---------------------------------------------------------- converters
         convert_weights<nslab>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
-                               abort_flag, tmo, ntiles, threadIdx.x - 32 * kConvWarp0);
+                               abort_flag, tmo, ntiles,
+                               32 * (warp < kTokenWarp ? warp - 6 : warp - 7) + lane);
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;          // which 32-column chunks it takes
+        // which 32-column chunks the warp takes: every other one when two warps
+        // share a lane quarter (bf16 mode), all of them in FP8 mode
+        const int half = FP8A ? 0 : (warp - 2) >> 2;
+        constexpr int kChunkStep = FP8A ? kStageRows : 2 * kStageRows;
         bf16* stg = staging + (warp - 2) * kStageRows * 32;
         uint32_t ab = 0, aphase = 0;
         for (int i = blockIdx.x; i < ntiles; i += gridDim.x) {
@@ -563,7 +573,7 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                 for (int s = 0; s < nout; ++s) {
                     const int fbase = t.out_col0 + s * kSlabRows + q * 32;
                     const uint32_t ts = tq + s * args.n_max;
-                    for (int c0 = kStageRows * half; c0 < npad; c0 += 2 * kStageRows) {
+                    for (int c0 = kStageRows * half; c0 < npad; c0 += kChunkStep) {
                         const int ncol = min(kStageRows, npad - c0);     // 32 or 16 (uniform)
                         float v[kStageRows];
                         if constexpr (kSwiGLU) {
