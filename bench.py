@@ -49,6 +49,9 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="k2_decode")
+    p.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                   help="routed experts' weight storage: bf16, or E4M3 codes with one "
+                        "power-of-two scale per 128x128 block (quantized once, untimed)")
     p.add_argument("--cpu-sample", type=int, default=None,
                    help="tokens in the oracle's timed sample (default: sized from the core count)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -157,7 +160,8 @@ def source_digest(paths):
 
 
 KERNEL_SOURCES = ["sparse_moe_ffn_sigmoid_b200/csrc/gemm.cuh", "sparse_moe_ffn_sigmoid_b200/csrc/ptx.cuh",
-                  "sparse_moe_ffn_sigmoid_b200/csrc/common.cuh"]
+                  "sparse_moe_ffn_sigmoid_b200/csrc/common.cuh",
+                  "sparse_moe_ffn_sigmoid_b200/csrc/quant.cuh"]
 
 
 def profiled_traffic(workload: str, kernel: str):
@@ -196,23 +200,30 @@ def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_total: float
 
 # ----------------------------------------------------- accounting (per step)
 
-def layer_accounting(cfg, touched: int):
+def layer_accounting(cfg, touched: int, weights: str = "bf16"):
     """Algorithmic bytes and FLOPs of one layer forward, and of its two GEMMs.
 
     touched: routed experts with at least one token this step (the shared
     expert is always touched on top).  Weight bytes per expert follow the
-    pages' 3 x d x inter parameter count ("Kimi K2.5 Q&A", Q2.1)."""
+    pages' 3 x d x inter parameter count ("Kimi K2.5 Q&A", Q2.1).  With FP8
+    storage a routed expert's weights are one byte each plus one int8 scale
+    per 128 x 128 block; the shared expert stays bf16."""
     T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
     rows = T * (k + 1)
     w_gu = 2 * I * d * 2                 # gate + up weights of one expert, bytes
     w_dn = d * I * 2
+    if weights == "fp8":
+        r_gu = 2 * I * d + (2 * I // 128) * (d // 128)
+        r_dn = d * I + (d // 128) * (I // 128)
+    else:
+        r_gu, r_dn = w_gu, w_dn
     acc = {}
-    acc["gate_up_bytes"] = (touched + 1) * w_gu + rows * d * 2 + rows * I * 2
-    acc["down_bytes"] = (touched + 1) * w_dn + rows * I * 2 + rows * d * 2
+    acc["gate_up_bytes"] = touched * r_gu + w_gu + rows * d * 2 + rows * I * 2
+    acc["down_bytes"] = touched * r_dn + w_dn + rows * I * 2 + rows * d * 2
     acc["gate_up_flops"] = 2.0 * rows * 2 * I * d
     acc["down_flops"] = 2.0 * rows * I * d
     acc["router_flops"] = 2.0 * T * d * E
-    acc["weight_bytes"] = (touched + 1) * (w_gu + w_dn) + E * d * 2
+    acc["weight_bytes"] = touched * (r_gu + r_dn) + (w_gu + w_dn) + E * d * 2
     acc["flops"] = acc["gate_up_flops"] + acc["down_flops"] + acc["router_flops"]
     return acc
 
@@ -225,7 +236,7 @@ class OracleSample:
     tokens select, the shared expert).  Rows are independent, so the oracle's
     tokens/s on the sample is its rate on the workload."""
 
-    def __init__(self, cfg, inputs_dev, n_tokens):
+    def __init__(self, cfg, inputs_dev, n_tokens, weights: str = "bf16"):
         import torch
         import oracle
         self.cfg = cfg
@@ -242,9 +253,14 @@ class OracleSample:
         self.need = sorted(set(ridx.reshape(-1).tolist()))
         self.egu = [None] * cfg.E
         self.edn = [None] * cfg.E
+        self.weights = weights
         for e in self.need:
             self.egu[e] = inputs_dev["w_gate_up"][e].cpu()
             self.edn[e] = inputs_dev["w_down"][e].cpu()
+            if weights == "fp8":
+                # the weights FP8 storage stands for, from the oracle's own quantizer
+                self.egu[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.egu[e]))
+                self.edn[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.edn[e]))
         self.sgu, self.sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
 
     def run(self) -> float:
@@ -258,13 +274,19 @@ class OracleSample:
         return time.perf_counter() - t0
 
     def describe(self) -> str:
+        fp8 = " (routed weights: the oracle's FP8 quantization, dequantized)" \
+            if self.weights == "fp8" else ""
         return (f"{len(self.tokens)} of {self.cfg.T} tokens (evenly spaced), full routing + "
-                f"{len(self.need)} routed experts + shared expert, fp64")
+                f"{len(self.need)} routed experts + shared expert, fp64{fp8}")
 
 
-def default_cpu_sample(cfg):
+def default_cpu_sample(cfg, weights: str = "bf16"):
     # ~0.8 GFLOP of fp64 per K2 token, one thread per token: 64 tokens keep a
-    # 16-core host busy for several seconds without copying every expert
+    # 16-core host busy for several seconds without copying every expert.
+    # With FP8 weights the oracle first quantizes every expert the sample
+    # selects (about a second each), so the sample is smaller.
+    if weights == "fp8":
+        return min(cfg.T, 8)
     return min(cfg.T, max(64, 4 * host_cores()))
 
 
@@ -311,9 +333,23 @@ def main(argv=None):
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    fp8 = args.weights == "fp8"
+    if fp8:
+        # storage format conversion, once, outside every timed region
+        qgu, egu = moe.moe_quantize_fp8(g["w_gate_up"])
+        qdn, edn = moe.moe_quantize_fp8(g["w_down"])
+        torch.cuda.synchronize(dev)
+
+    def layer(x_in):
+        if fp8:
+            moe.moe_layer_forward_fp8(x_in, g["w_router"], g["bias"], qgu, egu, qdn, edn,
+                                      g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+        else:
+            moe.moe_layer_forward(x_in, g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                                  g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+
     def step():
-        moe.moe_layer_forward(g["x"], g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
-                              g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+        layer(g["x"])
 
     for _ in range(args.warmup):
         step()
@@ -367,8 +403,7 @@ def main(argv=None):
 
         def e2e_step():
             x_dev.copy_(x_host, non_blocking=True)
-            moe.moe_layer_forward(x_dev, g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
-                                  g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+            layer(x_dev)
             out_host.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -389,7 +424,7 @@ def main(argv=None):
 
     # ---------------------------------------------------------- roofline
     peaks, peak_src = load_peaks()
-    acc = layer_accounting(cfg, touched)
+    acc = layer_accounting(cfg, touched, args.weights)
     kname = "gemm_gate_up_swiglu"
     k_ms = kernel_ms.get(kname, 0.0) / max(n_calls, 1)
     # decode and the DeepSeek-V3 shape stream weights (HBM roofline); prefill and
@@ -417,12 +452,13 @@ def main(argv=None):
                       "hbm_ideal_ms": t_hbm * 1e3, "hbm_frac": t_hbm / (ms_step / 1e3),
                       "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
                       "touched_experts": touched}
-    roof["traffic"] = profiled_traffic(args.workload, kname)
+    roof["traffic"] = profiled_traffic(args.workload + ("_fp8" if fp8 else ""), kname)
 
     # ---------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(cfg, g, args.cpu_sample or default_cpu_sample(cfg))
+        smp = OracleSample(cfg, g, args.cpu_sample or default_cpu_sample(cfg, args.weights),
+                           args.weights)
         dt = smp.run()
         cpu = {"value": len(smp.tokens) / dt, "unit": UNIT, "cores": smp.threads,
                "kind": "oracle", "sample": smp.describe(), "seconds": dt}
@@ -435,6 +471,7 @@ def main(argv=None):
             "config": {"workload": args.workload + "".join(f" {x}" for x in args.set),
                        "T": T, "d": d, "E": E, "k": k, "inter": I,
                        "scale": cfg.scale, "bias": cfg.bias, "parallelism": f"replicas{world}",
+                       "weights": "fp8_e4m3_block128_pow2" if fp8 else "bf16",
                        "l2": "inputs larger than L2: every step streams "
                              f"{acc['weight_bytes'] / 1e9:.1f} GB of expert weights"},
             "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
