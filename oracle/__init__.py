@@ -82,6 +82,10 @@ def _bind(L):
     L.oracle_quantize_fp8.restype = i32
     L.oracle_dequantize_fp8.argtypes = [P, P, i64, i64, P]
     L.oracle_dequantize_fp8.restype = i32
+    L.oracle_bias_update.argtypes = [P, i32, i32, i32, ctypes.c_float, P]
+    L.oracle_bias_update.restype = None
+    L.oracle_seq_aux_loss.argtypes = [P, P, i32, i32, i32, i32, f64, P, P, P]
+    L.oracle_seq_aux_loss.restype = None
     return L
 
 
@@ -164,6 +168,29 @@ def dequantize_fp8(q, sexp):
     if rc != 0:
         raise ValueError("oracle_dequantize_fp8: rows and cols must be multiples of 128")
     return out
+
+
+def bias_update(counts, T: int, k: int, gamma: float, bias):
+    """New fp32 bias after one loss-free balancing step (see the C header)."""
+    c = _np(counts, np.int32)
+    b = np.array(_np(bias, np.float32), copy=True)
+    lib().oracle_bias_update(_ptr(c), int(T), c.size, int(k), float(gamma), _ptr(b))
+    return b
+
+
+def seq_aux_loss(scores, topk_idx, S: int, alpha: float):
+    """Sequence-level balance loss per sequence of S tokens -> (loss [B], f [B,E], p [B,E])."""
+    sc = _np(scores, np.float64)
+    idx = _np(topk_idx, np.int32)
+    T, E = sc.shape
+    k = idx.shape[1]
+    B = T // S
+    loss = np.empty(B)
+    f = np.empty((B, E))
+    p = np.empty((B, E))
+    lib().oracle_seq_aux_loss(_ptr(sc), _ptr(idx), B, int(S), E, k, float(alpha), _ptr(loss),
+                              _ptr(f), _ptr(p))
+    return loss, f, p
 
 
 def sigmoid(z: float) -> float:

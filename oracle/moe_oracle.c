@@ -361,3 +361,44 @@ int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, in
                 ldexp(oracle_e4m3_decode(q[r * cols + c]), sexp[(r / 128) * bc + c / 128]));
     return 0;
 }
+
+/* ------------------------------------------------------------ load balance */
+
+void oracle_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias) {
+    const long long total = (long long)T * k;
+    for (int e = 0; e < E; ++e) {
+        const long long scaled = (long long)counts[e] * E;     /* load vs mean, exactly */
+        float b = bias[e];
+        if (scaled > total)
+            b = b - gamma;                                    /* over-loaded: lower */
+        else if (scaled < total)
+            b = b + gamma;                                    /* under-loaded: raise */
+        bias[e] = b;
+    }
+}
+
+void oracle_seq_aux_loss(const double* scores, const int32_t* topk_idx, int B, int S, int E,
+                         int k, double alpha, double* loss, double* f, double* p) {
+    double* fb = (double*)calloc((size_t)E, sizeof(double));
+    double* pb = (double*)calloc((size_t)E, sizeof(double));
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < E; ++i) fb[i] = pb[i] = 0.0;
+        for (int t = b * S; t < (b + 1) * S; ++t) {
+            for (int j = 0; j < k; ++j) fb[topk_idx[(size_t)t * k + j]] += 1.0;
+            double tot = 0.0;
+            for (int i = 0; i < E; ++i) tot += scores[(size_t)t * E + i];
+            for (int i = 0; i < E; ++i) pb[i] += scores[(size_t)t * E + i] / tot;
+        }
+        double l = 0.0;
+        for (int i = 0; i < E; ++i) {
+            fb[i] *= (double)E / ((double)k * S);
+            pb[i] /= S;
+            l += fb[i] * pb[i];
+            if (f) f[(size_t)b * E + i] = fb[i];
+            if (p) p[(size_t)b * E + i] = pb[i];
+        }
+        loss[b] = alpha * l;
+    }
+    free(fb);
+    free(pb);
+}

@@ -145,6 +145,33 @@ int oracle_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* 
 int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, int64_t cols,
                           uint16_t* w_out);
 
+/*
+ * Load balancing ("Kimi K2.5 Q&A", Q7.2; "Kimi K2.5 deep dive", CH10.2 step 2).
+ *
+ * Bias update (noaux_tc): the selection bias is a buffer, not learned; after a
+ * step, experts that took more than their share of the step's T*k routed rows
+ * have their bias lowered by gamma, experts that took less have it raised, and
+ * an expert exactly at the mean T*k/E keeps it.  The pages give neither the
+ * rate nor the comparison; the reading: a fixed step gamma (an argument), the
+ * load compared with the mean exactly (counts[e]*E against T*k), the update
+ * done in the buffer's own precision: bias[e] = fp32(bias[e] -/+ gamma).
+ */
+void oracle_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias);
+
+/*
+ * Sequence-level auxiliary balance loss (seq_aux = true, aux_loss_alpha).  The
+ * pages name it and give alpha = 0.001 but not the formula; the reading is the
+ * sequence-wise balance loss of the DeepSeek-V3 line the pages say K2 continues:
+ * for each sequence b of S tokens,
+ *   f_i = E / (k * S) * #{t in b : i in topk(t)}
+ *   P_i = (1 / S) * sum_{t in b} s_{t,i} / sum_j s_{t,j}     (sigmoid affinities)
+ *   L_b = alpha * sum_i f_i * P_i
+ * scores [B*S, E] (sigmoid s), topk_idx [B*S, k]; out: loss [B], and optionally
+ * f [B, E], p [B, E].  fp64 throughout.
+ */
+void oracle_seq_aux_loss(const double* scores, const int32_t* topk_idx, int B, int S, int E,
+                         int k, double alpha, double* loss, double* f, double* p);
+
 #ifdef __cplusplus
 }
 #endif

@@ -398,12 +398,86 @@ def pin_fp8_quantize_bounds():
             top = np.abs(wq[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]).max()
             assert 224.0 <= top / 2.0 ** sexp[i, j] <= 448.0
 
+
+# ---------------------------------------------------------- load balancing
+# "Kimi K2.5 Q&A", Q7.2 and "Kimi K2.5 deep dive", CH10.2 step 2: the selection
+# bias is a non-learned buffer lowered for over-loaded and raised for
+# under-loaded experts; a weak sequence-level balance loss (alpha = 0.001).
+
+def pin_bias_update_worked_example():
+    """Hand-computed steps: loads against the exact mean T*k/E, fp32 buffer."""
+    b = oracle.bias_update(np.array([3, 1, 2, 2]), T=4, k=2, gamma=0.125,
+                           bias=np.array([0.0, 0.0, 0.5, -0.25], np.float32))
+    assert np.array_equal(b, np.array([-0.125, 0.125, 0.5, -0.25], np.float32))
+    # mean 7/3 is not an integer: 2 < 7/3 < 3, none sits at the mean
+    b = oracle.bias_update(np.array([3, 2, 2]), T=7, k=1, gamma=0.5,
+                           bias=np.zeros(3, np.float32))
+    assert np.array_equal(b, np.array([-0.5, 0.5, 0.5], np.float32))
+    # the update is made in fp32: 1 + 2^-25 rounds back to 1
+    b = oracle.bias_update(np.array([0, 2]), T=2, k=1, gamma=2.0 ** -25,
+                           bias=np.array([1.0, 1.0], np.float32))
+    assert b[0] == np.float32(1.0) and b[1] == np.float32(1.0)
+
+
+def pin_bias_update_invariants():
+    rng = np.random.default_rng(5)
+    for _ in range(20):
+        E = int(rng.integers(2, 64))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        T = int(rng.integers(1, 200))
+        counts = np.bincount(rng.integers(0, E, T * k), minlength=E)
+        bias = (rng.integers(-64, 64, E) * 2.0 ** -10).astype(np.float32)
+        gamma = 2.0 ** -7
+        nb = oracle.bias_update(counts, T, k, gamma, bias)
+        d = nb.astype(np.float64) - bias
+        over = counts * E > T * k
+        under = counts * E < T * k
+        assert np.all(d[over] == -gamma) and np.all(d[under] == gamma)
+        assert np.all(d[~over & ~under] == 0.0)
+
+
+def pin_bias_update_moves_load():
+    """Lowering an over-loaded expert's bias (and raising the others' by at most
+    gamma) cannot give it more tokens, and the least-loaded expert cannot lose
+    any: checked with the oracle's own router."""
+    x, wr, bias = _rand_router(96, 64, 16, seed=77)
+    k = 4
+    idx, _, _ = oracle.route(x, wr, bias, k, K2_SCALE)
+    counts = np.bincount(idx.reshape(-1), minlength=16)
+    nb = oracle.bias_update(counts, 96, k, 0.05, bias.numpy() if hasattr(bias, "numpy") else bias)
+    idx2, _, _ = oracle.route(x, wr, torch.as_tensor(nb), k, K2_SCALE)
+    c2 = np.bincount(idx2.reshape(-1), minlength=16)
+    hi, lo = int(np.argmax(counts)), int(np.argmin(counts))
+    assert c2[hi] <= counts[hi] and c2[lo] >= counts[lo]
+    assert c2[hi] < counts[hi] or c2[lo] > counts[lo]      # and the step does move load
+
+
+def pin_seq_aux_loss_closed_forms():
+    alpha = 0.001
+    # uniform affinities and a perfectly even selection: f_i = 1, P_i = 1/E, L = alpha
+    E, k, S = 8, 2, 4
+    scores = np.full((S, E), 0.3)
+    idx = np.array([[0, 1], [2, 3], [4, 5], [6, 7]], np.int32)
+    loss, f, p = oracle.seq_aux_loss(scores, idx, S, alpha)
+    assert abs(loss[0] - alpha) < 1e-15 and np.allclose(f, 1.0) and np.allclose(p, 1.0 / E)
+    # hand example: E=4, k=1, S=2, both tokens pick expert 0
+    sc = np.array([[0.5, 0.5, 0.5, 0.5], [0.6, 0.2, 0.1, 0.1]])
+    loss, f, p = oracle.seq_aux_loss(sc, np.array([[0], [0]], np.int32), 2, alpha)
+    assert np.allclose(f[0], [4.0, 0.0, 0.0, 0.0]) and np.allclose(p[0], [0.425, 0.225, 0.175, 0.175])
+    assert abs(loss[0] - 1.7 * alpha) < 1e-15
+    # each sequence on its own; a token's affinities matter only up to a factor
+    sc2 = np.concatenate([sc, sc * np.array([[3.0], [0.5]])])
+    loss2, _, _ = oracle.seq_aux_loss(sc2, np.array([[0], [0], [0], [0]], np.int32), 2, alpha)
+    assert np.allclose(loss2, [1.7 * alpha, 1.7 * alpha], rtol=0, atol=1e-15)
+
 ALL_PINS = [pin_bf16_rounding, pin_sigmoid_silu, pin_route_worked_example,
             pin_router_scores_library, pin_topk_brute_force, pin_exact_ties,
             pin_weights_closed_form, pin_bias_selection_only, pin_permute_brute_force,
             pin_swiglu_textbook, pin_dense_vs_sparse, pin_special_cases,
             pin_row_independence, pin_combine, pin_fp8_decode_library, pin_fp8_anchor_values,
-            pin_fp8_encode_library, pin_fp8_block_exponent_brute_force, pin_fp8_quantize_bounds]
+            pin_fp8_encode_library, pin_fp8_block_exponent_brute_force, pin_fp8_quantize_bounds,
+            pin_bias_update_worked_example, pin_bias_update_invariants, pin_bias_update_moves_load,
+            pin_seq_aux_loss_closed_forms]
 
 
 def failing_pins():

@@ -63,6 +63,13 @@ MUTANTS = [
      "q[r * cols + c] = oracle_e4m3_encode(ldexp(oracle_bf16_to_f64(w[r * cols + c]), -2 * s));"),
     ("fp8_dequant_block_transposed", "sexp[(r / 128) * bc + c / 128]",
      "sexp[(r / 128) + (c / 128) * (rows / 128)]"),
+    ("bias_update_sign_flipped", "b = b - gamma;                                    /* over-loaded: lower */",
+     "b = b + gamma;                                    /* over-loaded: lower */"),
+    ("bias_update_truncated_mean",
+     "        else if (scaled < total)\n            b = b + gamma;",
+     "        else if ((long long)counts[e] < total / E)\n            b = b + gamma;"),
+    ("seq_aux_unnormalized", "pb[i] += scores[(size_t)t * E + i] / tot;", "pb[i] += scores[(size_t)t * E + i];"),
+    ("seq_aux_no_f_scale", "fb[i] *= (double)E / ((double)k * S);", "fb[i] *= 1.0;"),
 ]
 
 
