@@ -248,6 +248,54 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Expert load balancing ("Kimi K2.5 Q&A", Q7.2; "Kimi K2.5 deep dive", CH10.2
+ * step 2): the selection bias is a buffer outside the gradient, lowered for
+ * over-loaded experts and raised for under-loaded ones, and a weak
+ * sequence-level balance loss (aux_loss_alpha = 0.001 in the pages) backs it up.
+ *
+ * moe_bias_update: one loss-free balancing step from a step's loads.
+ *   counts [E] int32 device  rows each expert received (moe_permute's counts;
+ *                           they sum to T*k)
+ *   bias   [E] fp32  device  updated in place, in fp32:
+ *       bias[e] -= gamma  if counts[e] * E > T * k   (above the mean load)
+ *       bias[e] += gamma  if counts[e] * E < T * k   (below it)
+ *       unchanged         if counts[e] * E == T * k
+ * The pages give no rate; gamma is the caller's.  Asynchronous on `stream`.
+ * Errors: MOE_ERR_UNSUPPORTED_SHAPE for E or k out of range, MOE_ERR_INVALID_ARG
+ * for T < 0, null pointers or a NaN gamma.  T == 0 changes nothing.
+ */
+int moe_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias,
+                    void* stream);
+
+/*
+ * moe_router_scores: the unbiased sigmoid scores of every expert,
+ *   scores[t, e] = sigmoid(x[t] . w_router[e])   [T, E] fp32, device,
+ * the same fp32 values the top-k selection of moe_route starts from (fp32
+ * accumulation over d, split-K partials added in a fixed order).  Scratch:
+ * workspace of moe_workspace_size(T, d, E, k, inter) bytes for any k, inter.
+ * Errors as in moe_route.
+ */
+int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d, int E,
+                      float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_seq_aux_loss: the sequence-level balance loss over B sequences of S
+ * tokens (rows b*S .. b*S+S-1).  The pages give alpha but no formula; this is
+ * the sequence-wise balance loss of the DeepSeek-V3 line that K2 continues:
+ *   f_i = E / (k S) * #{t in sequence : i in topk(t)}
+ *   P_i = (1 / S) * sum_t scores[t, i] / sum_j scores[t, j]
+ *   loss[b] = alpha * sum_i f_i * P_i
+ *   scores [B*S, E] fp32 (moe_router_scores), topk_idx [B*S, k] int32 (moe_route);
+ *   loss [B] fp32; f, p [B, E] fp32 or NULL; all device memory.
+ * fp32 with fixed reduction orders (deterministic).  Errors:
+ * MOE_ERR_UNSUPPORTED_SHAPE for E or k out of range or E*4 + S*4 > 48 KiB,
+ * MOE_ERR_INVALID_ARG for B < 0, S < 1, null pointers, NaN alpha; an
+ * out-of-range index is recorded in the device status and skipped.
+ */
+int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
+                     float alpha, float* loss, float* f, float* p, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word:
  * *device_status = MOE_OK, or the first problem a kernel recorded since the
  * last read (MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT).  Returns MOE_OK or

@@ -21,7 +21,8 @@ __all__ = [
     "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
     "moe_layer_forward_noalloc", "moe_quantize_fp8", "moe_layer_forward_fp8",
-    "moe_layer_forward_fp8_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "moe_layer_forward_fp8_ws", "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
+    "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
@@ -31,6 +32,7 @@ EXPORTED_SYMBOLS = [
     "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
     "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
+    "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
 ]
 
 MOE_OK = 0
@@ -69,6 +71,9 @@ def _load():
         "moe_layer_forward_fp8": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P], I),
         "moe_layer_forward_fp8_ws": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, SZ, P],
                                      I),
+        "moe_bias_update": ([P, I, I, I, F, P, P], I),
+        "moe_router_scores": ([P, P, I, I, I, P, P, SZ, P], I),
+        "moe_seq_aux_loss": ([P, P, I, I, I, I, F, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -256,6 +261,38 @@ def moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_d
                                        _ptr(workspace, torch.uint8, "workspace"),
                                        workspace.numel(), _stream(stream))
     _check("moe_layer_forward_fp8_ws", rc)
+
+
+def moe_bias_update(counts, T: int, k: int, gamma: float, bias, stream=None):
+    """One loss-free balancing step on `bias` (fp32 [E], in place) from the
+    step's per-expert row counts (int32 [E])."""
+    E = counts.numel()
+    rc = _LIB.moe_bias_update(_ptr(counts, I32, "counts"), int(T), E, int(k), float(gamma),
+                              _ptr(bias, F32, "bias"), _stream(stream))
+    _check("moe_bias_update", rc)
+
+
+def moe_router_scores(x, w_router, scores, workspace, stream=None):
+    """Unbiased sigmoid router scores of every expert into scores [T, E] fp32."""
+    T, d = x.shape
+    E = w_router.shape[0]
+    rc = _LIB.moe_router_scores(_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"), T, d, E,
+                                _ptr(scores, F32, "scores"),
+                                _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                _stream(stream))
+    _check("moe_router_scores", rc)
+
+
+def moe_seq_aux_loss(scores, topk_idx, S: int, alpha: float, loss, f=None, p=None, stream=None):
+    """Sequence-level balance loss of the B = T / S sequences into loss [B]
+    (and f, p [B, E] if given)."""
+    T, E = scores.shape
+    k = topk_idx.shape[1]
+    rc = _LIB.moe_seq_aux_loss(_ptr(scores, F32, "scores"), _ptr(topk_idx, I32, "topk_idx"),
+                               T // S, int(S), E, k, float(alpha), _ptr(loss, F32, "loss"),
+                               _ptr(f, F32, "f", optional=True), _ptr(p, F32, "p", optional=True),
+                               _stream(stream))
+    _check("moe_seq_aux_loss", rc)
 
 
 def moe_device_status(stream=None) -> int:

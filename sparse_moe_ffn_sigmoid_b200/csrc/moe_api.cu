@@ -17,6 +17,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "balance.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -282,9 +283,9 @@ int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const float* bias, int T,
-                 int d, int E, int k, float scale, int* idx, float* w, float* partials,
-                 int splits, cudaStream_t st, Recorder& rec) {
+// Router GEMM: fp32 logit partials [splits, T, E] (split-K over d).
+int launch_router_gemm(const DeviceInfo& di, const bf16* x, const bf16* wr, int T, int d, int E,
+                       float* partials, int splits, cudaStream_t st) {
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     const int nt = (T + kMaxN - 1) / kMaxN;
@@ -307,7 +308,13 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
     a.out_ld = E;
     a.col_limit = E;
     fill_pipeline(a, 1, chunk);
-    int rc = launch_gemm<kEpiStoreF32, false>(a, std::min(a.ntiles_host, di.sms), st);
+    return launch_gemm<kEpiStoreF32, false>(a, std::min(a.ntiles_host, di.sms), st);
+}
+
+int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const float* bias, int T,
+                 int d, int E, int k, float scale, int* idx, float* w, float* partials,
+                 int splits, cudaStream_t st, Recorder& rec) {
+    int rc = launch_router_gemm(di, x, wr, T, d, E, partials, splits, st);
     if (rc != MOE_OK) return rc;
     rec.mark(st);
     const int npl = (E + 31) / 32;
@@ -814,6 +821,55 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
     return moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
                                     wq_down_exp, ws_gate_up, ws_down, T, d, E, k, inter, scale,
                                     out, ws, need, stream);
+}
+
+int moe_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias,
+                    void* stream) {
+    if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (counts == nullptr || bias == nullptr || !(gamma == gamma)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;           // no rows routed: every expert sits at the mean
+    bias_update_kernel<<<(E + kBalanceThreads - 1) / kBalanceThreads, kBalanceThreads, 0,
+                         static_cast<cudaStream_t>(stream)>>>(
+        counts, static_cast<long long>(T) * k, E, gamma, bias);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d, int E,
+                      float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, 1, 64);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, scores, workspace)) return MOE_ERR_INVALID_ARG;
+    const int splits = router_splits(T, d, E);
+    if (workspace_bytes < static_cast<size_t>(splits) * T * E * sizeof(float))
+        return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* partials = static_cast<float*>(workspace);
+    rc = launch_router_gemm(di, reinterpret_cast<const bf16*>(x),
+                            reinterpret_cast<const bf16*>(w_router), T, d, E, partials, splits, st);
+    if (rc != MOE_OK) return rc;
+    const long long n = static_cast<long long>(T) * E;
+    router_scores_kernel<<<static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads),
+                           kBalanceThreads, 0, st>>>(partials, splits, n, n, scores);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
+                     float alpha, float* loss, float* f, float* p, void* stream) {
+    if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (B < 0 || S < 1) return MOE_ERR_INVALID_ARG;
+    const size_t smem = static_cast<size_t>(E) * sizeof(int) + static_cast<size_t>(S) * sizeof(float);
+    if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED_SHAPE;     // S up to ~11.5k tokens
+    if (B == 0) return MOE_OK;
+    if (scores == nullptr || topk_idx == nullptr || loss == nullptr || !(alpha == alpha))
+        return MOE_ERR_INVALID_ARG;
+    seq_aux_loss_kernel<<<B, kBalanceThreads, smem, static_cast<cudaStream_t>(stream)>>>(
+        scores, topk_idx, S, E, k, alpha, loss, f, p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int moe_device_status(void* stream, int* device_status) {

@@ -144,3 +144,25 @@ def test_quantize_fp8_rejects_bad_shapes():
     assert L.moe_quantize_fp8(FAKE, 0, 128, FAKE, FAKE, NULL) == OK
     assert L.moe_quantize_fp8(NULL, 128, 128, FAKE, FAKE, NULL) == INVALID
     assert L.moe_quantize_fp8(FAKE, 128, 128, FAKE, NULL, NULL) == INVALID
+
+
+# ------------------------------------------------------------ load balance
+
+def test_balance_calls_reject_bad_arguments():
+    L = moe.lib()
+    f = ctypes.c_float
+    assert L.moe_bias_update(FAKE, 64, 0, 8, f(1e-3), FAKE, NULL) == SHAPE
+    assert L.moe_bias_update(FAKE, 64, 384, 33, f(1e-3), FAKE, NULL) == SHAPE
+    assert L.moe_bias_update(FAKE, -1, 384, 8, f(1e-3), FAKE, NULL) == INVALID
+    assert L.moe_bias_update(NULL, 64, 384, 8, f(1e-3), FAKE, NULL) == INVALID
+    assert L.moe_bias_update(FAKE, 64, 384, 8, f(float("nan")), FAKE, NULL) == INVALID
+    assert L.moe_bias_update(FAKE, 0, 384, 8, f(1e-3), FAKE, NULL) == OK
+    assert L.moe_router_scores(FAKE, FAKE, 64, 7100, 384, FAKE, FAKE, 1 << 30, NULL) == SHAPE
+    assert L.moe_router_scores(FAKE, FAKE, 64, 7168, 384, FAKE, FAKE, 16, NULL) == INVALID
+    assert L.moe_router_scores(FAKE, FAKE, 0, 7168, 384, FAKE, FAKE, 0, NULL) == OK
+    assert L.moe_seq_aux_loss(FAKE, FAKE, 4, 64, 2048, 8, f(1e-3), FAKE, NULL, NULL, NULL) == SHAPE
+    assert L.moe_seq_aux_loss(FAKE, FAKE, 1, 20000, 384, 8, f(1e-3), FAKE, NULL, NULL,
+                              NULL) == SHAPE
+    assert L.moe_seq_aux_loss(FAKE, FAKE, 4, 0, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == INVALID
+    assert L.moe_seq_aux_loss(NULL, FAKE, 4, 64, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == INVALID
+    assert L.moe_seq_aux_loss(FAKE, FAKE, 0, 64, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == OK
