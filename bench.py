@@ -49,6 +49,10 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="k2_decode")
+    p.add_argument("--balance", type=int, default=0, metavar="S",
+                   help="time the load-balancing pass instead of the layer: router scores, "
+                        "route, permute, the sequence-level loss over sequences of S tokens "
+                        "and the bias update")
     p.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
                    help="routed experts' weight storage: bf16, or E4M3 codes with one "
                         "power-of-two scale per 128x128 block (quantized once, untimed)")
@@ -317,6 +321,8 @@ def main(argv=None):
         if rank != 0:
             return 0
         return run_reference(args, cfg, world)
+    if args.balance:
+        return run_balance(args, cfg)
 
     import torch
     import torch.distributed as dist
@@ -482,6 +488,83 @@ def main(argv=None):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_balance(args, cfg):
+    """One GPU, one line: the training-side load-balancing pass at the workload's
+    shape ("Kimi K2.5 Q&A", Q7.2): unbiased router scores, route, permute, the
+    sequence-level balance loss (sequences of S tokens) and the bias update.
+    The roofline line is the loss kernels' (token totals, per-block partial
+    sums, selection counts, finish): they read the [T, E] fp32 scores twice and
+    the [T, k] indices once."""
+    import torch
+    import sparse_moe_ffn_sigmoid_b200 as moe
+    from moe_inputs import make_inputs
+    S = args.balance
+    T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
+    if T % S:
+        raise SystemExit(f"--balance {S}: T = {T} is not a multiple of S")
+    B = T // S
+    dev = torch.device("cuda", 0)
+    g = make_inputs(cfg, seed=0, device=dev)
+    ws = torch.empty(moe.moe_workspace_size(T, d, E, k, I), dtype=torch.uint8, device=dev)
+    aux_ws = torch.empty(max(moe.moe_seq_aux_workspace_size(B, S, E), 16), dtype=torch.uint8,
+                         device=dev)
+    scores = torch.empty((T, E), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    i32 = lambda n: torch.empty((n,), dtype=torch.int32, device=dev)
+    counts, offs, rt, sr = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+    loss = torch.empty(B, dtype=torch.float32, device=dev)
+    bias = g["bias"].clone()
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    aux_ms = []
+
+    def step(timed):
+        moe.moe_router_scores(g["x"], g["w_router"], scores, ws)
+        moe.moe_route(g["x"], g["w_router"], bias, k, cfg.scale, idx, w, ws)
+        moe.moe_permute(idx, E, counts, offs, rt, sr, ws)
+        if timed:
+            ev[0].record(stream)
+        moe.moe_seq_aux_loss(scores, idx, S, 0.001, loss, workspace=aux_ws)
+        if timed:
+            ev[1].record(stream)
+        moe.moe_bias_update(counts, T, k, 1e-3, bias)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    steps = args.steps or 50
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step(True)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        aux_ms.append(ev[0].elapsed_time(ev[1]))
+    total_ms = t0.elapsed_time(t1)
+    if moe.moe_device_status() != 0:
+        raise SystemExit("device status not clean after the timed region")
+    peaks, peak_src = load_peaks()
+    aux_bytes = 2 * T * E * 4 + T * k * 4 + T * 4     # scores twice, indices, totals
+    a_ms = sum(aux_ms) / len(aux_ms)
+    achieved = aux_bytes / (a_ms / 1e3) / 1e9
+    line = {"metric": "load-balancing pass tokens/s (router scores, route, permute, "
+                      "sequence loss, bias update)",
+            "value": T * steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps,
+            "higher_is_better": True, "dtype": "fp32", "data": "synthetic",
+            "config": {"workload": args.workload, "T": T, "E": E, "k": k, "S": S, "B": B,
+                       "note": "each step synchronised to time the loss kernels"},
+            "roofline": {"bound": "hbm", "kernel": "seq_aux_loss (4 kernels)",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "avg_launch_ms": a_ms,
+                         "algorithmic_bytes_per_launch": aux_bytes,
+                         "peak_source": f"{peak_src} hbm_gbs", "traffic": None},
+            "loss": loss.cpu().tolist()}
+    print(json.dumps(line), flush=True)
     return 0
 
 

@@ -286,14 +286,17 @@ int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d,
  *   P_i = (1 / S) * sum_t scores[t, i] / sum_j scores[t, j]
  *   loss[b] = alpha * sum_i f_i * P_i
  *   scores [B*S, E] fp32 (moe_router_scores), topk_idx [B*S, k] int32 (moe_route);
- *   loss [B] fp32; f, p [B, E] fp32 or NULL; all device memory.
+ *   loss [B] fp32; f, p [B, E] fp32 or NULL; all device memory; workspace of
+ *   moe_seq_aux_workspace_size(B, S, E) bytes (16-byte aligned, caller-owned).
  * fp32 with fixed reduction orders (deterministic).  Errors:
- * MOE_ERR_UNSUPPORTED_SHAPE for E or k out of range or E*4 + S*4 > 48 KiB,
- * MOE_ERR_INVALID_ARG for B < 0, S < 1, null pointers, NaN alpha; an
- * out-of-range index is recorded in the device status and skipped.
+ * MOE_ERR_UNSUPPORTED_SHAPE for E or k out of range, MOE_ERR_INVALID_ARG for
+ * B < 0, S < 1, null pointers, NaN alpha or a short workspace; an out-of-range
+ * index is recorded in the device status and skipped.
  */
+size_t moe_seq_aux_workspace_size(int B, int S, int E);
 int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
-                     float alpha, float* loss, float* f, float* p, void* stream);
+                     float alpha, float* loss, float* f, float* p, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /*
  * Synchronise `stream`, then read and clear the current device's status word:

@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = [
     "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
     "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
-    "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
+    "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss", "moe_seq_aux_workspace_size",
 ]
 
 MOE_OK = 0
@@ -73,7 +73,8 @@ def _load():
                                      I),
         "moe_bias_update": ([P, I, I, I, F, P, P], I),
         "moe_router_scores": ([P, P, I, I, I, P, P, SZ, P], I),
-        "moe_seq_aux_loss": ([P, P, I, I, I, I, F, P, P, P, P], I),
+        "moe_seq_aux_loss": ([P, P, I, I, I, I, F, P, P, P, P, SZ, P], I),
+        "moe_seq_aux_workspace_size": ([I, I, I], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -283,14 +284,25 @@ def moe_router_scores(x, w_router, scores, workspace, stream=None):
     _check("moe_router_scores", rc)
 
 
-def moe_seq_aux_loss(scores, topk_idx, S: int, alpha: float, loss, f=None, p=None, stream=None):
+def moe_seq_aux_workspace_size(B: int, S: int, E: int) -> int:
+    return int(_LIB.moe_seq_aux_workspace_size(int(B), int(S), int(E)))
+
+
+def moe_seq_aux_loss(scores, topk_idx, S: int, alpha: float, loss, f=None, p=None,
+                     workspace=None, stream=None):
     """Sequence-level balance loss of the B = T / S sequences into loss [B]
-    (and f, p [B, E] if given)."""
+    (and f, p [B, E] if given); workspace: moe_seq_aux_workspace_size bytes
+    (allocated here if not given)."""
     T, E = scores.shape
     k = topk_idx.shape[1]
+    B = T // S
+    if workspace is None:
+        workspace = torch.empty(max(moe_seq_aux_workspace_size(B, S, E), 16), dtype=torch.uint8,
+                                device=scores.device)
     rc = _LIB.moe_seq_aux_loss(_ptr(scores, F32, "scores"), _ptr(topk_idx, I32, "topk_idx"),
-                               T // S, int(S), E, k, float(alpha), _ptr(loss, F32, "loss"),
+                               B, int(S), E, k, float(alpha), _ptr(loss, F32, "loss"),
                                _ptr(f, F32, "f", optional=True), _ptr(p, F32, "p", optional=True),
+                               _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                                _stream(stream))
     _check("moe_seq_aux_loss", rc)
 

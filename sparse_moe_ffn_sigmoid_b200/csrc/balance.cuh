@@ -11,6 +11,7 @@
 // of the DeepSeek-V3 line:
 //   f_i = E / (k S) #{t in seq : i in topk(t)},   P_i = mean_t s_ti / sum_j s_tj,
 //   L   = alpha sum_i f_i P_i.
+// All reductions run in fixed orders, so every run gives the same bits.
 #pragma once
 
 #include "common.cuh"
@@ -44,70 +45,96 @@ __global__ void __launch_bounds__(kBalanceThreads) router_scores_kernel(
     scores[i] = sigmoid_f32(acc);
 }
 
-// Fixed-shape block sum (deterministic): warp shuffles, then warp 0 over the
-// per-warp sums in warp order.
-__device__ __forceinline__ float block_sum(float v, float* scratch /*[32]*/) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+constexpr int kAuxExperts = 32;            // experts per block of the loss kernel
+constexpr int kAuxWarps = 8;
+
+// inv_tot[t] = 1 / sum_j scores[t, j]: one warp per token, lanes over experts,
+// a fixed-shape shuffle sum.
+__global__ void __launch_bounds__(kBalanceThreads) token_totals_kernel(
+    const float* __restrict__ scores, long long T, int E, float* __restrict__ inv_tot) {
+    const long long t = static_cast<long long>(blockIdx.x) * (kBalanceThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const float* row = scores + t * E;
+    float v = 0.0f;
+    for (int i = lane; i < E; i += 32) v += row[i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    __syncthreads();
-    if (lane == 0) scratch[w] = v;
-    __syncthreads();
-    float r = 0.0f;
-    if (w == 0) {
-        r = lane < static_cast<int>(blockDim.x >> 5) ? scratch[lane] : 0.0f;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
-        if (lane == 0) scratch[0] = r;
-    }
-    __syncthreads();
-    return scratch[0];
+    if (lane == 0) inv_tot[t] = 1.0f / v;
 }
 
-// One block per sequence b of S tokens.  Dynamic shared memory: E ints (the
-// selection counts) + S floats (each token's 1 / sum_j s_tj).
-__global__ void __launch_bounds__(kBalanceThreads) seq_aux_loss_kernel(
-    const float* __restrict__ scores, const int* __restrict__ topk_idx, int S, int E, int k,
-    float alpha, float* __restrict__ loss, float* __restrict__ f_out, float* __restrict__ p_out) {
-    extern __shared__ int bal_smem[];
-    int* cnt = bal_smem;
-    float* inv_tot = reinterpret_cast<float*>(bal_smem + E);
-    __shared__ float scratch[32];
-    const long long t0 = static_cast<long long>(blockIdx.x) * S;
-    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+constexpr int kAuxTokens = 256;            // tokens per block of the loss kernel
+
+// Block (b, c, s): experts i = 32 c + lane of sequence b over its tokens
+// [256 s, 256 s + 256).  Warp w sums 32 consecutive tokens (coalesced 128-byte
+// rows of scores), the warps' sums are added in warp order into
+// part[(b * nsplit + s) * E + i] = sum_t scores[t, i] / sum_j scores[t, j].
+__global__ void __launch_bounds__(32 * kAuxWarps) seq_aux_partial_kernel(
+    const float* __restrict__ scores, const float* __restrict__ inv_tot, int S, int E,
+    float* __restrict__ part) {
+    __shared__ float sp[kAuxWarps][kAuxExperts];
+    const int b = blockIdx.x, c = blockIdx.y, sblk = blockIdx.z;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int i = c * kAuxExperts + lane;
+    const long long t0 = static_cast<long long>(b) * S;
+    const int tb = sblk * kAuxTokens + w * (kAuxTokens / kAuxWarps);
+    const int te = min(S, tb + kAuxTokens / kAuxWarps);
+    float acc = 0.0f;
+    if (i < E)
+        for (int t = tb; t < te; ++t) acc = fmaf(scores[(t0 + t) * E + i], inv_tot[t0 + t], acc);
+    sp[w][lane] = acc;
     __syncthreads();
-    // selection counts (integer atomics: order-free) and per-token totals
-    for (long long j = threadIdx.x; j < static_cast<long long>(S) * k; j += blockDim.x) {
-        const int e = topk_idx[t0 * k + j];
-        if (e >= 0 && e < E)
-            atomicAdd(&cnt[e], 1);
-        else
-            record_status(kStatusInvalidArg);
-    }
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int t = w; t < S; t += nw) {
-        const float* row = scores + (t0 + t) * E;
+    if (w == 0 && i < E) {
         float v = 0.0f;
-        for (int i = lane; i < E; i += 32) v += row[i];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) inv_tot[t] = 1.0f / v;
+        for (int ww = 0; ww < kAuxWarps; ++ww) v += sp[ww][lane];
+        part[(static_cast<long long>(b) * gridDim.z + sblk) * E + i] = v;
     }
-    __syncthreads();
-    // thread i: f_i and P_i (tokens in order), then the block sum of f_i P_i
-    float part = 0.0f;
+}
+
+// cnt[b * E + e] += 1 for every selection of sequence b (integer atomics).
+__global__ void __launch_bounds__(kBalanceThreads) seq_aux_count_kernel(
+    const int* __restrict__ topk_idx, long long n, int Sk, int E, int* __restrict__ cnt) {
+    const long long j = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (j >= n) return;
+    const int e = topk_idx[j];
+    if (e < 0 || e >= E) {
+        record_status(kStatusInvalidArg);
+        return;
+    }
+    atomicAdd(&cnt[(j / Sk) * E + e], 1);
+}
+
+// One block per sequence: P_i = (sum over token blocks, in order) / S,
+// f_i = cnt * E / (k S), loss[b] = alpha * (fixed-shape block sum of f_i P_i).
+__global__ void __launch_bounds__(kBalanceThreads) seq_aux_finish_kernel(
+    const float* __restrict__ part, const int* __restrict__ cnt, int nsplit, int S, int E, int k,
+    float alpha, float* __restrict__ loss, float* __restrict__ f_out, float* __restrict__ p_out) {
+    __shared__ float scratch[32];
+    const int b = blockIdx.x;
     const float fscale = static_cast<float>(E) / (static_cast<float>(k) * S);
+    float acc = 0.0f;
     for (int i = threadIdx.x; i < E; i += blockDim.x) {
         float p = 0.0f;
-        for (int t = 0; t < S; ++t) p = fmaf(scores[(t0 + t) * E + i], inv_tot[t], p);
+        for (int s = 0; s < nsplit; ++s) p += part[(static_cast<long long>(b) * nsplit + s) * E + i];
         p /= static_cast<float>(S);
-        const float f = cnt[i] * fscale;
-        if (f_out) f_out[static_cast<long long>(blockIdx.x) * E + i] = f;
-        if (p_out) p_out[static_cast<long long>(blockIdx.x) * E + i] = p;
-        part = fmaf(f, p, part);
+        const float f = cnt[static_cast<long long>(b) * E + i] * fscale;
+        if (f_out) f_out[static_cast<long long>(b) * E + i] = f;
+        if (p_out) p_out[static_cast<long long>(b) * E + i] = p;
+        acc = fmaf(f, p, acc);
     }
-    const float total = block_sum(part, scratch);
-    if (threadIdx.x == 0) loss[blockIdx.x] = alpha * total;
+    // fixed-shape block sum
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) scratch[w] = acc;
+    __syncthreads();
+    if (w == 0) {
+        float r = lane < static_cast<int>(blockDim.x >> 5) ? scratch[lane] : 0.0f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+        if (lane == 0) loss[b] = alpha * r;
+    }
 }
 
 }  // namespace moe

@@ -823,6 +823,33 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
                                     out, ws, need, stream);
 }
 
+// Scratch of moe_seq_aux_loss: 1 / (token score sums) [B*S], the per-block
+// partial sums [B, ceil(S/256), E] and the selection counts [B, E] (int).
+struct AuxLayout {
+    size_t inv_tot, part, cnt, total;
+    int nsplit;
+};
+
+AuxLayout aux_layout(int B, int S, int E) {
+    AuxLayout L{};
+    const long long T = static_cast<long long>(B) * S;
+    L.nsplit = (S + kAuxTokens - 1) / kAuxTokens;
+    size_t off = 0;
+    L.inv_tot = off;
+    off = align256(off + static_cast<size_t>(T) * sizeof(float));
+    L.part = off;
+    off = align256(off + static_cast<size_t>(B) * L.nsplit * E * sizeof(float));
+    L.cnt = off;
+    off = align256(off + static_cast<size_t>(B) * E * sizeof(int));
+    L.total = off;
+    return L;
+}
+
+size_t moe_seq_aux_workspace_size(int B, int S, int E) {
+    if (B < 0 || S < 1 || E < 1 || E > 1024) return 0;
+    return aux_layout(B, S, E).total;
+}
+
 int moe_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias,
                     void* stream) {
     if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -859,16 +886,34 @@ int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d,
 }
 
 int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
-                     float alpha, float* loss, float* f, float* p, void* stream) {
+                     float alpha, float* loss, float* f, float* p, void* workspace,
+                     size_t workspace_bytes, void* stream) {
     if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (B < 0 || S < 1) return MOE_ERR_INVALID_ARG;
-    const size_t smem = static_cast<size_t>(E) * sizeof(int) + static_cast<size_t>(S) * sizeof(float);
-    if (smem > 48 * 1024) return MOE_ERR_UNSUPPORTED_SHAPE;     // S up to ~11.5k tokens
     if (B == 0) return MOE_OK;
-    if (scores == nullptr || topk_idx == nullptr || loss == nullptr || !(alpha == alpha))
+    if (scores == nullptr || topk_idx == nullptr || loss == nullptr || !(alpha == alpha) ||
+        !aligned16(workspace))
         return MOE_ERR_INVALID_ARG;
-    seq_aux_loss_kernel<<<B, kBalanceThreads, smem, static_cast<cudaStream_t>(stream)>>>(
-        scores, topk_idx, S, E, k, alpha, loss, f, p);
+    const AuxLayout L = aux_layout(B, S, E);
+    if (workspace_bytes < L.total || L.nsplit > 65535) return MOE_ERR_INVALID_ARG;
+    const long long T = static_cast<long long>(B) * S;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    float* inv_tot = reinterpret_cast<float*>(base + L.inv_tot);
+    float* part = reinterpret_cast<float*>(base + L.part);
+    int* cnt = reinterpret_cast<int*>(base + L.cnt);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(B) * E * sizeof(int), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    token_totals_kernel<<<static_cast<unsigned>((T + 7) / 8), kBalanceThreads, 0, st>>>(
+        scores, T, E, inv_tot);
+    const int nchunk = (E + kAuxExperts - 1) / kAuxExperts;
+    seq_aux_partial_kernel<<<dim3(B, nchunk, L.nsplit), 32 * kAuxWarps, 0, st>>>(scores, inv_tot,
+                                                                                S, E, part);
+    const long long n = T * k;
+    seq_aux_count_kernel<<<static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads),
+                           kBalanceThreads, 0, st>>>(topk_idx, n, S * k, E, cnt);
+    seq_aux_finish_kernel<<<B, kBalanceThreads, 0, st>>>(part, cnt, L.nsplit, S, E, k, alpha, loss,
+                                                         f, p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

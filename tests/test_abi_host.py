@@ -160,9 +160,11 @@ def test_balance_calls_reject_bad_arguments():
     assert L.moe_router_scores(FAKE, FAKE, 64, 7100, 384, FAKE, FAKE, 1 << 30, NULL) == SHAPE
     assert L.moe_router_scores(FAKE, FAKE, 64, 7168, 384, FAKE, FAKE, 16, NULL) == INVALID
     assert L.moe_router_scores(FAKE, FAKE, 0, 7168, 384, FAKE, FAKE, 0, NULL) == OK
-    assert L.moe_seq_aux_loss(FAKE, FAKE, 4, 64, 2048, 8, f(1e-3), FAKE, NULL, NULL, NULL) == SHAPE
-    assert L.moe_seq_aux_loss(FAKE, FAKE, 1, 20000, 384, 8, f(1e-3), FAKE, NULL, NULL,
-                              NULL) == SHAPE
-    assert L.moe_seq_aux_loss(FAKE, FAKE, 4, 0, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == INVALID
-    assert L.moe_seq_aux_loss(NULL, FAKE, 4, 64, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == INVALID
-    assert L.moe_seq_aux_loss(FAKE, FAKE, 0, 64, 384, 8, f(1e-3), FAKE, NULL, NULL, NULL) == OK
+    need = moe.moe_seq_aux_workspace_size(4, 64, 384)
+    assert need >= 4 * 64 * 4
+    aux = lambda *a, ws=need: L.moe_seq_aux_loss(*a, FAKE, NULL, NULL, FAKE, ws, NULL)
+    assert aux(FAKE, FAKE, 4, 64, 2048, 8, f(1e-3)) == SHAPE
+    assert aux(FAKE, FAKE, 4, 0, 384, 8, f(1e-3)) == INVALID
+    assert aux(NULL, FAKE, 4, 64, 384, 8, f(1e-3)) == INVALID
+    assert aux(FAKE, FAKE, 4, 64, 384, 8, f(1e-3), ws=need - 1) == INVALID
+    assert aux(FAKE, FAKE, 0, 64, 384, 8, f(1e-3)) == OK

@@ -81,7 +81,7 @@ def test_router_scores(moe):
 
 
 @pytest.mark.parametrize("B,S,E,k", [(4, 64, 384, 8), (3, 37, 7, 3), (1, 500, 1024, 32),
-                                     (8, 1, 16, 4)])
+                                     (8, 1, 16, 4), (2, 4096, 384, 8)])
 def test_seq_aux_loss(moe, B, S, E, k):
     rng = np.random.default_rng(B * S + E)
     T = B * S
