@@ -82,6 +82,13 @@ def _bind(L):
     L.oracle_quantize_fp8.restype = i32
     L.oracle_dequantize_fp8.argtypes = [P, P, i64, i64, P]
     L.oracle_dequantize_fp8.restype = i32
+    L.oracle_quantize_fp8_rows.argtypes = [P, i64, i64, P, P]
+    L.oracle_quantize_fp8_rows.restype = None
+    L.oracle_swiglu_row_fp8.argtypes = [P, P, P, P, P, i32, i32, P]
+    L.oracle_swiglu_row_fp8.restype = None
+    L.oracle_moe_rows_fp8.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P,
+                                      P, i32, P, i32]
+    L.oracle_moe_rows_fp8.restype = i32
     L.oracle_bias_update.argtypes = [P, i32, i32, i32, ctypes.c_float, P]
     L.oracle_bias_update.restype = None
     L.oracle_seq_aux_loss.argtypes = [P, P, i32, i32, i32, i32, f64, P, P, P]
@@ -168,6 +175,98 @@ def dequantize_fp8(q, sexp):
     if rc != 0:
         raise ValueError("oracle_dequantize_fp8: rows and cols must be multiples of 128")
     return out
+
+
+def quantize_fp8_rows(w):
+    """bf16 matrix [.., rows, cols] -> (codes uint8 [.., rows, cols], one
+    exponent per row int8 [.., rows]): the FP8-compute format."""
+    u = _u16(w)
+    cols = u.shape[-1]
+    rows = u.size // cols
+    q = np.empty(u.shape, dtype=np.uint8)
+    sexp = np.empty(u.shape[:-1], dtype=np.int8)
+    lib().oracle_quantize_fp8_rows(_ptr(u), rows, cols, _ptr(q), _ptr(sexp))
+    return q, sexp
+
+
+def swiglu_row_fp8(xrow, q_gate_up, s_gate_up, q_down, s_down):
+    """One expert on one token in FP8 compute (see the C header) -> y f64 [d]."""
+    xu = _u16(xrow)
+    qg, sg = _np(q_gate_up, np.uint8), _np(s_gate_up, np.int8)
+    qd, sd = _np(q_down, np.uint8), _np(s_down, np.int8)
+    d = xu.shape[-1]
+    inter = qg.shape[0] // 2
+    y = np.empty((d,), np.float64)
+    lib().oracle_swiglu_row_fp8(_ptr(xu), _ptr(qg), _ptr(sg), _ptr(qd), _ptr(sd), d, inter,
+                                _ptr(y))
+    return y
+
+
+def moe_rows_fp8(x, topk_idx, topk_w, expert_q, shared_q, tokens=None,
+                 nthreads: int | None = None):
+    """Steps 5-7 in FP8 compute on the listed tokens.
+
+    expert_q: sequence indexed by expert of (q_gate_up, s_gate_up, q_down,
+    s_down) from quantize_fp8_rows, or None for experts no listed token
+    selects; shared_q: the same tuple for the shared expert."""
+    xu = _u16(x)
+    T, d = xu.shape
+    idx = _np(topk_idx, np.int32)
+    w = _np(topk_w, np.float64)
+    k = idx.shape[1]
+    E = len(expert_q)
+    keep = []
+    ptrs = [(ctypes.c_void_p * E)() for _ in range(4)]
+    for e in range(E):
+        if expert_q[e] is None:
+            continue
+        arrs = [_np(expert_q[e][0], np.uint8), _np(expert_q[e][1], np.int8),
+                _np(expert_q[e][2], np.uint8), _np(expert_q[e][3], np.int8)]
+        keep += arrs
+        for j in range(4):
+            ptrs[j][e] = arrs[j].ctypes.data
+    sq = [_np(shared_q[0], np.uint8), _np(shared_q[1], np.int8),
+          _np(shared_q[2], np.uint8), _np(shared_q[3], np.int8)]
+    inter = sq[0].shape[0] // 2
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    n = T if tok is None else tok.shape[0]
+    out = np.empty((n, d), np.float64)
+    rc = lib().oracle_moe_rows_fp8(_ptr(xu), T, d, E, k, inter, _ptr(idx), _ptr(w),
+                                   *[ctypes.cast(p, ctypes.c_void_p) for p in ptrs],
+                                   *[_ptr(a) for a in sq], _ptr(tok), n, _ptr(out),
+                                   nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_moe_rows_fp8: a selected expert's weights are missing")
+    del keep
+    return out
+
+
+def quantize_expert_rows(inputs: dict, experts):
+    """The FP8-compute weights of the listed experts and of the shared expert,
+    from the oracle's own row quantizer: ({e: (qgu, sgu, qdn, sdn)}, shared)."""
+    out = {}
+    for e in experts:
+        qg, sg = quantize_fp8_rows(inputs["w_gate_up"][e])
+        qd, sd = quantize_fp8_rows(inputs["w_down"][e])
+        out[e] = (qg, sg, qd, sd)
+    qg, sg = quantize_fp8_rows(inputs["ws_gate_up"])
+    qd, sd = quantize_fp8_rows(inputs["ws_down"])
+    return out, (qg, sg, qd, sd)
+
+
+def moe_forward_fp8(inputs: dict, k: int, scale: float, tokens=None,
+                    nthreads: int | None = None):
+    """Whole layer with FP8 compute in every expert (routing stays bf16 /
+    fp64): route all tokens, quantize the selected experts' weights per row
+    with the oracle's quantizer, evaluate the listed rows.
+    Returns (out f64 [n,d], topk_idx, topk_w, gap)."""
+    idx, w, gap = route(inputs["x"], inputs["w_router"], inputs["bias"], k, scale, nthreads)
+    E = inputs["w_router"].shape[0]
+    need = sorted(set(np.unique(idx if tokens is None else idx[np.asarray(tokens)]).tolist()))
+    qe, qs = quantize_expert_rows(inputs, need)
+    expert_q = [qe.get(e) for e in range(E)]
+    out = moe_rows_fp8(inputs["x"], idx, w, expert_q, qs, tokens=tokens, nthreads=nthreads)
+    return out, idx, w, gap
 
 
 def bias_update(counts, T: int, k: int, gamma: float, bias):

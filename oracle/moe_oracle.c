@@ -402,3 +402,111 @@ void oracle_seq_aux_loss(const double* scores, const int32_t* topk_idx, int B, i
     free(fb);
     free(pb);
 }
+
+/* ------------------------------------------------------------- FP8 compute */
+
+/* quantize n values (bf16 bits, or doubles already bf16-exact) with one exponent */
+static int quantize_row_f64(const double* v, int64_t n, uint8_t* q) {
+    double amax = 0.0;
+    for (int64_t i = 0; i < n; ++i)
+        if (fabs(v[i]) > amax) amax = fabs(v[i]);
+    const int s = oracle_fp8_block_exponent(amax);
+    for (int64_t i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(ldexp(v[i], -s));
+    return s;
+}
+
+void oracle_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
+                              int8_t* sexp) {
+    double* v = (double*)calloc((size_t)cols, sizeof(double));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) v[c] = oracle_bf16_to_f64(w[r * cols + c]);
+        sexp[r] = (int8_t)quantize_row_f64(v, cols, q + r * cols);
+    }
+    free(v);
+}
+
+void oracle_swiglu_row_fp8(const uint16_t* xrow, const uint8_t* wq_gu, const int8_t* s_gu,
+                           const uint8_t* wq_dn, const int8_t* s_dn, int d, int inter, double* y) {
+    double* xv = (double*)calloc((size_t)d, sizeof(double));
+    uint8_t* xq = (uint8_t*)malloc((size_t)d);
+    double* h = (double*)calloc((size_t)inter, sizeof(double));
+    uint8_t* hq = (uint8_t*)malloc((size_t)inter);
+    double* xd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* hd = (double*)malloc(sizeof(double) * (size_t)inter);
+    for (int i = 0; i < d; ++i) xv[i] = oracle_bf16_to_f64(xrow[i]);
+    const int sx = quantize_row_f64(xv, d, xq);
+    for (int i = 0; i < d; ++i) xd[i] = oracle_e4m3_decode(xq[i]);
+    for (int n = 0; n < inter; ++n) {
+        const uint8_t* wg = wq_gu + (size_t)n * d;
+        const uint8_t* wu = wq_gu + (size_t)(inter + n) * d;
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < d; ++i) {
+            g += oracle_e4m3_decode(wg[i]) * xd[i];
+            u += oracle_e4m3_decode(wu[i]) * xd[i];
+        }
+        g = ldexp(g, s_gu[n] + sx);
+        u = ldexp(u, s_gu[inter + n] + sx);
+        /* the stored intermediate is bf16 */
+        h[n] = oracle_bf16_to_f64(oracle_f64_to_bf16(oracle_silu(g) * u));
+    }
+    const int sh = quantize_row_f64(h, inter, hq);
+    for (int n = 0; n < inter; ++n) hd[n] = oracle_e4m3_decode(hq[n]);
+    for (int o = 0; o < d; ++o) {
+        const uint8_t* wd = wq_dn + (size_t)o * inter;
+        double acc = 0.0;
+        for (int n = 0; n < inter; ++n) acc += oracle_e4m3_decode(wd[n]) * hd[n];
+        y[o] = ldexp(acc, s_dn[o] + sh);
+    }
+    free(xv); free(xq); free(h); free(hq); free(xd); free(hd);
+}
+
+typedef struct {
+    const uint16_t* x; int d, k, inter;
+    const int32_t* topk_idx; const double* topk_w;
+    const uint8_t* const* egq; const int8_t* const* egs;
+    const uint8_t* const* edq; const int8_t* const* eds;
+    const uint8_t* sgq; const int8_t* sgs; const uint8_t* sdq; const int8_t* sds;
+    const int32_t* tokens; double* out;
+} rows8_ctx;
+
+static void rows8_tokens(void* p, int r0, int r1) {
+    rows8_ctx* c = (rows8_ctx*)p;
+    const int d = c->d, k = c->k;
+    double* y = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int r = r0; r < r1; ++r) {
+        int t = c->tokens ? c->tokens[r] : r;
+        const uint16_t* xt = c->x + (size_t)t * d;
+        double* o = c->out + (size_t)r * d;
+        oracle_swiglu_row_fp8(xt, c->sgq, c->sgs, c->sdq, c->sds, d, c->inter, o);
+        for (int j = 0; j < k; ++j) {
+            int e = c->topk_idx[(size_t)t * k + j];
+            double w = c->topk_w[(size_t)t * k + j];
+            oracle_swiglu_row_fp8(xt, c->egq[e], c->egs[e], c->edq[e], c->eds[e], d, c->inter, y);
+            for (int i = 0; i < d; ++i) o[i] += w * y[i];
+        }
+    }
+    free(y);
+}
+
+int oracle_moe_rows_fp8(const uint16_t* x, int T, int d, int E, int k, int inter,
+                        const int32_t* topk_idx, const double* topk_w,
+                        const uint8_t* const* egu_q, const int8_t* const* egu_s,
+                        const uint8_t* const* edn_q, const int8_t* const* edn_s,
+                        const uint8_t* sgu_q, const int8_t* sgu_s, const uint8_t* sdn_q,
+                        const int8_t* sdn_s, const int32_t* tokens, int n_tokens, double* out,
+                        int nthreads) {
+    if (!sgu_q || !sgu_s || !sdn_q || !sdn_s) return -1;
+    if (!tokens) n_tokens = T;
+    for (int r = 0; r < n_tokens; ++r) {
+        int t = tokens ? tokens[r] : r;
+        if (t < 0 || t >= T) return -1;
+        for (int j = 0; j < k; ++j) {
+            int e = topk_idx[(size_t)t * k + j];
+            if (e < 0 || e >= E || !egu_q[e] || !egu_s[e] || !edn_q[e] || !edn_s[e]) return -1;
+        }
+    }
+    rows8_ctx c = {x, d, k, inter, topk_idx, topk_w, egu_q, egu_s, edn_q, edn_s,
+                   sgu_q, sgu_s, sdn_q, sdn_s, tokens, out};
+    oracle_parallel_for(n_tokens, nthreads, rows8_tokens, &c);
+    return 0;
+}

@@ -146,6 +146,44 @@ int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, in
                           uint16_t* w_out);
 
 /*
+ * FP8 compute ("Kimi K2.5 Q&A", Q7.1 names V3's "compute in FP8" beside K2.5's
+ * quantized storage; "Kimi K2 deep dive", 3.2: FP8 for speed).  The pages give
+ * no format.  The one taken for FP8 compute: E4M3 operands with one power-of-two
+ * scale per ROW (each weight row = output channel, each activation row = token),
+ * chosen by the rule above (s = smallest integer with row amax <= 448 * 2^s,
+ * clamped to [-124, 127]); the scales then factor out of every K sum.
+ */
+
+/* Per-row quantization: w [rows, cols] bf16 -> q [rows, cols], sexp [rows]. */
+void oracle_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
+                              int8_t* sexp);
+
+/*
+ * One expert on one token row in FP8 compute:
+ *   x row -> (xq, sx) per-row quantization of the bf16 row
+ *   g_n = 2^(sg_n + sx) sum_i dec(wq_gu[n, i]) dec(xq_i),  u_n likewise (row inter + n)
+ *   h_n = bf16( silu(g_n) * u_n )            (the stored intermediate)
+ *   (hq, sh) = per-row quantization of h
+ *   y_o = 2^(sd_o + sh) sum_n dec(wq_dn[o, n]) dec(hq_n)
+ * wq_gu [2I, d] + s_gu [2I]; wq_dn [d, I] + s_dn [d].  y in fp64.
+ */
+void oracle_swiglu_row_fp8(const uint16_t* xrow, const uint8_t* wq_gu, const int8_t* s_gu,
+                           const uint8_t* wq_dn, const int8_t* s_dn, int d, int inter, double* y);
+
+/*
+ * Whole layer, FP8 compute for every expert (routed and shared), on a subset of
+ * tokens; routing (topk_idx, topk_w) from oracle_route on the bf16 router.
+ * expert_* arrays of pointers as in oracle_moe_rows (NULL for unused experts).
+ */
+int oracle_moe_rows_fp8(const uint16_t* x, int T, int d, int E, int k, int inter,
+                        const int32_t* topk_idx, const double* topk_w,
+                        const uint8_t* const* egu_q, const int8_t* const* egu_s,
+                        const uint8_t* const* edn_q, const int8_t* const* edn_s,
+                        const uint8_t* sgu_q, const int8_t* sgu_s, const uint8_t* sdn_q,
+                        const int8_t* sdn_s, const int32_t* tokens, int n_tokens, double* out,
+                        int nthreads);
+
+/*
  * Load balancing ("Kimi K2.5 Q&A", Q7.2; "Kimi K2.5 deep dive", CH10.2 step 2).
  *
  * Bias update (noaux_tc): the selection bias is a buffer, not learned; after a

@@ -399,6 +399,135 @@ def pin_fp8_quantize_bounds():
             assert 224.0 <= top / 2.0 ** sexp[i, j] <= 448.0
 
 
+# FP8 compute ("Kimi K2.5 Q&A", Q7.1 names V3's compute in FP8; "Kimi K2 deep
+# dive", 3.2): E4M3 operands with one power-of-two exponent per row (weight
+# output channel, token), which factors out of every K sum.
+
+def _brute_exponent(amax):
+    if amax == 0.0:
+        return 0
+    return min(max(next(t for t in range(-300, 300) if amax <= 448.0 * 2.0 ** t), -124), 127)
+
+
+def _u16_of(w):
+    return _bf16(w).view(torch.int16).numpy().view(np.uint16)
+
+
+def _torch_e4m3_decode(q):
+    return torch.from_numpy(np.ascontiguousarray(q, dtype=np.uint8)).view(
+        torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def pin_fp8_rows_quantizer_library():
+    """Each row's exponent by brute force from its own amax (negative maxima,
+    an exact 448 * 2^s boundary, zero and clamped rows), its codes from torch's
+    float8_e4m3fn cast of w * 2^-s."""
+    rng = np.random.default_rng(5)
+    rows, cols = 12, 200
+    w = rng.normal(0, 1, (rows, cols)) * 2.0 ** rng.integers(-30, 30, (rows, 1))
+    w[3] = 0.0
+    w[4] = rng.normal(0, 1e-39, cols)              # amax below 448 * 2^-124: clamped
+    w[5] = rng.normal(0, 1e-3, cols)
+    w[5, 7] = 56.0                                 # = 448 * 2^-3 exactly: s = -3
+    w[6, 9] = -50.0 * np.abs(w[6]).max()           # the row maximum is negative
+    wb = _u16_of(w)
+    wf = oracle.bf16_to_f64(wb)
+    q, s = oracle.quantize_fp8_rows(wb)
+    assert q.shape == (rows, cols) and s.shape == (rows,)
+    for r in range(rows):
+        se = _brute_exponent(np.abs(wf[r]).max())
+        assert s[r] == se, (r, s[r], se)
+        assert np.array_equal(q[r], _torch_e4m3(wf[r] * 2.0 ** -se)), r
+    assert s[3] == 0 and s[4] == -124 and s[5] == -3
+
+
+def _e4m3_exact(rng, shape, row_exp):
+    """Values code * 2^e with E4M3 normal codes, random signs, each row's
+    largest magnitude 448 * 2^e (so the row quantizer is exact on them)."""
+    codes = rng.integers(0x08, 0x7F, shape)
+    vals = _torch_e4m3_decode(codes.astype(np.uint8)) * rng.choice([-1.0, 1.0], shape)
+    vals[:, 0] = 448.0
+    return vals * 2.0 ** np.asarray(row_exp, dtype=float)[:, None]
+
+
+def pin_fp8_compute_exact_inputs():
+    """On inputs whose rows the quantizer represents exactly, FP8 compute is the
+    bf16 oracle's SwiGLU activation rounded to bf16 and quantized per row (the
+    exponent by brute force, the codes by torch's cast), then a matrix product."""
+    rng = np.random.default_rng(6)
+    d, inter = 96, 80
+    x = _e4m3_exact(rng, (1, d), [-9])[0]
+    wgu = _e4m3_exact(rng, (2 * inter, d), rng.integers(-16, -12, 2 * inter))
+    wdn = _e4m3_exact(rng, (d, inter), rng.integers(-16, -12, d))
+    xb, gub, dnb = _u16_of(x), _u16_of(wgu), _u16_of(wdn)
+    assert np.array_equal(oracle.bf16_to_f64(gub), wgu)     # exact in bf16
+    qg, sg = oracle.quantize_fp8_rows(gub)
+    qd, sd = oracle.quantize_fp8_rows(dnb)
+    y = oracle.swiglu_row_fp8(xb, qg, sg, qd, sd)
+    _, act = oracle.swiglu_row(xb, gub, dnb, want_act=True)
+    h = oracle.bf16_to_f64(oracle.f64_to_bf16(act))
+    sh = _brute_exponent(np.abs(h).max())
+    hq = _torch_e4m3_decode(_torch_e4m3(h * 2.0 ** -sh)) * 2.0 ** sh
+    ref = wdn @ hq
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def pin_fp8_compute_exponent_bookkeeping():
+    """Power-of-two rescalings that leave every code unchanged move the result
+    exactly: x * 2^3 with the gate|up rows * 2^-3 gives the same y; the up rows
+    * 2^5 give y * 2^5 (through the activation's exponent); one down row * 2^-4
+    scales that output alone."""
+    rng = np.random.default_rng(7)
+    d, inter = 128, 64
+    x = rng.normal(0, 1, d)
+    wgu = rng.normal(0, 0.05, (2 * inter, d))
+    wdn = rng.normal(0, 0.05, (d, inter))
+
+    def run(x_, gu_, dn_):
+        qg, sg = oracle.quantize_fp8_rows(_u16_of(gu_))
+        qd, sd = oracle.quantize_fp8_rows(_u16_of(dn_))
+        return oracle.swiglu_row_fp8(_u16_of(x_), qg, sg, qd, sd)
+
+    y = run(x, wgu, wdn)
+    assert np.abs(y).max() > 0
+    assert np.array_equal(run(x * 8.0, wgu / 8.0, wdn), y)
+    up = wgu.copy()
+    up[inter:] *= 32.0
+    assert np.array_equal(run(x, up, wdn), y * 32.0)
+    dn = wdn.copy()
+    dn[5] /= 16.0
+    want = y.copy()
+    want[5] /= 16.0
+    assert np.array_equal(run(x, wgu, dn), want)
+
+
+def pin_fp8_compute_layer_identities():
+    """Whole layer in FP8 compute with expert e = the base expert with its up
+    rows * 2^e, shared expert = base: row t is exactly
+    y_base(x_t) (1 + sum_j w_tj 2^(e_tj)); a token subset gives the same rows."""
+    rng = np.random.default_rng(8)
+    T, d, inter, E, k = 5, 64, 32, 4, 2
+    x = rng.normal(0, 1, (T, d))
+    gu = rng.normal(0, 0.05, (2 * inter, d))
+    dn = rng.normal(0, 0.05, (d, inter))
+    base = oracle.quantize_fp8_rows(_u16_of(gu)) + oracle.quantize_fp8_rows(_u16_of(dn))
+    experts = []
+    for e in range(E):
+        g = gu.copy()
+        g[inter:] *= 2.0 ** e
+        experts.append(oracle.quantize_fp8_rows(_u16_of(g)) + base[2:])
+    idx = np.array([[0, 3], [2, 1], [3, 0], [1, 2], [2, 3]], np.int32)
+    w = rng.uniform(0.1, 1.5, (T, k))
+    xb = _u16_of(x)
+    out = oracle.moe_rows_fp8(xb, idx, w, experts, base)
+    for t in range(T):
+        yb = oracle.swiglu_row_fp8(xb[t], *base)
+        want = yb * (1.0 + sum(w[t, j] * 2.0 ** idx[t, j] for j in range(k)))
+        assert np.allclose(out[t], want, rtol=1e-13, atol=1e-13 * np.abs(want).max()), t
+    sub = oracle.moe_rows_fp8(xb, idx, w, experts, base, tokens=np.array([4, 1]))
+    assert np.array_equal(sub, out[[4, 1]])
+
+
 # ---------------------------------------------------------- load balancing
 # "Kimi K2.5 Q&A", Q7.2 and "Kimi K2.5 deep dive", CH10.2 step 2: the selection
 # bias is a non-learned buffer lowered for over-loaded and raised for
@@ -477,7 +606,9 @@ ALL_PINS = [pin_bf16_rounding, pin_sigmoid_silu, pin_route_worked_example,
             pin_row_independence, pin_combine, pin_fp8_decode_library, pin_fp8_anchor_values,
             pin_fp8_encode_library, pin_fp8_block_exponent_brute_force, pin_fp8_quantize_bounds,
             pin_bias_update_worked_example, pin_bias_update_invariants, pin_bias_update_moves_load,
-            pin_seq_aux_loss_closed_forms]
+            pin_seq_aux_loss_closed_forms, pin_fp8_rows_quantizer_library,
+            pin_fp8_compute_exact_inputs, pin_fp8_compute_exponent_bookkeeping,
+            pin_fp8_compute_layer_identities]
 
 
 def failing_pins():

@@ -70,6 +70,24 @@ MUTANTS = [
      "        else if ((long long)counts[e] < total / E)\n            b = b + gamma;"),
     ("seq_aux_unnormalized", "pb[i] += scores[(size_t)t * E + i] / tot;", "pb[i] += scores[(size_t)t * E + i];"),
     ("seq_aux_no_f_scale", "fb[i] *= (double)E / ((double)k * S);", "fb[i] *= 1.0;"),
+    ("fp8c_drops_x_exponent", "g = ldexp(g, s_gu[n] + sx);", "g = ldexp(g, s_gu[n]);"),
+    ("fp8c_up_uses_gate_exponent", "u = ldexp(u, s_gu[inter + n] + sx);",
+     "u = ldexp(u, s_gu[n] + sx);"),
+    ("fp8c_x_exponent_sign", "g = ldexp(g, s_gu[n] + sx);", "g = ldexp(g, s_gu[n] - sx);"),
+    ("fp8c_h_not_rounded",
+     "h[n] = oracle_bf16_to_f64(oracle_f64_to_bf16(oracle_silu(g) * u));",
+     "h[n] = oracle_silu(g) * u;"),
+    ("fp8c_down_exponent_dropped", "y[o] = ldexp(acc, s_dn[o] + sh);", "y[o] = ldexp(acc, sh);"),
+    ("fp8c_activation_exponent_dropped", "y[o] = ldexp(acc, s_dn[o] + sh);",
+     "y[o] = ldexp(acc, s_dn[o]);"),
+    ("fp8c_shared_dropped",
+     "oracle_swiglu_row_fp8(xt, c->sgq, c->sgs, c->sdq, c->sds, d, c->inter, o);",
+     "for (int i = 0; i < d; ++i) o[i] = 0.0;"),
+    ("fp8c_expert_by_slot",
+     "oracle_swiglu_row_fp8(xt, c->egq[e], c->egs[e], c->edq[e], c->eds[e], d, c->inter, y);",
+     "oracle_swiglu_row_fp8(xt, c->egq[j], c->egs[j], c->edq[j], c->eds[j], d, c->inter, y);"),
+    ("fp8_rows_signed_max", "if (fabs(v[i]) > amax) amax = fabs(v[i]);",
+     "if (v[i] > amax) amax = v[i];"),
 ]
 
 
