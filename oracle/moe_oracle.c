@@ -482,7 +482,7 @@ static void rows8_tokens(void* p, int r0, int r1) {
             int e = c->topk_idx[(size_t)t * k + j];
             double w = c->topk_w[(size_t)t * k + j];
             oracle_swiglu_row_fp8(xt, c->egq[e], c->egs[e], c->edq[e], c->eds[e], d, c->inter, y);
-            for (int i = 0; i < d; ++i) o[i] += w * y[i];
+            for (int i = 0; i < d; ++i) o[i] += y[i] * w;
         }
     }
     free(y);

@@ -86,6 +86,8 @@ MUTANTS = [
     ("fp8c_expert_by_slot",
      "oracle_swiglu_row_fp8(xt, c->egq[e], c->egs[e], c->edq[e], c->eds[e], d, c->inter, y);",
      "oracle_swiglu_row_fp8(xt, c->egq[j], c->egs[j], c->edq[j], c->eds[j], d, c->inter, y);"),
+    ("fp8c_routed_weight_dropped", "for (int i = 0; i < d; ++i) o[i] += y[i] * w;",
+     "for (int i = 0; i < d; ++i) o[i] += y[i];"),
     ("fp8_rows_signed_max", "if (fabs(v[i]) > amax) amax = fabs(v[i]);",
      "if (v[i] > amax) amax = v[i];"),
 ]
