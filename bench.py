@@ -53,9 +53,11 @@ def parse_args(argv=None):
                    help="time the load-balancing pass instead of the layer: router scores, "
                         "route, permute, the sequence-level loss over sequences of S tokens "
                         "and the bias update")
-    p.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
-                   help="routed experts' weight storage: bf16, or E4M3 codes with one "
-                        "power-of-two scale per 128x128 block (quantized once, untimed)")
+    p.add_argument("--weights", choices=["bf16", "fp8", "w8a8"], default="bf16",
+                   help="expert weights: bf16; fp8 = routed experts stored as E4M3 codes with "
+                        "one power-of-two scale per 128x128 block, bf16 compute; w8a8 = FP8 "
+                        "compute in every expert, E4M3 weights and activations with one "
+                        "power-of-two scale per row (weights quantized once, untimed)")
     p.add_argument("--cpu-sample", type=int, default=None,
                    help="tokens in the oracle's timed sample (default: sized from the core count)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -211,19 +213,27 @@ def layer_accounting(cfg, touched: int, weights: str = "bf16"):
     expert is always touched on top).  Weight bytes per expert follow the
     pages' 3 x d x inter parameter count ("Kimi K2.5 Q&A", Q2.1).  With FP8
     storage a routed expert's weights are one byte each plus one int8 scale
-    per 128 x 128 block; the shared expert stays bf16."""
+    per 128 x 128 block; the shared expert stays bf16.  With FP8 compute every
+    expert's weights (shared too) are one byte each plus one int8 exponent per
+    row, and the GEMMs read their token rows as one byte per element plus one
+    exponent per row."""
     T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
     rows = T * (k + 1)
     w_gu = 2 * I * d * 2                 # gate + up weights of one expert, bytes
     w_dn = d * I * 2
+    a_in_gu, a_in_dn = rows * d * 2, rows * I * 2      # token rows the GEMMs read
     if weights == "fp8":
         r_gu = 2 * I * d + (2 * I // 128) * (d // 128)
         r_dn = d * I + (d // 128) * (I // 128)
+    elif weights == "w8a8":
+        r_gu, r_dn = 2 * I * d + 2 * I, d * I + d
+        w_gu, w_dn = r_gu, r_dn
+        a_in_gu, a_in_dn = rows * (d + 1), rows * (I + 1)
     else:
         r_gu, r_dn = w_gu, w_dn
     acc = {}
-    acc["gate_up_bytes"] = touched * r_gu + w_gu + rows * d * 2 + rows * I * 2
-    acc["down_bytes"] = touched * r_dn + w_dn + rows * I * 2 + rows * d * 2
+    acc["gate_up_bytes"] = touched * r_gu + w_gu + a_in_gu + rows * I * 2
+    acc["down_bytes"] = touched * r_dn + w_dn + a_in_dn + rows * d * 2
     acc["gate_up_flops"] = 2.0 * rows * 2 * I * d
     acc["down_flops"] = 2.0 * rows * I * d
     acc["router_flops"] = 2.0 * T * d * E
@@ -266,6 +276,12 @@ class OracleSample:
                 self.egu[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.egu[e]))
                 self.edn[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.edn[e]))
         self.sgu, self.sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
+        if weights == "w8a8":
+            # FP8-compute weights from the oracle's own row quantizer
+            host = {"w_gate_up": self.egu, "w_down": self.edn, "ws_gate_up": self.sgu,
+                    "ws_down": self.sdn}
+            qe, self.qs = oracle.quantize_expert_rows(host, self.need)
+            self.qe = [qe.get(e) for e in range(cfg.E)]
 
     def run(self) -> float:
         """Seconds for the oracle's full layer (routing + experts) on the sample."""
@@ -273,13 +289,17 @@ class OracleSample:
         t0 = time.perf_counter()
         ridx, rw, _ = oracle.route(self.x, self.wr, self.bias, self.cfg.k, self.cfg.scale,
                                    nthreads=self.threads)
-        oracle.moe_rows(self.x, ridx, rw, self.egu, self.edn, self.sgu, self.sdn,
-                        nthreads=self.threads)
+        if self.weights == "w8a8":
+            oracle.moe_rows_fp8(self.x, ridx, rw, self.qe, self.qs, nthreads=self.threads)
+        else:
+            oracle.moe_rows(self.x, ridx, rw, self.egu, self.edn, self.sgu, self.sdn,
+                            nthreads=self.threads)
         return time.perf_counter() - t0
 
     def describe(self) -> str:
-        fp8 = " (routed weights: the oracle's FP8 quantization, dequantized)" \
-            if self.weights == "fp8" else ""
+        fp8 = {"fp8": " (routed weights: the oracle's FP8 quantization, dequantized)",
+               "w8a8": " (FP8 compute: the oracle's per-row E4M3 quantization of weights "
+                       "and activations)"}.get(self.weights, "")
         return (f"{len(self.tokens)} of {self.cfg.T} tokens (evenly spaced), full routing + "
                 f"{len(self.need)} routed experts + shared expert, fp64{fp8}")
 
@@ -289,7 +309,7 @@ def default_cpu_sample(cfg, weights: str = "bf16"):
     # 16-core host busy for several seconds without copying every expert.
     # With FP8 weights the oracle first quantizes every expert the sample
     # selects (about a second each), so the sample is smaller.
-    if weights == "fp8":
+    if weights in ("fp8", "w8a8"):
         return min(cfg.T, 8)
     return min(cfg.T, max(64, 4 * host_cores()))
 
@@ -340,14 +360,22 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
 
     fp8 = args.weights == "fp8"
+    w8a8 = args.weights == "w8a8"
     if fp8:
         # storage format conversion, once, outside every timed region
         qgu, egu = moe.moe_quantize_fp8(g["w_gate_up"])
         qdn, edn = moe.moe_quantize_fp8(g["w_down"])
         torch.cuda.synchronize(dev)
+    if w8a8:
+        wq = []
+        for key in ("w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+            wq += list(moe.moe_quantize_fp8_rows(g[key]))
+        torch.cuda.synchronize(dev)
 
     def layer(x_in):
-        if fp8:
+        if w8a8:
+            moe.moe_layer_forward_w8a8(x_in, g["w_router"], g["bias"], *wq, k, cfg.scale, out)
+        elif fp8:
             moe.moe_layer_forward_fp8(x_in, g["w_router"], g["bias"], qgu, egu, qdn, edn,
                                       g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
         else:
@@ -448,17 +476,23 @@ def main(argv=None):
     else:
         achieved = acc["gate_up_flops"] / (k_ms / 1e3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        src = f"{peak_src} bf16_tflops_sustained"
+        if w8a8:
+            # E4M3 x E4M3: the measured bf16 peak times the nominal ratio 4.5 / 2.25
+            peak *= 2.0
+            src += " x 2 (nominal e4m3 / bf16 ratio)"
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "kernel": kname,
                 "algorithmic_flops_per_launch": acc["gate_up_flops"],
-                "avg_launch_ms": k_ms, "peak_source": f"{peak_src} bf16_tflops_sustained"}
+                "avg_launch_ms": k_ms, "peak_source": src}
         t_tc = acc["flops"] / (peak * 1e12)
         t_hbm = acc["weight_bytes"] / (peaks["hbm_gbs"] * 1e9)
         layer_roof = {"bound": "tensor", "ideal_ms": t_tc * 1e3, "frac": t_tc / (ms_step / 1e3),
                       "hbm_ideal_ms": t_hbm * 1e3, "hbm_frac": t_hbm / (ms_step / 1e3),
                       "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
                       "touched_experts": touched}
-    roof["traffic"] = profiled_traffic(args.workload + ("_fp8" if fp8 else ""), kname)
+    roof["traffic"] = profiled_traffic(
+        args.workload + {"fp8": "_fp8", "w8a8": "_w8a8"}.get(args.weights, ""), kname)
 
     # ---------------------------------------------------------- CPU baseline
     cpu = None
@@ -473,11 +507,13 @@ def main(argv=None):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if w8a8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": args.workload + "".join(f" {x}" for x in args.set),
                        "T": T, "d": d, "E": E, "k": k, "inter": I,
                        "scale": cfg.scale, "bias": cfg.bias, "parallelism": f"replicas{world}",
-                       "weights": "fp8_e4m3_block128_pow2" if fp8 else "bf16",
+                       "weights": {"fp8": "fp8_e4m3_block128_pow2",
+                                   "w8a8": "w8a8_e4m3_row_pow2"}.get(args.weights, "bf16"),
                        "l2": "inputs larger than L2: every step streams "
                              f"{acc['weight_bytes'] / 1e9:.1f} GB of expert weights"},
             "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cpu, "e2e": e2e,
@@ -588,7 +624,7 @@ def run_reference(args, cfg, world):
         per_token = probe.run()
         waves = max(1, int(REFERENCE_BUDGET_S / runs / per_token))
         n = max(1, min(cfg.T, waves * host_cores()))
-    smp = OracleSample(cfg, g, n)
+    smp = OracleSample(cfg, g, n, args.weights)
     del g
     per_step = []
     for i in range(runs):
@@ -603,7 +639,8 @@ def run_reference(args, cfg, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "inter": cfg.inter, "scale": cfg.scale, "bias": cfg.bias},
+                   "inter": cfg.inter, "scale": cfg.scale, "bias": cfg.bias,
+                   "weights": args.weights},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.threads, "kind": "oracle",
                          "sample": smp.describe()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

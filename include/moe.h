@@ -248,6 +248,58 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * FP8 compute ("Kimi K2.5 Q&A", Q7.1 names DeepSeek-V3's "compute in FP8" next
+ * to K2.5's quantized storage; "Kimi K2 deep dive", 3.2: FP8 for speed).  The
+ * pages give no format; this library's: E4M3 codes (as above) with one
+ * power-of-two exponent per ROW, s an int8 chosen by the rule above over the
+ * row (smallest integer with max|row| <= 448 * 2^s, clamped to [-124, 127], 0
+ * for an all-zero row), q = E4M3 nearest to w * 2^-s, ties to even.  A weight
+ * row is an output channel, an activation row a token, so both exponents
+ * factor out of each dot product: the tensor cores multiply codes
+ * (E4M3 x E4M3 -> fp32) and the result is scaled by 2^(s_w + s_x) exactly.
+ *
+ * moe_quantize_fp8_rows: w [rows, cols] bf16 row-major (cols a multiple of 16)
+ * -> q [rows, cols] uint8 codes and exps [rows] int8, caller-owned device
+ * memory, asynchronous on `stream`.  Stacked experts quantize in one call:
+ * [E, 2*inter, d] as rows = E*2*inter (exps [E, 2*inter]), [E, d, inter] as
+ * rows = E*d (exps [E, d]).  MOE_ERR_UNSUPPORTED_SHAPE for other shapes,
+ * MOE_ERR_INVALID_ARG for null or unaligned (16-byte) w or q, or null exps.
+ *
+ * moe_layer_forward_w8a8: the layer with FP8 compute in every expert, routed
+ * and shared (the router and top-k stay as in moe_layer_forward, bf16 / fp32):
+ *   wq_gate_up [E, 2*inter, d] uint8 + wq_gate_up_exp [E, 2*inter] int8
+ *   wq_down    [E, d, inter]   uint8 + wq_down_exp    [E, d]       int8
+ *   wsq_gate_up   [2*inter, d] uint8 + wsq_gate_up_exp   [2*inter]  int8
+ *   wsq_down      [d, inter]   uint8 + wsq_down_exp      [d]        int8
+ * all from moe_quantize_fp8_rows (exponents outside [-124, 127] are not
+ * supported).  Per expert and token row:
+ *   x_t -> per-row E4M3 (codes, s_x);
+ *   g_n = 2^(s_gn + s_x) codes . codes, u_n likewise (fp32 accumulation);
+ *   h_n = bf16(silu(g_n) * u_n);  h -> per-row E4M3 (codes, s_h);
+ *   y_o = 2^(s_do + s_h) codes . codes;
+ * then the routing weights combine the y rows as in moe_layer_forward.  d and
+ * inter must be multiples of 128.  Errors as in moe_layer_forward.  The _ws
+ * form takes a caller-owned workspace of moe_workspace_size_w8a8(T, d, E, k,
+ * inter) bytes (0 for unsupported dimensions), 16-byte aligned.
+ */
+int moe_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
+                          int8_t* exps, void* stream);
+size_t moe_workspace_size_w8a8(int T, int d, int E, int k, int inter);
+int moe_layer_forward_w8a8(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                           const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                           const uint8_t* wq_down, const int8_t* wq_down_exp,
+                           const uint8_t* wsq_gate_up, const int8_t* wsq_gate_up_exp,
+                           const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
+                           int E, int k, int inter, float scale, uint16_t* out, void* stream);
+int moe_layer_forward_w8a8_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                              const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                              const uint8_t* wq_down, const int8_t* wq_down_exp,
+                              const uint8_t* wsq_gate_up, const int8_t* wsq_gate_up_exp,
+                              const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
+                              int E, int k, int inter, float scale, uint16_t* out,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Expert load balancing ("Kimi K2.5 Q&A", Q7.2; "Kimi K2.5 deep dive", CH10.2
  * step 2): the selection bias is a buffer outside the gradient, lowered for
  * over-loaded experts and raised for under-loaded ones, and a weak
@@ -320,7 +372,7 @@ void moe_set_wait_timeout_ns(uint64_t timeout_ns);
  */
 int moe_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
-/* Kernels the last moe_layer_forward / moe_layer_forward_ws launched. */
+/* Kernels the last layer call (any moe_layer_forward* entry) launched. */
 int moe_last_launch_count(void);
 
 /*
@@ -328,16 +380,18 @@ int moe_last_launch_count(void);
  * support; no counterpart in the method).  After moe_profile_begin(n), the
  * next n calls of moe_layer_forward / moe_layer_forward_ws on the current
  * device record one event before their first kernel and one after each
- * kernel, on the call's stream.  moe_profile_end synchronises those events,
- * writes into total_ms[i] (i < max_kernels) the summed time of the i-th
- * kernel of a call over the recorded calls, stores the number of recorded
- * calls in *n_calls, frees the events and returns the number of kernels per
- * call (or a negative moe_status).
+ * kernel, on the call's stream (all moe_layer_forward* entries).
+ * moe_profile_end synchronises those events, writes into total_ms[i]
+ * (i < max_kernels) the summed time of kernel slot i (moe_kernel_name) over
+ * the recorded calls, stores the number of recorded calls in *n_calls, frees
+ * the events and returns the number of slots per call (or a negative
+ * moe_status).  A slot a call has no kernel for (quantize_h outside FP8
+ * compute) sums to zero.
  */
 int moe_profile_begin(int max_calls);
 int moe_profile_end(float* total_ms, int max_kernels, int* n_calls);
 
-/* Name of the i-th kernel a layer call launches ("" if out of range). */
+/* Name of kernel slot i of a layer call ("" if out of range). */
 const char* moe_kernel_name(int i);
 
 #ifdef __cplusplus

@@ -244,11 +244,14 @@ def moe_rows_fp8(x, topk_idx, topk_w, expert_q, shared_q, tokens=None,
 def quantize_expert_rows(inputs: dict, experts):
     """The FP8-compute weights of the listed experts and of the shared expert,
     from the oracle's own row quantizer: ({e: (qgu, sgu, qdn, sdn)}, shared)."""
-    out = {}
-    for e in experts:
-        qg, sg = quantize_fp8_rows(inputs["w_gate_up"][e])
-        qd, sd = quantize_fp8_rows(inputs["w_down"][e])
-        out[e] = (qg, sg, qd, sd)
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(e):
+        return quantize_fp8_rows(inputs["w_gate_up"][e]) + quantize_fp8_rows(inputs["w_down"][e])
+
+    # the C quantizer runs outside the GIL: one expert per host thread
+    with ThreadPoolExecutor(max_workers=max(1, min(default_threads(), len(experts)))) as ex:
+        out = dict(zip(experts, ex.map(one, experts)))
     qg, sg = quantize_fp8_rows(inputs["ws_gate_up"])
     qd, sd = quantize_fp8_rows(inputs["ws_down"])
     return out, (qg, sg, qd, sd)

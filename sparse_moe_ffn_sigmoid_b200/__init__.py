@@ -22,7 +22,8 @@ __all__ = [
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
     "moe_layer_forward_noalloc", "moe_quantize_fp8", "moe_layer_forward_fp8",
     "moe_layer_forward_fp8_ws", "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
-    "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
+    "moe_layer_forward_w8a8_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
@@ -33,6 +34,8 @@ EXPORTED_SYMBOLS = [
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
     "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
     "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss", "moe_seq_aux_workspace_size",
+    "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
+    "moe_layer_forward_w8a8_ws",
 ]
 
 MOE_OK = 0
@@ -75,6 +78,10 @@ def _load():
         "moe_router_scores": ([P, P, I, I, I, P, P, SZ, P], I),
         "moe_seq_aux_loss": ([P, P, I, I, I, I, F, P, P, P, P, SZ, P], I),
         "moe_seq_aux_workspace_size": ([I, I, I], SZ),
+        "moe_quantize_fp8_rows": ([P, I64, I64, P, P, P], I),
+        "moe_workspace_size_w8a8": ([I, I, I, I, I], SZ),
+        "moe_layer_forward_w8a8": ([P] * 11 + [I, I, I, I, I, F, P, P], I),
+        "moe_layer_forward_w8a8_ws": ([P] * 11 + [I, I, I, I, I, F, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -262,6 +269,65 @@ def moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_d
                                        _ptr(workspace, torch.uint8, "workspace"),
                                        workspace.numel(), _stream(stream))
     _check("moe_layer_forward_fp8_ws", rc)
+
+
+def moe_quantize_fp8_rows(w, stream=None):
+    """bf16 weights [..., cols] (cols a multiple of 16) -> (E4M3 codes uint8
+    [..., cols], one int8 exponent per row [...]), new tensors on w's device."""
+    if w.dim() < 2:
+        raise ValueError("w must have at least 2 dimensions")
+    cols = w.shape[-1]
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    exps = torch.empty(tuple(w.shape[:-1]), dtype=torch.int8, device=w.device)
+    rc = _LIB.moe_quantize_fp8_rows(_ptr(w, BF16, "w"), w.numel() // cols, cols,
+                                    _ptr(q, torch.uint8, "q"), _ptr(exps, torch.int8, "exps"),
+                                    _stream(stream))
+    _check("moe_quantize_fp8_rows", rc)
+    return q, exps
+
+
+def moe_workspace_size_w8a8(T: int, d: int, E: int, k: int, inter: int) -> int:
+    return int(_LIB.moe_workspace_size_w8a8(T, d, E, k, inter))
+
+
+def _layer_w8a8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                     wsq_gate_up, wsq_gate_up_exp, wsq_down, wsq_down_exp):
+    T, d = x.shape
+    E = w_router.shape[0]
+    inter = wq_gate_up.shape[1] // 2
+    u8, i8 = torch.uint8, torch.int8
+    return ([_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"), _ptr(bias, F32, "bias"),
+             _ptr(wq_gate_up, u8, "wq_gate_up"), _ptr(wq_gate_up_exp, i8, "wq_gate_up_exp"),
+             _ptr(wq_down, u8, "wq_down"), _ptr(wq_down_exp, i8, "wq_down_exp"),
+             _ptr(wsq_gate_up, u8, "wsq_gate_up"), _ptr(wsq_gate_up_exp, i8, "wsq_gate_up_exp"),
+             _ptr(wsq_down, u8, "wsq_down"), _ptr(wsq_down_exp, i8, "wsq_down_exp")],
+            T, d, E, inter)
+
+
+def moe_layer_forward_w8a8(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                           wsq_gate_up, wsq_gate_up_exp, wsq_down, wsq_down_exp, k: int,
+                           scale: float, out, stream=None):
+    """The layer with FP8 compute in every expert: codes + per-row exponents
+    from moe_quantize_fp8_rows (routed [E, ...] and shared); router stays bf16."""
+    ptrs, T, d, E, inter = _layer_w8a8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp,
+                                            wq_down, wq_down_exp, wsq_gate_up, wsq_gate_up_exp,
+                                            wsq_down, wsq_down_exp)
+    rc = _LIB.moe_layer_forward_w8a8(*ptrs, T, d, E, k, inter, float(scale),
+                                     _ptr(out, BF16, "out"), _stream(stream))
+    _check("moe_layer_forward_w8a8", rc)
+
+
+def moe_layer_forward_w8a8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
+                              wq_down_exp, wsq_gate_up, wsq_gate_up_exp, wsq_down, wsq_down_exp,
+                              k: int, scale: float, out, workspace, stream=None):
+    ptrs, T, d, E, inter = _layer_w8a8_args(x, w_router, bias, wq_gate_up, wq_gate_up_exp,
+                                            wq_down, wq_down_exp, wsq_gate_up, wsq_gate_up_exp,
+                                            wsq_down, wsq_down_exp)
+    rc = _LIB.moe_layer_forward_w8a8_ws(*ptrs, T, d, E, k, inter, float(scale),
+                                        _ptr(out, BF16, "out"),
+                                        _ptr(workspace, torch.uint8, "workspace"),
+                                        workspace.numel(), _stream(stream))
+    _check("moe_layer_forward_w8a8_ws", rc)
 
 
 def moe_bias_update(counts, T: int, k: int, gamma: float, bias, stream=None):

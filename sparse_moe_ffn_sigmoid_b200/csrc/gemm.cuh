@@ -23,6 +23,10 @@
 // FP8-weight mode (480 threads): warps 2..5 are the epilogue (one per lane
 // quarter, every chunk), warps 6..9 and 11..14 dequantize E4M3 weight codes
 // into the bf16 weight ring (convert_weights).
+// FP8-compute mode (352 threads, the roles above): weights and tokens are
+// E4M3 codes with one exponent per row; a K step is 128 codes (the same
+// 128-byte rows), the MMAs are kind::f8f6f4 (K = 32), and the epilogue scales
+// each accumulator by 2^(weight row exponent + token row exponent).
 // Weights come from HBM and tokens mostly from L2, so the two operands have
 // separate rings: a deep one for weights (their HBM latency needs many bytes
 // in flight) and a short one for tokens.  K step q uses weight slot q % SA and
@@ -64,6 +68,13 @@ constexpr int kGemmThreadsFP8 = 480;
 constexpr int kSlabBytes8 = kSlabRows * kBK;  // one FP8 slab per K step (128 rows x 64 codes)
 constexpr int kTmemCols = 512;
 
+// Operand formats of a launch.
+enum GemmOperands : int {
+    kOpsBF16 = 0,       // bf16 weights and tokens (kind::f16)
+    kOpsW8Convert = 1,  // routed weights as block-scaled E4M3, dequantized in shared memory
+    kOpsFP8 = 2,        // E4M3 weights and tokens with per-row exponents (kind::f8f6f4)
+};
+
 enum GemmEpilogue : int {
     kEpiSwiGLU = 0,   // 2 slabs (gate, up) -> bf16 silu(gate) * up
     kEpiStoreBF16 = 1,// 1-2 slabs -> bf16
@@ -103,6 +114,10 @@ struct __align__(64) GemmArgs {
     const int8_t* a8_scale;
     int a8_kblocks;
     int stages_a8;            // FP8 code ring depth
+    // FP8-compute mode only: one int8 exponent per weight row (a_exp[map],
+    // indexed like the A rows) and per token row (b_exp[map], like the B rows)
+    const int8_t* a_exp[2];
+    const int8_t* b_exp[2];
 };
 
 __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int i) {
@@ -287,12 +302,16 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
     }
 }
 
-// FP8A: routed weights arrive as E4M3 codes and are dequantized in shared
-// memory by the converter warps (kGemmThreadsFP8 threads); FP8A = false is the
-// all-bf16 kernel (kGemmThreads threads).
-template <int EPI, bool FP8A>
-__global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
+// OPS (GemmOperands): kOpsW8Convert has routed weights arrive as E4M3 codes
+// that the converter warps dequantize in shared memory (kGemmThreadsFP8
+// threads); kOpsBF16 is the all-bf16 kernel and kOpsFP8 the FP8-compute one
+// (kGemmThreads threads).
+template <int EPI, int OPS>
+__global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmArgs args) {
+    constexpr bool FP8A = (OPS == kOpsW8Convert);
+    constexpr bool F8C = (OPS == kOpsFP8);
+    constexpr int kStepK = F8C ? 2 * kBK : kBK;   // K elements per step (128-byte rows)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -304,7 +323,7 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
     constexpr int nslab = (EPI == kEpiStoreF32) ? 1 : 2;
     const uint32_t a_bytes = nslab * kSlabBytes;
     const uint32_t b_bytes = args.n_max * kBK * 2;
-    static_assert(!FP8A || nslab == 2, "FP8 weights are for the expert GEMMs");
+    static_assert((!FP8A && !F8C) || nslab == 2, "FP8 weights are for the expert GEMMs");
     const int SA8 = FP8A ? args.stages_a8 : 0;
     constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
     uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
@@ -429,18 +448,19 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                     if (weights) {
                         uint8_t* sa = ring_a + rq.stage * a_bytes;
                         const CUtensorMap* am = &args.a_map[t.map];
-                        ptx::tma_load_2d_hint(sa, am, bar, ks * kBK, t.a_row0, pol);
+                        ptx::tma_load_2d_hint(sa, am, bar, ks * kStepK, t.a_row0, pol);
                         if (nslab == 2)
-                            ptx::tma_load_2d_hint(sa + kSlabBytes, am, bar, ks * kBK, t.a_row1, pol);
+                            ptx::tma_load_2d_hint(sa + kSlabBytes, am, bar, ks * kStepK, t.a_row1,
+                                                  pol);
                     } else {
                         uint8_t* sb = ring_b + rb.stage * b_bytes;
                         int r = 0;
                         for (; r + kBoxRowsBig <= npad; r += kBoxRowsBig)
                             ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map64[t.map], bar,
-                                                  ks * kBK, t.b_row0 + r, pol);
+                                                  ks * kStepK, t.b_row0 + r, pol);
                         for (; r < npad; r += kBoxRows)
                             ptx::tma_load_2d_hint(sb + r * kBK * 2, &args.b_map[t.map], bar,
-                                                  ks * kBK, t.b_row0 + r, pol);
+                                                  ks * kStepK, t.b_row0 + r, pol);
                     }
                     issued |= 1u << rq.stage;
                     issued_parity = (issued_parity & ~(1u << rq.stage)) | (rq.phase << rq.stage);
@@ -470,7 +490,8 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
             for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
                 const Tile t = load_tile(args, i);
                 const int npad = pad16(t.n);
-                const uint32_t idesc = ptx::idesc_bf16_f32(kSlabRows, npad);
+                const uint32_t idesc = F8C ? ptx::idesc_e4m3_f32(kSlabRows, npad)
+                                           : ptx::idesc_bf16_f32(kSlabRows, npad);
                 // single-slab tiles of 32+ tokens: two N halves (multiples of 16)
                 const int n_lo = (nslab == 1 && npad >= 32) ? pad16(npad / 2) : npad;
                 const int n_hi = npad - n_lo;
@@ -492,8 +513,9 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                     // (the two slabs, or the two N halves of a single-slab tile): back-
                     // to-back MMAs into one accumulator wait on each other.  The
                     // descriptors' start-address field holds (address >> 4), so a slot,
-                    // slab or K offset of B bytes is an addition of B >> 4 (K by 16
-                    // elements = 32 B = +2); shared addresses stay below 2^18.
+                    // slab or K offset of B bytes is an addition of B >> 4 (one MMA's K,
+                    // 16 bf16 or 32 E4M3 elements = 32 B, is +2); shared addresses stay
+                    // below 2^18.
                     const uint64_t a0 = desc_ring_a + ra.stage * (a_bytes >> 4);
                     const uint64_t a1 = a0 + (kSlabBytes >> 4);
                     const uint64_t b0 = desc_ring_b + rb.stage * (b_bytes >> 4);
@@ -501,7 +523,10 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         const uint32_t acc = (ks > t.ks0 || kk > 0) ? 1u : 0u;
-                        if (nslab == 2) {
+                        if (F8C) {
+                            ptx::tc_mma_e4m3(dcol, a0 + 2 * kk, b0 + 2 * kk, idesc, acc);
+                            ptx::tc_mma_e4m3(dcol + args.n_max, a1 + 2 * kk, b0 + 2 * kk, idesc, acc);
+                        } else if (nslab == 2) {
                             ptx::tc_mma_bf16(dcol, a0 + 2 * kk, b0 + 2 * kk, idesc, acc);
                             ptx::tc_mma_bf16(dcol + args.n_max, a1 + 2 * kk, b0 + 2 * kk, idesc, acc);
                         } else if (n_hi > 0) {
@@ -570,9 +595,21 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                 constexpr bool kSwiGLU = (EPI == kEpiSwiGLU);
                 const int nout = kSwiGLU ? 1 : nslab;
                 bf16* out = static_cast<bf16*>(args.out);
+                // FP8 compute: this lane's weight row exponents (gate and up rows, or
+                // the row of each output slab) and the tile's token row exponents
+                [[maybe_unused]] const int8_t* bexp = F8C ? args.b_exp[t.map] + t.b_row0 : nullptr;
+                int ew0 = 0, ew1 = 0;
+                if constexpr (F8C) {
+                    const int8_t* aexp = args.a_exp[t.map];
+                    const int f0 = t.out_col0 + q * 32 + lane;
+                    if (kSwiGLU || f0 < args.col_limit) ew0 = aexp[t.a_row0 + q * 32 + lane];
+                    if (kSwiGLU || f0 + kSlabRows < args.col_limit)
+                        ew1 = aexp[t.a_row1 + q * 32 + lane];
+                }
                 for (int s = 0; s < nout; ++s) {
                     const int fbase = t.out_col0 + s * kSlabRows + q * 32;
                     const uint32_t ts = tq + s * args.n_max;
+                    [[maybe_unused]] const int ews = s == 0 ? ew0 : ew1;
                     for (int c0 = kStageRows * half; c0 < npad; c0 += kChunkStep) {
                         const int ncol = min(kStageRows, npad - c0);     // 32 or 16 (uniform)
                         float v[kStageRows];
@@ -587,9 +624,19 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                                                  *reinterpret_cast<uint32_t(*)[16]>(u));
                             }
                             ptx::tmem_wait_ld();
+                            if constexpr (F8C) {
+                                const int ex = c0 + lane < t.n ? bexp[c0 + lane] : 0;
 #pragma unroll
-                            for (int j = 0; j < kStageRows; ++j)
-                                v[j] = silu_fast(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                                for (int j = 0; j < kStageRows; ++j) {
+                                    const int ej = __shfl_sync(0xffffffffu, ex, j);
+                                    v[j] = silu_fast(mul_pow2(__uint_as_float(g[j]), ew0 + ej)) *
+                                           mul_pow2(__uint_as_float(u[j]), ew1 + ej);
+                                }
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < kStageRows; ++j)
+                                    v[j] = silu_fast(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                            }
                         } else {
                             uint32_t r[kStageRows];
                             if (ncol == kStageRows)
@@ -597,8 +644,16 @@ __global__ void __launch_bounds__(FP8A ? kGemmThreadsFP8 : kGemmThreads, 1)
                             else
                                 ptx::tmem_ld_x16(ts + c0, *reinterpret_cast<uint32_t(*)[16]>(r));
                             ptx::tmem_wait_ld();
+                            if constexpr (F8C) {
+                                const int ex = c0 + lane < t.n ? bexp[c0 + lane] : 0;
 #pragma unroll
-                            for (int j = 0; j < kStageRows; ++j) v[j] = __uint_as_float(r[j]);
+                                for (int j = 0; j < kStageRows; ++j)
+                                    v[j] = mul_pow2(__uint_as_float(r[j]),
+                                                    ews + __shfl_sync(0xffffffffu, ex, j));
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < kStageRows; ++j) v[j] = __uint_as_float(r[j]);
+                            }
                         }
                         store_block_bf16(stg, v, ncol, out, args.out_ld, t.out_row0 + c0,
                                          min(ncol, t.n - c0), fbase, args.col_limit, lane);

@@ -39,11 +39,13 @@ constexpr int kTopkBlockTokens = 512;      // top-k launch shape switch (tokens 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 std::atomic<int> g_last_launches{0};
 
-// Kernels of one layer call, in launch order (moe_kernel_name).
-constexpr int kLayerKernels = 9;
+// Kernels of one layer call, in launch order (moe_kernel_name).  gather_rows
+// also quantizes the rows in FP8 compute; quantize_h (the activation rows'
+// FP8 quantization) runs in FP8 compute only.
+constexpr int kLayerKernels = 10;
 const char* const kKernelNames[kLayerKernels] = {
     "router_gemm", "topk", "permute_hist", "scan_plan", "permute_scatter",
-    "gather_rows", "gemm_gate_up_swiglu", "gemm_down", "combine"};
+    "gather_rows", "gemm_gate_up_swiglu", "quantize_h", "gemm_down", "combine"};
 
 // Optional per-kernel CUDA-event timing of layer calls (moe_profile_begin/end).
 struct Profile {
@@ -57,11 +59,17 @@ struct Profile {
 // records an event on the stream after each of them.
 struct Recorder {
     cudaEvent_t* ev = nullptr;     // kLayerKernels + 1 events, or null
-    int n = 0;
+    int n = 0;                     // slots passed
+    int launches = 0;              // kernels launched
     void start(cudaStream_t st) {
         if (ev) cudaEventRecord(ev[0], st);
     }
     void mark(cudaStream_t st) {
+        ++launches;
+        skip(st);
+    }
+    // a slot this call has no kernel for (it times as zero)
+    void skip(cudaStream_t st) {
         ++n;
         if (ev && n <= kLayerKernels) cudaEventRecord(ev[n], st);
     }
@@ -114,13 +122,18 @@ int router_splits(int T, int d, int E) {
 
 struct Layout {
     size_t partials, topk_idx, topk_w, blk, counts, offsets, row_token, slot_row;
-    size_t tiles1, tiles2, ntiles, xperm, h, y, total;
+    size_t tiles1, tiles2, ntiles, xperm, h, y;
+    // FP8 compute: the token rows' codes live in xperm (T*k permuted rows, then
+    // the T rows in token order); their exponents, the activation's codes and
+    // its exponents in regions of their own
+    size_t xexp, hq, hexp;
+    size_t total;
     int splits, nblk, max_tiles1, max_tiles2;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-Layout make_layout(int T, int d, int E, int k, int inter) {
+Layout make_layout(int T, int d, int E, int k, int inter, bool fp8_compute = false) {
     Layout L{};
     const size_t Tk = static_cast<size_t>(T) * k;
     const size_t rows = Tk + T;   // routed rows, then the shared expert's rows
@@ -151,6 +164,11 @@ Layout make_layout(int T, int d, int E, int k, int inter) {
     L.xperm = take(Tk * d * sizeof(bf16));
     L.h = take(rows * inter * sizeof(bf16));
     L.y = take(rows * d * sizeof(bf16));
+    if (fp8_compute) {
+        L.xexp = take(rows);
+        L.hq = take(rows * inter);
+        L.hexp = take(rows);
+    }
     L.total = off;
     return L;
 }
@@ -174,11 +192,15 @@ int device_info(DeviceInfo* out) {
             return MOE_ERR_CUDA;
         const int smem = static_cast<int>(kMaxDynSmem);
         const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
-        if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, false>, dyn, smem) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, false>, dyn, smem) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32, false>, dyn, smem) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, true>, dyn, smem) != cudaSuccess ||
-            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, true>, dyn, smem) != cudaSuccess ||
+        if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsBF16>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsBF16>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreF32, kOpsBF16>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsW8Convert>, dyn, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsW8Convert>, dyn, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsFP8>, dyn, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsFP8>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(scan_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kScanSmem)) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -220,6 +242,22 @@ bool make_map8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major E4M3 code matrix [rows, cols] (uint8) read in boxes of box_rows x
+// 128 codes, 128-byte swizzled: the operand layout of the FP8-compute MMAs.
+bool make_map_e4m3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(2 * kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -274,12 +312,13 @@ void fill_pipeline_fp8(GemmArgs& a, int n_max) {
     a.stages_a8 = static_cast<int>(std::min<size_t>(12, left / a8_bytes));
 }
 
-template <int EPI, bool FP8A = false>
+template <int EPI, int OPS = kOpsBF16>
 int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
+    constexpr bool FP8A = (OPS == kOpsW8Convert);
     const size_t smem =
         gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max, FP8A ? a.stages_a8 : 0);
     if (smem > kMaxDynSmem || (FP8A && a.stages_a8 < 2)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    moe_gemm_kernel<EPI, FP8A><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
+    moe_gemm_kernel<EPI, OPS><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -308,7 +347,7 @@ int launch_router_gemm(const DeviceInfo& di, const bf16* x, const bf16* wr, int 
     a.out_ld = E;
     a.col_limit = E;
     fill_pipeline(a, 1, chunk);
-    return launch_gemm<kEpiStoreF32, false>(a, std::min(a.ntiles_host, di.sms), st);
+    return launch_gemm<kEpiStoreF32>(a, std::min(a.ntiles_host, di.sms), st);
 }
 
 int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const float* bias, int T,
@@ -424,13 +463,14 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     int rc;
     if (f8 != nullptr) {
         fill_pipeline_fp8(g1, n_max);
-        rc = launch_gemm<kEpiSwiGLU, true>(g1, std::min(max_tiles1, di.sms), st);
+        rc = launch_gemm<kEpiSwiGLU, kOpsW8Convert>(g1, std::min(max_tiles1, di.sms), st);
     } else {
         fill_pipeline(g1, 2, n_max);
         rc = launch_gemm<kEpiSwiGLU>(g1, std::min(max_tiles1, di.sms), st);
     }
     if (rc != MOE_OK) return rc;
     rec.mark(st);
+    rec.skip(st);   // no activation quantization
 
     GemmArgs g2;
     std::memset(&g2, 0, sizeof(g2));
@@ -460,7 +500,7 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     g2.col_limit = d;
     if (f8 != nullptr) {
         fill_pipeline_fp8(g2, n_max);
-        rc = launch_gemm<kEpiStoreBF16, true>(g2, std::min(max_tiles2, di.sms), st);
+        rc = launch_gemm<kEpiStoreBF16, kOpsW8Convert>(g2, std::min(max_tiles2, di.sms), st);
     } else {
         fill_pipeline(g2, 2, n_max);
         rc = launch_gemm<kEpiStoreBF16>(g2, std::min(max_tiles2, di.sms), st);
@@ -468,6 +508,94 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     if (rc != MOE_OK) return rc;
     rec.mark(st);
     return MOE_OK;
+}
+
+// FP8 compute: every expert's weights (routed and shared) as E4M3 codes with
+// one int8 exponent per row (quant.cuh): gate|up [E, 2I, d] + [E, 2I], down
+// [E, d, I] + [E, d], shared gate|up [2I, d] + [2I], shared down [d, I] + [d].
+struct Fp8Rows {
+    const uint8_t* gate_up;
+    const int8_t* gate_up_exp;
+    const uint8_t* down;
+    const int8_t* down_exp;
+    const uint8_t* s_gate_up;
+    const int8_t* s_gate_up_exp;
+    const uint8_t* s_down;
+    const int8_t* s_down_exp;
+};
+
+// FP8-compute FFN over a planned tile list (tiles with K steps of 2 * kBK):
+//   1. the token rows to E4M3 per row: the T*k permuted rows (a gather through
+//      row_token) then the T rows in token order, codes xq, exponents xexp
+//   2. gate|up on codes (kind::f8f6f4), SwiGLU epilogue with the exponents -> h
+//   3. h's rows to E4M3 per row -> hq, hexp
+//   4. down on codes -> y (bf16)
+int launch_ffn_fp8(const DeviceInfo& di, const bf16* x, const int* row_token, int T, int d,
+                   int E, int k, int inter, const Fp8Rows& w, uint8_t* xq, int8_t* xexp, bf16* h,
+                   uint8_t* hq, int8_t* hexp, bf16* y, const int4* tiles1, const int4* tiles2,
+                   const int* ntiles, int max_tiles1, int max_tiles2, cudaStream_t st,
+                   Recorder& rec) {
+    const long long rows_routed = static_cast<long long>(T) * k;
+    const long long rows_all = rows_routed + T;
+    const unsigned qblocks = static_cast<unsigned>((rows_all + kRowQuantWarps - 1) / kRowQuantWarps);
+    fp8_quantize_rows_kernel<<<qblocks, 32 * kRowQuantWarps, 0, st>>>(
+        x, d, row_token, rows_routed, T, rows_all, d, xq, xexp);
+    rec.mark(st);
+    const int n_max = std::min(kTileN, (T + 15) & ~15);
+    const uint8_t* xq_tok = xq + rows_routed * d;
+
+    GemmArgs g1;
+    std::memset(&g1, 0, sizeof(g1));
+    const uint64_t rr = static_cast<uint64_t>(std::max<long long>(rows_routed, 1));
+    if (!make_map_e4m3(&g1.a_map[0], w.gate_up, static_cast<uint64_t>(E) * 2 * inter, d,
+                       kSlabRows) ||
+        !make_map_e4m3(&g1.a_map[1], w.s_gate_up, 2ull * inter, d, kSlabRows) ||
+        !make_map_e4m3(&g1.b_map[0], xq, rr, d, kBoxRows) ||
+        !make_map_e4m3(&g1.b_map64[0], xq, rr, d, kBoxRowsBig) ||
+        !make_map_e4m3(&g1.b_map[1], xq_tok, T, d, kBoxRows) ||
+        !make_map_e4m3(&g1.b_map64[1], xq_tok, T, d, kBoxRowsBig))
+        return MOE_ERR_CUDA;
+    g1.a_exp[0] = w.gate_up_exp;
+    g1.a_exp[1] = w.s_gate_up_exp;
+    g1.b_exp[0] = xexp;
+    g1.b_exp[1] = xexp + rows_routed;
+    g1.tiles = tiles1;
+    g1.ntiles_dev = ntiles;
+    g1.out = h;
+    g1.out_ld = inter;
+    g1.col_limit = inter;
+    fill_pipeline(g1, 2, n_max);
+    int rc = launch_gemm<kEpiSwiGLU, kOpsFP8>(g1, std::min(max_tiles1, di.sms), st);
+    if (rc != MOE_OK) return rc;
+    rec.mark(st);
+
+    fp8_quantize_rows_kernel<<<qblocks, 32 * kRowQuantWarps, 0, st>>>(
+        h, inter, nullptr, 0, rows_all, rows_all, inter, hq, hexp);
+    rec.mark(st);
+
+    GemmArgs g2;
+    std::memset(&g2, 0, sizeof(g2));
+    if (!make_map_e4m3(&g2.a_map[0], w.down, static_cast<uint64_t>(E) * d, inter, kSlabRows) ||
+        !make_map_e4m3(&g2.a_map[1], w.s_down, d, inter, kSlabRows) ||
+        !make_map_e4m3(&g2.b_map[0], hq, rows_all, inter, kBoxRows) ||
+        !make_map_e4m3(&g2.b_map64[0], hq, rows_all, inter, kBoxRowsBig))
+        return MOE_ERR_CUDA;
+    g2.b_map[1] = g2.b_map[0];
+    g2.b_map64[1] = g2.b_map64[0];
+    g2.a_exp[0] = w.down_exp;
+    g2.a_exp[1] = w.s_down_exp;
+    g2.b_exp[0] = hexp;
+    g2.b_exp[1] = hexp;
+    g2.tiles = tiles2;
+    g2.ntiles_dev = ntiles + 1;
+    g2.out = y;
+    g2.out_ld = d;
+    g2.col_limit = d;
+    fill_pipeline(g2, 2, n_max);
+    rc = launch_gemm<kEpiStoreBF16, kOpsFP8>(g2, std::min(max_tiles2, di.sms), st);
+    if (rc != MOE_OK) return rc;
+    rec.mark(st);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* slot_row, int T,
@@ -494,8 +622,8 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
 int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* wgu,
                   const bf16* wdn, const bf16* sgu, const bf16* sdn, int T, int d, int E, int k,
                   int inter, float scale, bf16* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                  const Fp8Experts* f8 = nullptr) {
-    const Layout L = make_layout(T, d, E, k, inter);
+                  const Fp8Experts* f8 = nullptr, const Fp8Rows* f8c = nullptr) {
+    const Layout L = make_layout(T, d, E, k, inter, f8c != nullptr);
     if (ws == nullptr || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
     DeviceInfo di;
     int rc = device_info(&di);
@@ -527,14 +655,21 @@ int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* 
                       reinterpret_cast<float*>(P(L.partials)), L.splits, st, rec);
     if (rc != MOE_OK) return rc;
     PlanArgs plan{E, 1, T, d, inter, T * k, tiles1, tiles2, ntiles};
+    if (f8c != nullptr) plan.kstep = 2 * kBK;
     rc = launch_permute(idx, T, E, k, counts, offsets, row_token, slot_row,
                         reinterpret_cast<int*>(P(L.blk)), plan, st, rec);
     if (rc != MOE_OK) return rc;
-    rc = launch_ffn(di, x, row_token, T, d, E, k, inter, wgu, wdn, sgu, sdn, true, xperm, h, y,
-                    tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8);
+    if (f8c != nullptr)
+        rc = launch_ffn_fp8(di, x, row_token, T, d, E, k, inter, *f8c,
+                            reinterpret_cast<uint8_t*>(xperm), reinterpret_cast<int8_t*>(P(L.xexp)),
+                            h, P(L.hq), reinterpret_cast<int8_t*>(P(L.hexp)), y, tiles1, tiles2,
+                            ntiles, L.max_tiles1, L.max_tiles2, st, rec);
+    else
+        rc = launch_ffn(di, x, row_token, T, d, E, k, inter, wgu, wdn, sgu, sdn, true, xperm, h,
+                        y, tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8);
     if (rc != MOE_OK) return rc;
     rc = launch_combine(y, y + static_cast<size_t>(T) * k * d, w, slot_row, T, d, k, out, st, rec);
-    g_last_launches.store(rec.n);
+    g_last_launches.store(rec.launches);
     return rc;
 }
 
@@ -821,6 +956,73 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
     return moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
                                     wq_down_exp, ws_gate_up, ws_down, T, d, E, k, inter, scale,
                                     out, ws, need, stream);
+}
+
+int moe_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
+                          int8_t* exps, void* stream) {
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || cols > 0x7FFFFFFF ||
+        rows > 0x7FFFFFFFll * kRowQuantWarps)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!all_ok(w, q) || exps == nullptr) return MOE_ERR_INVALID_ARG;
+    const unsigned blocks = static_cast<unsigned>((rows + kRowQuantWarps - 1) / kRowQuantWarps);
+    fp8_quantize_rows_kernel<<<blocks, 32 * kRowQuantWarps, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const bf16*>(w), cols, nullptr, 0, rows, rows, static_cast<int>(cols), q,
+        exps);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_workspace_size_w8a8(int T, int d, int E, int k, int inter) {
+    if (check_dims(T, d, E, k, inter) != MOE_OK) return 0;
+    return make_layout(T, d, E, k, inter, true).total;
+}
+
+int moe_layer_forward_w8a8_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                              const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                              const uint8_t* wq_down, const int8_t* wq_down_exp,
+                              const uint8_t* wsq_gate_up, const int8_t* wsq_gate_up_exp,
+                              const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
+                              int E, int k, int inter, float scale, uint16_t* out,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (d % (2 * kBK) != 0 || inter % (2 * kBK) != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_down, wsq_gate_up, wsq_down, out, workspace) ||
+        wq_gate_up_exp == nullptr || wq_down_exp == nullptr || wsq_gate_up_exp == nullptr ||
+        wsq_down_exp == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    const Fp8Rows f8c{wq_gate_up, wq_gate_up_exp, wq_down, wq_down_exp,
+                      wsq_gate_up, wsq_gate_up_exp, wsq_down, wsq_down_exp};
+    return layer_forward(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                         bias, nullptr, nullptr, nullptr, nullptr, T, d, E, k, inter, scale,
+                         reinterpret_cast<bf16*>(out), workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream), nullptr, &f8c);
+}
+
+int moe_layer_forward_w8a8(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                           const uint8_t* wq_gate_up, const int8_t* wq_gate_up_exp,
+                           const uint8_t* wq_down, const int8_t* wq_down_exp,
+                           const uint8_t* wsq_gate_up, const int8_t* wsq_gate_up_exp,
+                           const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
+                           int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (d % (2 * kBK) != 0 || inter % (2 * kBK) != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_down, wsq_gate_up, wsq_down, out) ||
+        wq_gate_up_exp == nullptr || wq_down_exp == nullptr || wsq_gate_up_exp == nullptr ||
+        wsq_down_exp == nullptr || !(scale == scale))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = make_layout(T, d, E, k, inter, true).total;
+    void* ws = nullptr;
+    rc = owned_workspace(static_cast<cudaStream_t>(stream), need, &ws);
+    if (rc != MOE_OK) return rc;
+    return moe_layer_forward_w8a8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
+                                     wq_down_exp, wsq_gate_up, wsq_gate_up_exp, wsq_down,
+                                     wsq_down_exp, T, d, E, k, inter, scale, out, ws, need,
+                                     stream);
 }
 
 // Scratch of moe_seq_aux_loss: 1 / (token score sums) [B*S], the per-block

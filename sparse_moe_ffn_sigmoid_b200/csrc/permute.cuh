@@ -87,6 +87,7 @@ struct PlanArgs {
     int4* tiles1;          // gate|up tiles
     int4* tiles2;          // down tiles
     int* ntiles;           // [0] = gate|up count, [1] = down count
+    int kstep = kBK;       // K elements per GEMM step (FP8 compute: 2 * kBK)
 };
 
 constexpr int kPlanMaxG = 1025;   // up to 1024 routed experts and the shared one
@@ -108,13 +109,13 @@ __device__ __forceinline__ void plan_tile(const PlanArgs& p, int g, int c, int r
     if (!down) {
         const int a0 = e * 2 * p.inter + f * kSlabRows;
         p.tiles1[2 * pos] = make_int4(a0, a0 + p.inter, b_row, n | (map << 16));
-        p.tiles1[2 * pos + 1] = make_int4(out_row, f * kSlabRows, 0, p.d / kBK);
+        p.tiles1[2 * pos + 1] = make_int4(out_row, f * kSlabRows, 0, p.d / p.kstep);
     } else {
         const int a0 = e * p.d + f * 2 * kSlabRows;
         // down reads h rows where gate|up wrote them; both B map slots of the
         // down launch point at h, the slot only picks routed / shared weights
         p.tiles2[2 * pos] = make_int4(a0, a0 + kSlabRows, out_row, n | (map << 16));
-        p.tiles2[2 * pos + 1] = make_int4(out_row, f * 2 * kSlabRows, 0, p.inter / kBK);
+        p.tiles2[2 * pos + 1] = make_int4(out_row, f * 2 * kSlabRows, 0, p.inter / p.kstep);
     }
 }
 

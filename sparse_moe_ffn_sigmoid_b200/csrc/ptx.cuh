@@ -163,6 +163,18 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with E4M3 A and B (kind::f8f6f4, K = 32 per
+// instruction: the same 32 bytes of a 128-byte row as a bf16 K = 16 step).
+__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // 32 lanes x 32 bits, 16 consecutive columns: thread i of the warp gets TMEM
 // lane (base_lane + i), columns [col, col+16).
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -215,6 +227,14 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
 // 17-22, M>>4 at bits 24-28.
 __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3
+// (format code 0 in bits 7-9 and 10-12), both K-major, N>>3 at bits 17-22,
+// M>>4 at bits 24-28.
+__host__ __device__ __forceinline__ uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 

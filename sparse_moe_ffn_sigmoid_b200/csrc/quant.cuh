@@ -139,4 +139,80 @@ __device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 v, const Fp8Scale& sc) {
     return out;
 }
 
+// ------------------------------------------------------------- FP8 compute
+// Operands of the FP8-compute GEMMs ("Kimi K2.5 Q&A", Q7.1: V3 computes in
+// FP8): E4M3 codes with one power-of-two exponent per ROW (a weight row is an
+// output channel, an activation row a token), by the same smallest-exponent
+// rule as the blocks above.  The exponents factor out of every K sum, so the
+// tensor cores multiply codes and the epilogue applies 2^(s_w + s_x) exactly.
+
+constexpr int kRowQuantWarps = 8;         // rows per block (one warp each)
+
+// Row r of q [rows, cols] / sexp [rows] is the quantization of source row
+// row_map[r] (r < n_map: a gather) or r - n_map (after it) of src (bf16,
+// leading dimension ld, src_rows rows).  A source index out of range zeroes
+// the row and records kStatusInvalidArg.  cols: a multiple of 8.
+__global__ void __launch_bounds__(32 * kRowQuantWarps) fp8_quantize_rows_kernel(
+    const bf16* __restrict__ src, long long ld, const int* __restrict__ row_map, long long n_map,
+    long long src_rows, long long rows, int cols, uint8_t* __restrict__ q,
+    int8_t* __restrict__ sexp) {
+    const long long r = static_cast<long long>(blockIdx.x) * kRowQuantWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const long long sr = r < n_map ? static_cast<long long>(row_map[r]) : r - n_map;
+    uint2* qr = reinterpret_cast<uint2*>(q + r * cols);
+    const int nv = cols / 8;
+    if (sr < 0 || sr >= src_rows) {
+        if (lane == 0) {
+            record_status(kStatusInvalidArg);
+            sexp[r] = 0;
+        }
+        for (int v = lane; v < nv; v += 32) qr[v] = make_uint2(0u, 0u);
+        return;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(src + sr * ld);
+    float amax = 0.0f;
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) {
+        const uint4 u = __ldg(s + v);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int e = fp8_block_exponent(amax);
+    if (lane == 0) sexp[r] = static_cast<int8_t>(e);
+    // w * 2^-e in two exact steps (2^-e alone may be below the normal range)
+    const float m1 = pow2f(-(e / 2));
+    const float m2 = pow2f(-(e - e / 2));
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) {
+        const uint4 u = __ldg(s + v);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint2 out;
+        uint8_t* o = reinterpret_cast<uint8_t*>(&out);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            o[2 * j] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.x, m1), m2), __NV_SATFINITE,
+                                             __NV_E4M3);
+            o[2 * j + 1] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.y, m1), m2),
+                                                 __NV_SATFINITE, __NV_E4M3);
+        }
+        qr[v] = out;
+    }
+}
+
+// v * 2^e for the sum of two row exponents (e in [-248, 254] for exponents the
+// quantizers produce), in two power-of-two factors that are normal floats.
+__device__ __forceinline__ float mul_pow2(float v, int e) {
+    const int e1 = max(-126, min(127, e >> 1));
+    const int e2 = max(-126, min(127, e - e1));
+    return __fmul_rn(__fmul_rn(v, pow2f(e1)), pow2f(e2));
+}
+
 }  // namespace moe

@@ -146,6 +146,53 @@ def test_quantize_fp8_rejects_bad_shapes():
     assert L.moe_quantize_fp8(FAKE, 128, 128, FAKE, NULL, NULL) == INVALID
 
 
+# ------------------------------------------------------------ FP8 compute
+
+def _layer_w8a8(T=64, d=7168, E=384, k=8, inter=2048, scale=2.827, ptrs=None, out=FAKE,
+                ws=None):
+    p = ptrs if ptrs is not None else [FAKE] * 11
+    L = moe.lib()
+    if ws is None:
+        return L.moe_layer_forward_w8a8(*p, T, d, E, k, inter, ctypes.c_float(scale), out, NULL)
+    return L.moe_layer_forward_w8a8_ws(*p, T, d, E, k, inter, ctypes.c_float(scale), out, FAKE,
+                                       ws, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=7104), SHAPE), (dict(inter=2112), SHAPE), (dict(d=7100), SHAPE), (dict(E=0), SHAPE),
+    (dict(k=9, E=8), SHAPE), (dict(T=-1), INVALID), (dict(scale=float("nan")), INVALID),
+])
+def test_w8a8_layer_rejects_bad_shapes(kw, code):
+    # K steps of 128 codes: d and inter must be multiples of 128
+    assert _layer_w8a8(**kw) == code
+
+
+def test_w8a8_layer_rejects_null_pointers_and_small_workspace():
+    for i in range(11):
+        p = [FAKE] * 11
+        p[i] = NULL
+        assert _layer_w8a8(ptrs=p) == INVALID
+    assert _layer_w8a8(out=NULL) == INVALID
+    need = moe.moe_workspace_size_w8a8(64, 7168, 384, 8, 2048)
+    # the bf16 layer's workspace is too small: the codes' exponents and the
+    # activation's codes need room of their own
+    assert need > moe.moe_workspace_size(64, 7168, 384, 8, 2048)
+    assert _layer_w8a8(ws=need - 1) == INVALID
+    assert _layer_w8a8(T=0) == OK
+    assert moe.moe_workspace_size_w8a8(64, 7100, 384, 8, 2048) == 0
+
+
+def test_quantize_fp8_rows_rejects_bad_shapes():
+    L = moe.lib()
+    assert L.moe_quantize_fp8_rows(FAKE, 100, 120, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_fp8_rows(FAKE, -1, 128, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_fp8_rows(FAKE, 0, 128, FAKE, FAKE, NULL) == OK
+    assert L.moe_quantize_fp8_rows(FAKE, 5, 0, FAKE, FAKE, NULL) == OK
+    assert L.moe_quantize_fp8_rows(NULL, 5, 128, FAKE, FAKE, NULL) == INVALID
+    assert L.moe_quantize_fp8_rows(FAKE, 5, 128, ctypes.c_void_p(0x10008), FAKE, NULL) == INVALID
+    assert L.moe_quantize_fp8_rows(FAKE, 5, 128, FAKE, NULL, NULL) == INVALID
+
+
 # ------------------------------------------------------------ load balance
 
 def test_balance_calls_reject_bad_arguments():

@@ -244,7 +244,8 @@ def test_layer_deterministic_and_ws_variant(moe):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
     kernels = [moe.moe_kernel_name(i) for i in range(32) if moe.moe_kernel_name(i)]
-    assert moe.moe_last_launch_count() == len(kernels)
+    # every slot but the activation quantizer of FP8 compute
+    assert moe.moe_last_launch_count() == len([n for n in kernels if n != "quantize_h"])
 
 
 def test_staged_calls_compose_to_layer(moe):
