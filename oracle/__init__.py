@@ -82,6 +82,10 @@ def _bind(L):
     L.oracle_quantize_fp8.restype = i32
     L.oracle_dequantize_fp8.argtypes = [P, P, i64, i64, P]
     L.oracle_dequantize_fp8.restype = i32
+    L.oracle_quantize_int4.argtypes = [P, i64, i64, P, P]
+    L.oracle_quantize_int4.restype = i32
+    L.oracle_dequantize_int4.argtypes = [P, P, i64, i64, P]
+    L.oracle_dequantize_int4.restype = i32
     L.oracle_quantize_fp8_rows.argtypes = [P, i64, i64, P, P]
     L.oracle_quantize_fp8_rows.restype = None
     L.oracle_swiglu_row_fp8.argtypes = [P, P, P, P, P, i32, i32, P]
@@ -174,6 +178,31 @@ def dequantize_fp8(q, sexp):
     rc = lib().oracle_dequantize_fp8(_ptr(q), _ptr(sexp), rows, cols, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_dequantize_fp8: rows and cols must be multiples of 128")
+    return out
+
+
+def quantize_int4(w):
+    """bf16 matrix [.., rows, cols] (cols a multiple of 32) -> (codes int8 in
+    [-8, 7], same shape; group scales as bf16 bits uint16 [.., rows, cols/32])."""
+    u = _u16(w)
+    cols = u.shape[-1]
+    rows = u.size // cols
+    q = np.empty(u.shape, dtype=np.int8)
+    sc = np.empty(u.shape[:-1] + (cols // 32,), dtype=np.uint16)
+    if lib().oracle_quantize_int4(_ptr(u), rows, cols, _ptr(q), _ptr(sc)) != 0:
+        raise ValueError("oracle_quantize_int4: cols must be a multiple of 32")
+    return q, sc
+
+
+def dequantize_int4(q, scale):
+    """codes + group scales -> the bf16 weights the model computes with (uint16)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    sc = np.ascontiguousarray(scale, dtype=np.uint16)
+    cols = q.shape[-1]
+    rows = q.size // cols
+    out = np.empty(q.shape, dtype=np.uint16)
+    if lib().oracle_dequantize_int4(_ptr(q), _ptr(sc), rows, cols, _ptr(out)) != 0:
+        raise ValueError("oracle_dequantize_int4: cols must be a multiple of 32")
     return out
 
 

@@ -510,3 +510,46 @@ int oracle_moe_rows_fp8(const uint16_t* x, int T, int d, int E, int k, int inter
     oracle_parallel_for(n_tokens, nthreads, rows8_tokens, &c);
     return 0;
 }
+
+/* ------------------------------------------------------------ INT4 storage */
+
+int oracle_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, int8_t* q,
+                         uint16_t* scale) {
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+    const int64_t groups = cols / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const uint16_t* wg = w + r * cols + g * 32;
+            int8_t* qg = q + r * cols + g * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                const double v = fabs(oracle_bf16_to_f64(wg[i]));
+                if (v > amax) amax = v;
+            }
+            const uint16_t sb = oracle_f64_to_bf16(amax / 7.0);
+            scale[r * groups + g] = sb;
+            const double sv = oracle_bf16_to_f64(sb);
+            for (int i = 0; i < 32; ++i) {
+                double n = 0.0;
+                if (sv != 0.0) {
+                    n = rint(oracle_bf16_to_f64(wg[i]) / sv);      /* ties to even */
+                    if (n > 7.0) n = 7.0;
+                    if (n < -8.0) n = -8.0;
+                }
+                qg[i] = (int8_t)n;
+            }
+        }
+    }
+    return 0;
+}
+
+int oracle_dequantize_int4(const int8_t* q, const uint16_t* scale, int64_t rows, int64_t cols,
+                           uint16_t* w_out) {
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+    const int64_t groups = cols / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            w_out[r * cols + c] = oracle_f64_to_bf16(
+                (double)q[r * cols + c] * oracle_bf16_to_f64(scale[r * groups + c / 32]));
+    return 0;
+}

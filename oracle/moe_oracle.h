@@ -146,6 +146,27 @@ int oracle_dequantize_fp8(const uint8_t* q, const int8_t* sexp, int64_t rows, in
                           uint16_t* w_out);
 
 /*
+ * INT4 storage of the routed experts' weights ("Kimi K2.5 deep dive", CH7.2: the
+ * K2.5 quantization config, 4-bit integer weights, strategy "group" with
+ * group_size 32, symmetric; shared experts on the ignore list stay BF16;
+ * "Kimi K2.5 Q&A", Q7.1: storage quantized, compute BF16).  The config gives
+ * neither the scale rule nor the scale type; the plainest symmetric reading:
+ *   - a group is 32 consecutive K elements of one weight row;
+ *   - s = bf16( amax / 7 ) (amax = largest |w| of the group; the quotient taken
+ *     in fp64, then rounded to nearest-even bf16);
+ *   - q = clamp( nearest integer to w / s, ties to even, -8, 7 ), q = 0 when s = 0;
+ *   - the weight the model computes with is bf16( q * s ) (the exact product
+ *     rounded to nearest-even bf16), then the bf16 layer as usual.
+ * q [rows, cols] int8 in [-8, 7]; scale [rows, cols/32] bf16 bits.
+ * Returns 0, or -1 if cols is not a multiple of 32.
+ */
+int oracle_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, int8_t* q,
+                         uint16_t* scale);
+/* w_out[r, c] = bf16( q[r, c] * scale[r, c / 32] ).  Returns 0 or -1 as above. */
+int oracle_dequantize_int4(const int8_t* q, const uint16_t* scale, int64_t rows, int64_t cols,
+                           uint16_t* w_out);
+
+/*
  * FP8 compute ("Kimi K2.5 Q&A", Q7.1 names V3's "compute in FP8" beside K2.5's
  * quantized storage; "Kimi K2 deep dive", 3.2: FP8 for speed).  The pages give
  * no format.  The one taken for FP8 compute: E4M3 operands with one power-of-two

@@ -528,6 +528,70 @@ def pin_fp8_compute_layer_identities():
     assert np.array_equal(sub, out[[4, 1]])
 
 
+# INT4 storage ("Kimi K2.5 deep dive", CH7.2: 4-bit integer weights, group of
+# 32, symmetric; "Kimi K2.5 Q&A", Q7.1: storage quantized, compute BF16).
+
+def _int4_weights(seed):
+    rng = np.random.default_rng(seed)
+    rows, cols = 6, 256
+    w = rng.normal(0, 1, (rows, cols)) * 2.0 ** rng.integers(-20, 10, (rows, cols // 32)).repeat(32, 1)
+    w[0, :32] = 0.0                                   # all-zero group
+    w[1, 32:64] = rng.normal(0, 1e-3, 32)
+    w[1, 40] = -5.0                                   # the group's maximum is negative
+    w[2, 64:96] = np.arange(32) - 16.0                # integers: exact ties of w / s
+    w[3, 96:128] = rng.normal(0, 1e-39, 32)           # bf16 subnormals: amax / 7 may round to 0
+    return _u16_of(w)
+
+
+def pin_int4_scale_library():
+    """Each group's scale is torch's bf16 rounding of (its amax / 7) in fp32."""
+    wb = _int4_weights(11)
+    wf = oracle.bf16_to_f64(wb)
+    q, sc = oracle.quantize_int4(wb)
+    assert q.shape == wb.shape and sc.shape == (wb.shape[0], wb.shape[1] // 32)
+    amax = np.abs(wf.reshape(wf.shape[0], -1, 32)).max(axis=2)
+    ref = (torch.from_numpy(amax.astype(np.float32)) / 7.0).to(torch.bfloat16)
+    assert np.array_equal(sc, ref.view(torch.int16).numpy().view(np.uint16))
+    assert sc[0, 0] == 0 and np.all(q[0, :32] == 0)
+
+
+def pin_int4_codes_brute_force():
+    """q minimises |w - q s| over the 16 codes, ties to the even code; zero
+    scale gives zero codes."""
+    wb = _int4_weights(12)
+    wf = oracle.bf16_to_f64(wb)
+    q, sc = oracle.quantize_int4(wb)
+    s = oracle.bf16_to_f64(sc)
+    cand = np.arange(-8, 8, dtype=np.float64)
+    for r in range(wf.shape[0]):
+        for c in range(wf.shape[1]):
+            sv = s[r, c // 32]
+            if sv == 0.0:
+                assert q[r, c] == 0
+                continue
+            err = np.abs(wf[r, c] - cand * sv)
+            best = cand[err == err.min()]
+            want = best[0] if len(best) == 1 else best[(best % 2) == 0][0]
+            assert q[r, c] == want, (r, c, wf[r, c], sv, q[r, c], want)
+
+
+def pin_int4_dequantize_library():
+    """Dequantized weights are torch's bf16 rounding of q * s (exact in fp32),
+    within half a step of w, and every nonzero group reaches |q| = 7."""
+    wb = _int4_weights(13)
+    wf = oracle.bf16_to_f64(wb)
+    q, sc = oracle.quantize_int4(wb)
+    deq = oracle.dequantize_int4(q, sc)
+    s = torch.from_numpy(sc.view(np.int16)).view(torch.bfloat16).float()
+    ref = (torch.from_numpy(q.astype(np.float32)) * s.repeat_interleave(32, 1)).to(torch.bfloat16)
+    assert np.array_equal(deq, ref.view(torch.int16).numpy().view(np.uint16))
+    sv = oracle.bf16_to_f64(sc).repeat(32, 1)
+    d = oracle.bf16_to_f64(deq)
+    assert np.all(np.abs(wf - d) <= sv / 2 + np.abs(d) * 2.0 ** -8 + 1e-300)
+    g = np.abs(q.reshape(q.shape[0], -1, 32)).max(axis=2)
+    assert np.all((g == 7) | (oracle.bf16_to_f64(sc) == 0))
+
+
 # ---------------------------------------------------------- load balancing
 # "Kimi K2.5 Q&A", Q7.2 and "Kimi K2.5 deep dive", CH10.2 step 2: the selection
 # bias is a non-learned buffer lowered for over-loaded and raised for
@@ -608,7 +672,8 @@ ALL_PINS = [pin_bf16_rounding, pin_sigmoid_silu, pin_route_worked_example,
             pin_bias_update_worked_example, pin_bias_update_invariants, pin_bias_update_moves_load,
             pin_seq_aux_loss_closed_forms, pin_fp8_rows_quantizer_library,
             pin_fp8_compute_exact_inputs, pin_fp8_compute_exponent_bookkeeping,
-            pin_fp8_compute_layer_identities]
+            pin_fp8_compute_layer_identities, pin_int4_scale_library,
+            pin_int4_codes_brute_force, pin_int4_dequantize_library]
 
 
 def failing_pins():

@@ -88,6 +88,15 @@ MUTANTS = [
      "oracle_swiglu_row_fp8(xt, c->egq[j], c->egs[j], c->edq[j], c->eds[j], d, c->inter, y);"),
     ("fp8c_routed_weight_dropped", "for (int i = 0; i < d; ++i) o[i] += y[i] * w;",
      "for (int i = 0; i < d; ++i) o[i] += y[i];"),
+    ("int4_scale_over_8", "const uint16_t sb = oracle_f64_to_bf16(amax / 7.0);",
+     "const uint16_t sb = oracle_f64_to_bf16(amax / 8.0);"),
+    ("int4_truncates", "n = rint(oracle_bf16_to_f64(wg[i]) / sv);",
+     "n = trunc(oracle_bf16_to_f64(wg[i]) / sv);"),
+    ("int4_signed_max", "const double v = fabs(oracle_bf16_to_f64(wg[i]));",
+     "const double v = oracle_bf16_to_f64(wg[i]);"),
+    ("int4_scale_transposed", "scale[r * groups + g] = sb;", "scale[g * rows + r] = sb;"),
+    ("int4_dequant_wrong_group", "oracle_bf16_to_f64(scale[r * groups + c / 32])",
+     "oracle_bf16_to_f64(scale[r * groups + c / 64])"),
     ("fp8_rows_signed_max", "if (fabs(v[i]) > amax) amax = fabs(v[i]);",
      "if (v[i] > amax) amax = v[i];"),
 ]
