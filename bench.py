@@ -53,9 +53,10 @@ def parse_args(argv=None):
                    help="time the load-balancing pass instead of the layer: router scores, "
                         "route, permute, the sequence-level loss over sequences of S tokens "
                         "and the bias update")
-    p.add_argument("--weights", choices=["bf16", "fp8", "w8a8"], default="bf16",
+    p.add_argument("--weights", choices=["bf16", "fp8", "w8a8", "w4a16"], default="bf16",
                    help="expert weights: bf16; fp8 = routed experts stored as E4M3 codes with "
-                        "one power-of-two scale per 128x128 block, bf16 compute; w8a8 = FP8 "
+                        "one power-of-two scale per 128x128 block, bf16 compute; w4a16 = routed "
+                        "experts as INT4 with a bf16 scale per group of 32, bf16 compute; w8a8 = FP8 "
                         "compute in every expert, E4M3 weights and activations with one "
                         "power-of-two scale per row (weights quantized once, untimed)")
     p.add_argument("--cpu-sample", type=int, default=None,
@@ -225,6 +226,9 @@ def layer_accounting(cfg, touched: int, weights: str = "bf16"):
     if weights == "fp8":
         r_gu = 2 * I * d + (2 * I // 128) * (d // 128)
         r_dn = d * I + (d // 128) * (I // 128)
+    elif weights == "w4a16":
+        r_gu = I * d + (2 * I) * (d // 32) * 2
+        r_dn = d * I // 2 + d * (I // 32) * 2
     elif weights == "w8a8":
         r_gu, r_dn = 2 * I * d + 2 * I, d * I + d
         w_gu, w_dn = r_gu, r_dn
@@ -275,6 +279,9 @@ class OracleSample:
                 # the weights FP8 storage stands for, from the oracle's own quantizer
                 self.egu[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.egu[e]))
                 self.edn[e] = oracle.dequantize_fp8(*oracle.quantize_fp8(self.edn[e]))
+            elif weights == "w4a16":
+                self.egu[e] = oracle.dequantize_int4(*oracle.quantize_int4(self.egu[e]))
+                self.edn[e] = oracle.dequantize_int4(*oracle.quantize_int4(self.edn[e]))
         self.sgu, self.sdn = inputs_dev["ws_gate_up"].cpu(), inputs_dev["ws_down"].cpu()
         if weights == "w8a8":
             # FP8-compute weights from the oracle's own row quantizer
@@ -298,6 +305,7 @@ class OracleSample:
 
     def describe(self) -> str:
         fp8 = {"fp8": " (routed weights: the oracle's FP8 quantization, dequantized)",
+               "w4a16": " (routed weights: the oracle's INT4 quantization, dequantized)",
                "w8a8": " (FP8 compute: the oracle's per-row E4M3 quantization of weights "
                        "and activations)"}.get(self.weights, "")
         return (f"{len(self.tokens)} of {self.cfg.T} tokens (evenly spaced), full routing + "
@@ -309,7 +317,7 @@ def default_cpu_sample(cfg, weights: str = "bf16"):
     # 16-core host busy for several seconds without copying every expert.
     # With FP8 weights the oracle first quantizes every expert the sample
     # selects (about a second each), so the sample is smaller.
-    if weights in ("fp8", "w8a8"):
+    if weights in ("fp8", "w8a8", "w4a16"):
         return min(cfg.T, 8)
     return min(cfg.T, max(64, 4 * host_cores()))
 
@@ -361,6 +369,11 @@ def main(argv=None):
 
     fp8 = args.weights == "fp8"
     w8a8 = args.weights == "w8a8"
+    w4 = args.weights == "w4a16"
+    if w4:
+        qgu, sgu = moe.moe_quantize_int4(g["w_gate_up"])
+        qdn, sdn = moe.moe_quantize_int4(g["w_down"])
+        torch.cuda.synchronize(dev)
     if fp8:
         # storage format conversion, once, outside every timed region
         qgu, egu = moe.moe_quantize_fp8(g["w_gate_up"])
@@ -373,7 +386,10 @@ def main(argv=None):
         torch.cuda.synchronize(dev)
 
     def layer(x_in):
-        if w8a8:
+        if w4:
+            moe.moe_layer_forward_w4a16(x_in, g["w_router"], g["bias"], qgu, sgu, qdn, sdn,
+                                        g["ws_gate_up"], g["ws_down"], k, cfg.scale, out)
+        elif w8a8:
             moe.moe_layer_forward_w8a8(x_in, g["w_router"], g["bias"], *wq, k, cfg.scale, out)
         elif fp8:
             moe.moe_layer_forward_fp8(x_in, g["w_router"], g["bias"], qgu, egu, qdn, edn,
@@ -492,7 +508,8 @@ def main(argv=None):
                       "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
                       "touched_experts": touched}
     roof["traffic"] = profiled_traffic(
-        args.workload + {"fp8": "_fp8", "w8a8": "_w8a8"}.get(args.weights, ""), kname)
+        args.workload + {"fp8": "_fp8", "w8a8": "_w8a8", "w4a16": "_w4a16"}.get(args.weights, ""),
+        kname)
 
     # ---------------------------------------------------------- CPU baseline
     cpu = None
@@ -513,6 +530,7 @@ def main(argv=None):
                        "T": T, "d": d, "E": E, "k": k, "inter": I,
                        "scale": cfg.scale, "bias": cfg.bias, "parallelism": f"replicas{world}",
                        "weights": {"fp8": "fp8_e4m3_block128_pow2",
+                                   "w4a16": "int4_group32_sym_bf16_scale",
                                    "w8a8": "w8a8_e4m3_row_pow2"}.get(args.weights, "bf16"),
                        "l2": "inputs larger than L2: every step streams "
                              f"{acc['weight_bytes'] / 1e9:.1f} GB of expert weights"},

@@ -248,6 +248,49 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * INT4 storage of the routed experts' weights ("Kimi K2.5 deep dive", CH7.2:
+ * the K2.5 quantization config, 4-bit symmetric integers in groups of 32 along
+ * K, shared experts exempt; "Kimi K2.5 Q&A", Q7.1: storage quantized, compute
+ * BF16).  The config gives no scale rule or type; this library's (per group
+ * of 32 consecutive elements of a row):
+ *     s = bf16(amax / 7), nearest-even;
+ *     q = clamp(nearest integer to w / s, ties to even, -8, 7), 0 when s = 0;
+ * and the layer computes with the bf16 weights bf16(q * s) (nearest-even),
+ * bf16 tensor-core math as in moe_layer_forward.
+ *
+ * moe_quantize_int4: w [rows, cols] bf16 row-major (cols a multiple of 64) ->
+ *   codes  [rows, cols/2] bytes: in each 32-bit little-endian word j of a row,
+ *          element 8j+2i sits in bits 4i..4i+3 and element 8j+2i+1 in bits
+ *          16+4i..16+4i+3, each stored as q + 8;
+ *   scales [cols/32, rows] bf16, group-major (one row of scales per group).
+ * Caller-owned device memory, asynchronous on `stream`.  Stacked experts
+ * quantize in one call: [E, 2*inter, d] as rows = E*2*inter (scales
+ * [d/32, E*2*inter]); [E, d, inter] as rows = E*d (scales [inter/32, E*d]).
+ * MOE_ERR_UNSUPPORTED_SHAPE for other shapes, MOE_ERR_INVALID_ARG for null or
+ * unaligned (16-byte) pointers.
+ *
+ * moe_layer_forward_w4a16: the layer of moe_layer_forward with the routed
+ * experts' weights as (codes, scales) from moe_quantize_int4; router, shared
+ * expert, activations and output bf16 as there.  The codes are dequantized in
+ * shared memory just before the tensor cores read them.  Errors as in
+ * moe_layer_forward; the _ws form takes moe_workspace_size(T, d, E, k, inter)
+ * bytes.
+ */
+int moe_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* codes,
+                      uint16_t* scales, void* stream);
+int moe_layer_forward_w4a16(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                            const uint8_t* wq_gate_up, const uint16_t* wq_gate_up_scale,
+                            const uint8_t* wq_down, const uint16_t* wq_down_scale,
+                            const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                            int E, int k, int inter, float scale, uint16_t* out, void* stream);
+int moe_layer_forward_w4a16_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                               const uint8_t* wq_gate_up, const uint16_t* wq_gate_up_scale,
+                               const uint8_t* wq_down, const uint16_t* wq_down_scale,
+                               const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                               int E, int k, int inter, float scale, uint16_t* out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * FP8 compute ("Kimi K2.5 Q&A", Q7.1 names DeepSeek-V3's "compute in FP8" next
  * to K2.5's quantized storage; "Kimi K2 deep dive", 3.2: FP8 for speed).  The
  * pages give no format; this library's: E4M3 codes (as above) with one

@@ -23,7 +23,8 @@ __all__ = [
     "moe_layer_forward_noalloc", "moe_quantize_fp8", "moe_layer_forward_fp8",
     "moe_layer_forward_fp8_ws", "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
     "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
-    "moe_layer_forward_w8a8_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "moe_layer_forward_w8a8_ws", "moe_quantize_int4", "moe_layer_forward_w4a16",
+    "moe_layer_forward_w4a16_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
@@ -35,7 +36,8 @@ EXPORTED_SYMBOLS = [
     "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
     "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss", "moe_seq_aux_workspace_size",
     "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
-    "moe_layer_forward_w8a8_ws",
+    "moe_layer_forward_w8a8_ws", "moe_quantize_int4", "moe_layer_forward_w4a16",
+    "moe_layer_forward_w4a16_ws",
 ]
 
 MOE_OK = 0
@@ -79,6 +81,9 @@ def _load():
         "moe_seq_aux_loss": ([P, P, I, I, I, I, F, P, P, P, P, SZ, P], I),
         "moe_seq_aux_workspace_size": ([I, I, I], SZ),
         "moe_quantize_fp8_rows": ([P, I64, I64, P, P, P], I),
+        "moe_quantize_int4": ([P, I64, I64, P, P, P], I),
+        "moe_layer_forward_w4a16": ([P] * 9 + [I, I, I, I, I, F, P, P], I),
+        "moe_layer_forward_w4a16_ws": ([P] * 9 + [I, I, I, I, I, F, P, P, SZ, P], I),
         "moe_workspace_size_w8a8": ([I, I, I, I, I], SZ),
         "moe_layer_forward_w8a8": ([P] * 11 + [I, I, I, I, I, F, P, P], I),
         "moe_layer_forward_w8a8_ws": ([P] * 11 + [I, I, I, I, I, F, P, P, SZ, P], I),
@@ -269,6 +274,59 @@ def moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_d
                                        _ptr(workspace, torch.uint8, "workspace"),
                                        workspace.numel(), _stream(stream))
     _check("moe_layer_forward_fp8_ws", rc)
+
+
+def moe_quantize_int4(w, stream=None):
+    """bf16 weights [..., rows, cols] (cols a multiple of 64) -> (packed INT4
+    codes uint8 [..., rows, cols/2], group scales bf16 [cols/32, prod(...) *
+    rows], group-major), new tensors on w's device."""
+    if w.dim() < 2:
+        raise ValueError("w must have at least 2 dimensions")
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    codes = torch.empty(tuple(w.shape[:-1]) + (cols // 2,), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((cols // 32, rows), dtype=BF16, device=w.device)
+    rc = _LIB.moe_quantize_int4(_ptr(w, BF16, "w"), rows, cols, _ptr(codes, torch.uint8, "codes"),
+                                _ptr(scales, BF16, "scales"), _stream(stream))
+    _check("moe_quantize_int4", rc)
+    return codes, scales
+
+
+def _layer_w4_args(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down, wq_down_scale,
+                   ws_gate_up, ws_down):
+    T, d = x.shape
+    E = w_router.shape[0]
+    inter = wq_gate_up.shape[1] // 2
+    return ([_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"), _ptr(bias, F32, "bias"),
+             _ptr(wq_gate_up, torch.uint8, "wq_gate_up"),
+             _ptr(wq_gate_up_scale, BF16, "wq_gate_up_scale"),
+             _ptr(wq_down, torch.uint8, "wq_down"), _ptr(wq_down_scale, BF16, "wq_down_scale"),
+             _ptr(ws_gate_up, BF16, "ws_gate_up"), _ptr(ws_down, BF16, "ws_down")],
+            T, d, E, inter)
+
+
+def moe_layer_forward_w4a16(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down,
+                            wq_down_scale, ws_gate_up, ws_down, k: int, scale: float, out,
+                            stream=None):
+    """moe_layer_forward with the routed experts' weights as INT4 codes + group
+    scales (from moe_quantize_int4); router and shared expert stay bf16."""
+    ptrs, T, d, E, inter = _layer_w4_args(x, w_router, bias, wq_gate_up, wq_gate_up_scale,
+                                          wq_down, wq_down_scale, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_w4a16(*ptrs, T, d, E, k, inter, float(scale),
+                                      _ptr(out, BF16, "out"), _stream(stream))
+    _check("moe_layer_forward_w4a16", rc)
+
+
+def moe_layer_forward_w4a16_ws(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down,
+                               wq_down_scale, ws_gate_up, ws_down, k: int, scale: float, out,
+                               workspace, stream=None):
+    ptrs, T, d, E, inter = _layer_w4_args(x, w_router, bias, wq_gate_up, wq_gate_up_scale,
+                                          wq_down, wq_down_scale, ws_gate_up, ws_down)
+    rc = _LIB.moe_layer_forward_w4a16_ws(*ptrs, T, d, E, k, inter, float(scale),
+                                         _ptr(out, BF16, "out"),
+                                         _ptr(workspace, torch.uint8, "workspace"),
+                                         workspace.numel(), _stream(stream))
+    _check("moe_layer_forward_w4a16_ws", rc)
 
 
 def moe_quantize_fp8_rows(w, stream=None):

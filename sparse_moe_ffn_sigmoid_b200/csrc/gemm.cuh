@@ -66,6 +66,10 @@ constexpr int kConvWarps = 8;
 constexpr int kConvThreads = 32 * kConvWarps;
 constexpr int kGemmThreadsFP8 = 480;
 constexpr int kSlabBytes8 = kSlabRows * kBK;  // one FP8 slab per K step (128 rows x 64 codes)
+// INT4 slab per K step: 128 rows x 64 codes packed in 32 bytes, then the step's two
+// group scales of the 128 rows (bf16, group-major)
+constexpr int kSlabCodes4 = kSlabRows * kBK / 2;
+constexpr int kSlabBytes4 = kSlabCodes4 + kSlabRows * 2 * 2;
 constexpr int kTmemCols = 512;
 
 // Operand formats of a launch.
@@ -73,7 +77,17 @@ enum GemmOperands : int {
     kOpsBF16 = 0,       // bf16 weights and tokens (kind::f16)
     kOpsW8Convert = 1,  // routed weights as block-scaled E4M3, dequantized in shared memory
     kOpsFP8 = 2,        // E4M3 weights and tokens with per-row exponents (kind::f8f6f4)
+    kOpsW4Convert = 3,  // routed weights as INT4 with group-32 scales, dequantized in shared memory
 };
+
+// Modes whose routed weights are converted to bf16 in shared memory, and the
+// bytes one weight slab of a K step takes in their code ring.
+__host__ __device__ constexpr bool ops_convert(int ops) {
+    return ops == kOpsW8Convert || ops == kOpsW4Convert;
+}
+__host__ __device__ constexpr int code_slab_bytes(int ops) {
+    return ops == kOpsW4Convert ? kSlabBytes4 : kSlabBytes8;
+}
 
 enum GemmEpilogue : int {
     kEpiSwiGLU = 0,   // 2 slabs (gate, up) -> bf16 silu(gate) * up
@@ -110,7 +124,10 @@ struct __align__(64) GemmArgs {
     // FP8-weight mode only: routed tiles (map 0) read E4M3 codes through a8_map
     // ([rows, K] uint8, 64 x 128 boxes) and one int8 exponent per 128 x 128 block
     // (a8_scale[(row / 128) * a8_kblocks + k / 128]); shared tiles (map 1) stay bf16
+    // INT4-weight mode: a8_map reads the packed codes ([rows, K/2] bytes, 32 x 128
+    // boxes) and a4s_map the group scales ([K/32, rows] bf16, 128 x 2 boxes)
     CUtensorMap a8_map;
+    CUtensorMap a4s_map;
     const int8_t* a8_scale;
     int a8_kblocks;
     int stages_a8;            // FP8 code ring depth
@@ -221,13 +238,17 @@ __device__ __forceinline__ bool wait_lane0(uint64_t* bar, uint32_t parity, volat
 // weights into the slot with TMA (arrive.expect_tx on full).  The weight
 // producer, which runs up to SA8 routed steps ahead, never touches the bf16
 // ring in this mode.
-template <int nslab>
+// OPS = kOpsW8Convert: E4M3 codes (64 bytes per slab row) and one block exponent
+// per slab and step; kOpsW4Convert: packed INT4 codes (32 bytes per slab row,
+// one 32-bit word per unit) and the step's two group scales per row in the slot.
+template <int nslab, int OPS>
 __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint8_t* ring8,
                                                 uint8_t* ring_a, int SA, int SA8, uint64_t* full,
                                                 uint64_t* empty, uint64_t* full8,
                                                 uint64_t* empty8, volatile int* abort_flag,
                                                 uint64_t tmo, int ntiles, int ct) {
-    constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
+    constexpr bool kInt4 = (OPS == kOpsW4Convert);
+    constexpr uint32_t a8_bytes = nslab * code_slab_bytes(OPS);
     constexpr uint32_t a_bytes = nslab * kSlabBytes;
     constexpr int kUnits = nslab * kSlabRows * (kBK / 8) / kConvThreads;   // per thread
     const int lane = ct & 31;
@@ -239,12 +260,40 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
     for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
         const Tile t = load_tile(args, i);
         const bool routed = (t.map == 0);
-        const int8_t* sc0 = args.a8_scale + (t.a_row0 / kQuantBlock) * args.a8_kblocks;
-        const int8_t* sc1 = args.a8_scale + (t.a_row1 / kQuantBlock) * args.a8_kblocks;
+        const int8_t* sc0 =
+            kInt4 ? nullptr : args.a8_scale + (t.a_row0 / kQuantBlock) * args.a8_kblocks;
+        const int8_t* sc1 =
+            kInt4 ? nullptr : args.a8_scale + (t.a_row1 / kQuantBlock) * args.a8_kblocks;
         for (int ks = t.ks0; ks < t.ks1; ++ks) {
             bool w_ok = (!routed || wait_lane0(&full8[r8.stage], r8.phase, abort_flag, tmo, lane)) &&
                         wait_lane0(&empty[rq.stage], rq.phase ^ 1, abort_flag, tmo, lane);
-            if (routed && w_ok) {
+            if (kInt4 && routed && w_ok) {
+                const uint8_t* src = ring8 + r8.stage * a8_bytes;
+                uint8_t* dst = ring_a + rq.stage * a_bytes;
+                // unit u: slab u / 1024, row (u / 8) % 128, 8-code chunk u % 8 (group chunk / 4)
+                uint32_t words[kUnits];
+#pragma unroll
+                for (int j = 0; j < kUnits; ++j) {
+                    const int u = ct + kConvThreads * j;
+                    const int slab = u / (kSlabRows * 8);
+                    const int r = (u >> 3) & (kSlabRows - 1);
+                    words[j] = *reinterpret_cast<const uint32_t*>(src + slab * kSlabBytes4 +
+                                                                  r * (kBK / 2) + (u & 7) * 4);
+                }
+#pragma unroll
+                for (int j = 0; j < kUnits; ++j) {
+                    const int u = ct + kConvThreads * j;
+                    const int slab = u / (kSlabRows * 8);
+                    const int r = (u >> 3) & (kSlabRows - 1);
+                    const int c = u & 7;
+                    const bf16 sc = *reinterpret_cast<const bf16*>(
+                        src + slab * kSlabBytes4 + kSlabCodes4 + (c >> 2) * (kSlabRows * 2) + r * 2);
+                    *reinterpret_cast<uint4*>(dst + slab * kSlabBytes + r * (kBK * 2) +
+                                              ((c ^ (r & 7)) << 4)) =
+                        int4x8_to_bf16x8(words[j], __bfloat162bfloat162(sc));
+                }
+                ptx::fence_proxy_async_smem();
+            } else if (routed && w_ok) {
                 const Fp8Scale s0 = fp8_scale(__ldg(sc0 + ks * kBK / kQuantBlock));
                 const Fp8Scale s1 = nslab == 2 ? fp8_scale(__ldg(sc1 + ks * kBK / kQuantBlock)) : s0;
                 const uint8_t* src = ring8 + r8.stage * a8_bytes;
@@ -302,14 +351,15 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
     }
 }
 
-// OPS (GemmOperands): kOpsW8Convert has routed weights arrive as E4M3 codes
-// that the converter warps dequantize in shared memory (kGemmThreadsFP8
-// threads); kOpsBF16 is the all-bf16 kernel and kOpsFP8 the FP8-compute one
-// (kGemmThreads threads).
+// OPS (GemmOperands): kOpsW8Convert / kOpsW4Convert have routed weights arrive
+// as E4M3 / INT4 codes that the converter warps dequantize in shared memory
+// (kGemmThreadsFP8 threads); kOpsBF16 is the all-bf16 kernel and kOpsFP8 the
+// FP8-compute one (kGemmThreads threads).
 template <int EPI, int OPS>
-__global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemmThreads, 1)
+__global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ GemmArgs args) {
-    constexpr bool FP8A = (OPS == kOpsW8Convert);
+    constexpr bool FP8A = ops_convert(OPS);     // a converting mode (E4M3 or INT4 codes)
+    constexpr bool kInt4 = (OPS == kOpsW4Convert);
     constexpr bool F8C = (OPS == kOpsFP8);
     constexpr int kStepK = F8C ? 2 * kBK : kBK;   // K elements per step (128-byte rows)
     extern __shared__ uint8_t smem_raw[];
@@ -325,10 +375,10 @@ __global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemm
     const uint32_t b_bytes = args.n_max * kBK * 2;
     static_assert((!FP8A && !F8C) || nslab == 2, "FP8 weights are for the expert GEMMs");
     const int SA8 = FP8A ? args.stages_a8 : 0;
-    constexpr uint32_t a8_bytes = nslab * kSlabBytes8;
+    constexpr uint32_t a8_bytes = nslab * code_slab_bytes(OPS);
     uint8_t* ring_a = smem;                                  // [SA][nslab][128 x 64] bf16
     uint8_t* ring_b = ring_a + SA * a_bytes;                 // [SB][n_max x 64] bf16
-    uint8_t* ring8 = ring_b + SB * b_bytes;                  // [SA8][nslab][128 x 64] E4M3
+    uint8_t* ring8 = ring_b + SB * b_bytes;                  // [SA8][nslab][code slab]
     bf16* staging = reinterpret_cast<bf16*>(ring8 + SA8 * a8_bytes);
     uint64_t* full = reinterpret_cast<uint64_t*>(ring8 + SA8 * a8_bytes + kStagingBytes);
     uint64_t* empty = full + SA;
@@ -368,6 +418,7 @@ __global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemm
         ptx::prefetch_tensormap(&args.b_map64[0]);
         ptx::prefetch_tensormap(&args.b_map64[1]);
         if (FP8A) ptx::prefetch_tensormap(&args.a8_map);
+        if (kInt4) ptx::prefetch_tensormap(&args.a4s_map);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_holder, kTmemCols);
@@ -419,9 +470,21 @@ __global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemm
                         uint64_t* bar8 = &full8[r8.stage];
                         ptx::mbar_arrive_expect_tx(bar8, a8_bytes);
                         uint8_t* s8 = ring8 + r8.stage * a8_bytes;
-                        ptx::tma_load_2d_hint(s8, &args.a8_map, bar8, ks * kBK, t.a_row0, pol);
-                        ptx::tma_load_2d_hint(s8 + kSlabBytes8, &args.a8_map, bar8, ks * kBK,
-                                              t.a_row1, pol);
+                        if constexpr (kInt4) {
+                            // per slab: 128 rows x 32 code bytes, then 2 groups x 128 scales
+                            ptx::tma_load_2d_hint(s8, &args.a8_map, bar8, ks * (kBK / 2), t.a_row0,
+                                                  pol);
+                            ptx::tma_load_2d_hint(s8 + kSlabCodes4, &args.a4s_map, bar8, t.a_row0,
+                                                  ks * (kBK / kInt4Group), pol);
+                            ptx::tma_load_2d_hint(s8 + kSlabBytes4, &args.a8_map, bar8,
+                                                  ks * (kBK / 2), t.a_row1, pol);
+                            ptx::tma_load_2d_hint(s8 + kSlabBytes4 + kSlabCodes4, &args.a4s_map,
+                                                  bar8, t.a_row1, ks * (kBK / kInt4Group), pol);
+                        } else {
+                            ptx::tma_load_2d_hint(s8, &args.a8_map, bar8, ks * kBK, t.a_row0, pol);
+                            ptx::tma_load_2d_hint(s8 + kSlabBytes8, &args.a8_map, bar8, ks * kBK,
+                                                  t.a_row1, pol);
+                        }
                         issued8 |= 1u << r8.stage;
                         issued8_parity = (issued8_parity & ~(1u << r8.stage)) | (r8.phase << r8.stage);
                         r8.next();
@@ -556,7 +619,7 @@ __global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemm
         }
     } else if (FP8A && warp >= 2 + kEpiWarpsFP8) {
         // ---------------------------------------------------------- converters
-        convert_weights<nslab>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
+        convert_weights<nslab, OPS>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
                                abort_flag, tmo, ntiles,
                                32 * (warp < kTokenWarp ? warp - 6 : warp - 7) + lane);
     } else {
@@ -679,11 +742,13 @@ __global__ void __launch_bounds__(OPS == kOpsW8Convert ? kGemmThreadsFP8 : kGemm
     }
 }
 
-// Dynamic shared memory the kernel needs for a configuration.
-inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max, int stages_a8 = 0) {
+// Dynamic shared memory the kernel needs for a configuration (code_slab: the
+// bytes of one weight slab per K step in the code ring of a converting mode).
+inline size_t gemm_smem_bytes(int stages_a, int stages_b, int nslab, int n_max, int stages_a8 = 0,
+                              int code_slab = kSlabBytes8) {
     const size_t a = static_cast<size_t>(nslab) * kSlabBytes;
     const size_t b = static_cast<size_t>(n_max) * kBK * 2;
-    const size_t a8 = static_cast<size_t>(nslab) * kSlabBytes8;
+    const size_t a8 = static_cast<size_t>(nslab) * code_slab;
     return 1024 /* alignment slack */ + stages_a * a + stages_b * b + stages_a8 * a8 +
            kStagingBytes + (2 * stages_a + 2 * stages_a8 + 5) * 8 + 16;
 }

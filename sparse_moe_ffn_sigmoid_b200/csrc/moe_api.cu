@@ -199,6 +199,10 @@ int device_info(DeviceInfo* out) {
                 cudaSuccess ||
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsW8Convert>, dyn, smem) !=
                 cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsW4Convert>, dyn, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsW4Convert>, dyn, smem) !=
+                cudaSuccess ||
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsFP8>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsFP8>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(scan_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -244,6 +248,32 @@ bool make_map8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed INT4 codes [rows, cols / 2] (bytes) read in boxes of 128 rows x 32
+// bytes (one K step), and their group scales [cols / 32, rows] (bf16, group-
+// major) in boxes of 2 groups x 128 rows; both unswizzled (the converter warps
+// read them).
+bool make_map_int4(CUtensorMap* codes_map, CUtensorMap* scale_map, const void* codes,
+                   const void* scales, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t cdims[2] = {cols / 2, rows};
+    const cuuint64_t cstrides[1] = {cols / 2};
+    const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(kBK / 2), static_cast<cuuint32_t>(kSlabRows)};
+    const cuuint64_t sdims[2] = {rows, cols / kInt4Group};
+    const cuuint64_t sstrides[1] = {rows * sizeof(bf16)};
+    const cuuint32_t sbox[2] = {static_cast<cuuint32_t>(kSlabRows),
+                                static_cast<cuuint32_t>(kBK / kInt4Group)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(codes_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), cdims,
+               cstrides, cbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+               CUDA_SUCCESS &&
+           enc(scale_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(scales), sdims,
+               sstrides, sbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+               CUDA_SUCCESS;
 }
 
 // Row-major E4M3 code matrix [rows, cols] (uint8) read in boxes of box_rows x
@@ -297,13 +327,13 @@ void fill_pipeline(GemmArgs& a, int nslab, int n_max) {
     a.timeout_ns = g_timeout_ns.load();
 }
 
-// FP8-weight expert GEMMs: a shallow bf16 ring between the converter warps
-// and the MMAs, a deep code ring for the weight stream (half the bytes per
-// slot), the token ring as in the bf16 kernel.
-void fill_pipeline_fp8(GemmArgs& a, int n_max) {
+// Converting expert GEMMs (FP8 or INT4 weights): a shallow bf16 ring between
+// the converter warps and the MMAs, a deep code ring for the weight stream
+// (code_slab bytes per slab and step), the token ring as in the bf16 kernel.
+void fill_pipeline_fp8(GemmArgs& a, int n_max, int code_slab = kSlabBytes8) {
     fill_pipeline(a, 2, n_max);
     const size_t a_bytes = 2 * static_cast<size_t>(kSlabBytes);
-    const size_t a8_bytes = 2 * static_cast<size_t>(kSlabBytes8);
+    const size_t a8_bytes = 2 * static_cast<size_t>(code_slab);
     const size_t b_bytes = static_cast<size_t>(n_max) * kBK * 2;
     const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 1024;
     a.stages_b = (n_max <= 64 || n_max > 128) ? 2 : 3;
@@ -314,9 +344,9 @@ void fill_pipeline_fp8(GemmArgs& a, int n_max) {
 
 template <int EPI, int OPS = kOpsBF16>
 int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
-    constexpr bool FP8A = (OPS == kOpsW8Convert);
-    const size_t smem =
-        gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max, FP8A ? a.stages_a8 : 0);
+    constexpr bool FP8A = ops_convert(OPS);
+    const size_t smem = gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max,
+                                        FP8A ? a.stages_a8 : 0, code_slab_bytes(OPS));
     if (smem > kMaxDynSmem || (FP8A && a.stages_a8 < 2)) return MOE_ERR_UNSUPPORTED_SHAPE;
     moe_gemm_kernel<EPI, OPS><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -410,16 +440,26 @@ struct Fp8Experts {
     const int8_t* down_exp;
 };
 
+// Routed experts' weights as INT4 (quant.cuh): gate|up codes [E, 2I, d/2] bytes +
+// scales [d/32, E*2I] bf16; down codes [E, d, I/2] + scales [I/32, E*d].
+struct Int4Experts {
+    const uint8_t* gate_up;
+    const bf16* gate_up_scale;
+    const uint8_t* down;
+    const bf16* down_scale;
+};
+
 // gather + gate|up + down over a planned tile list.
 //   rows_b0: rows of the permuted token matrix (T*k); h_rows / y rows: rows_b0 (+ T if shared)
-//   f8: routed weights in FP8 (then w_gate_up / w_down are unused), or null for bf16
+//   f8 / i4: routed weights in FP8 or INT4 (then w_gate_up / w_down are unused),
+//   or both null for bf16
 int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T, int d, int E,
                int k, int inter, const bf16* w_gate_up, const bf16* w_down,
                const bf16* ws_gate_up, const bf16* ws_down, bool shared, bf16* xperm, bf16* h,
                bf16* y, const int4* tiles1, const int4* tiles2, const int* ntiles,
                int max_tiles1, int max_tiles2, cudaStream_t st, Recorder& rec,
-               const Fp8Experts* f8 = nullptr) {
-    if (f8 != nullptr && !shared) return MOE_ERR_INVALID_ARG;
+               const Fp8Experts* f8 = nullptr, const Int4Experts* i4 = nullptr) {
+    if ((f8 != nullptr || i4 != nullptr) && !shared) return MOE_ERR_INVALID_ARG;
     const int rows_routed = T * k;
     const int rows_all = rows_routed + (shared ? T : 0);
     if (rows_routed > 0) {
@@ -434,7 +474,13 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     GemmArgs g1;
     std::memset(&g1, 0, sizeof(g1));
     const bf16* xp = rows_routed > 0 ? xperm : x;
-    if (f8 != nullptr) {
+    if (i4 != nullptr) {
+        // routed tiles read codes and scales; slot 0 of the bf16 maps is never used
+        if (!make_map_int4(&g1.a8_map, &g1.a4s_map, i4->gate_up, i4->gate_up_scale,
+                           static_cast<uint64_t>(E) * 2 * inter, d) ||
+            !make_map(&g1.a_map[0], ws_gate_up, 2ull * inter, d, kSlabRows))
+            return MOE_ERR_CUDA;
+    } else if (f8 != nullptr) {
         // routed tiles read codes; slot 0 of the bf16 maps is never used
         if (!make_map8(&g1.a8_map, f8->gate_up, static_cast<uint64_t>(E) * 2 * inter, d) ||
             !make_map(&g1.a_map[0], ws_gate_up, 2ull * inter, d, kSlabRows))
@@ -461,7 +507,10 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     g1.out_ld = inter;
     g1.col_limit = inter;
     int rc;
-    if (f8 != nullptr) {
+    if (i4 != nullptr) {
+        fill_pipeline_fp8(g1, n_max, kSlabBytes4);
+        rc = launch_gemm<kEpiSwiGLU, kOpsW4Convert>(g1, std::min(max_tiles1, di.sms), st);
+    } else if (f8 != nullptr) {
         fill_pipeline_fp8(g1, n_max);
         rc = launch_gemm<kEpiSwiGLU, kOpsW8Convert>(g1, std::min(max_tiles1, di.sms), st);
     } else {
@@ -474,7 +523,12 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
 
     GemmArgs g2;
     std::memset(&g2, 0, sizeof(g2));
-    if (f8 != nullptr) {
+    if (i4 != nullptr) {
+        if (!make_map_int4(&g2.a8_map, &g2.a4s_map, i4->down, i4->down_scale,
+                           static_cast<uint64_t>(E) * d, inter) ||
+            !make_map(&g2.a_map[0], ws_down, d, inter, kSlabRows))
+            return MOE_ERR_CUDA;
+    } else if (f8 != nullptr) {
         if (!make_map8(&g2.a8_map, f8->down, static_cast<uint64_t>(E) * d, inter) ||
             !make_map(&g2.a_map[0], ws_down, d, inter, kSlabRows))
             return MOE_ERR_CUDA;
@@ -498,7 +552,10 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, int T,
     g2.out = y;
     g2.out_ld = d;
     g2.col_limit = d;
-    if (f8 != nullptr) {
+    if (i4 != nullptr) {
+        fill_pipeline_fp8(g2, n_max, kSlabBytes4);
+        rc = launch_gemm<kEpiStoreBF16, kOpsW4Convert>(g2, std::min(max_tiles2, di.sms), st);
+    } else if (f8 != nullptr) {
         fill_pipeline_fp8(g2, n_max);
         rc = launch_gemm<kEpiStoreBF16, kOpsW8Convert>(g2, std::min(max_tiles2, di.sms), st);
     } else {
@@ -622,7 +679,8 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
 int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* wgu,
                   const bf16* wdn, const bf16* sgu, const bf16* sdn, int T, int d, int E, int k,
                   int inter, float scale, bf16* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                  const Fp8Experts* f8 = nullptr, const Fp8Rows* f8c = nullptr) {
+                  const Fp8Experts* f8 = nullptr, const Fp8Rows* f8c = nullptr,
+                  const Int4Experts* i4 = nullptr) {
     const Layout L = make_layout(T, d, E, k, inter, f8c != nullptr);
     if (ws == nullptr || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
     DeviceInfo di;
@@ -666,7 +724,7 @@ int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* 
                             ntiles, L.max_tiles1, L.max_tiles2, st, rec);
     else
         rc = launch_ffn(di, x, row_token, T, d, E, k, inter, wgu, wdn, sgu, sdn, true, xperm, h,
-                        y, tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8);
+                        y, tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8, i4);
     if (rc != MOE_OK) return rc;
     rc = launch_combine(y, y + static_cast<size_t>(T) * k * d, w, slot_row, T, d, k, out, st, rec);
     g_last_launches.store(rec.launches);
@@ -956,6 +1014,64 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
     return moe_layer_forward_fp8_ws(x, w_router, bias, wq_gate_up, wq_gate_up_exp, wq_down,
                                     wq_down_exp, ws_gate_up, ws_down, T, d, E, k, inter, scale,
                                     out, ws, need, stream);
+}
+
+int moe_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* codes,
+                      uint16_t* scales, void* stream) {
+    if (rows < 0 || cols < 0 || cols % kBK != 0 || cols > 0x7FFFFFFF ||
+        rows * (cols / kInt4Group) > 0x7FFFFFFFll * kInt4Warps)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!all_ok(w, codes, scales)) return MOE_ERR_INVALID_ARG;
+    const long long groups = rows * (cols / kInt4Group);
+    const unsigned blocks = static_cast<unsigned>((groups + kInt4Warps - 1) / kInt4Warps);
+    int4_quantize_kernel<<<blocks, 32 * kInt4Warps, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const bf16*>(w), rows, static_cast<int>(cols),
+        reinterpret_cast<uint32_t*>(codes), reinterpret_cast<bf16*>(scales));
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_layer_forward_w4a16_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                               const uint8_t* wq_gate_up, const uint16_t* wq_gate_up_scale,
+                               const uint8_t* wq_down, const uint16_t* wq_down_scale,
+                               const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                               int E, int k, int inter, float scale, uint16_t* out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down, wq_down_scale,
+                ws_gate_up, ws_down, out, workspace))
+        return MOE_ERR_INVALID_ARG;
+    if (!(scale == scale)) return MOE_ERR_INVALID_ARG;
+    const Int4Experts i4{wq_gate_up, reinterpret_cast<const bf16*>(wq_gate_up_scale), wq_down,
+                         reinterpret_cast<const bf16*>(wq_down_scale)};
+    return layer_forward(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                         bias, nullptr, nullptr, reinterpret_cast<const bf16*>(ws_gate_up),
+                         reinterpret_cast<const bf16*>(ws_down), T, d, E, k, inter, scale,
+                         reinterpret_cast<bf16*>(out), workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream), nullptr, nullptr, &i4);
+}
+
+int moe_layer_forward_w4a16(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                            const uint8_t* wq_gate_up, const uint16_t* wq_gate_up_scale,
+                            const uint8_t* wq_down, const uint16_t* wq_down_scale,
+                            const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
+                            int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    int rc = check_dims(T, d, E, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down, wq_down_scale,
+                ws_gate_up, ws_down, out) ||
+        !(scale == scale))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = make_layout(T, d, E, k, inter).total;
+    void* ws = nullptr;
+    rc = owned_workspace(static_cast<cudaStream_t>(stream), need, &ws);
+    if (rc != MOE_OK) return rc;
+    return moe_layer_forward_w4a16_ws(x, w_router, bias, wq_gate_up, wq_gate_up_scale, wq_down,
+                                      wq_down_scale, ws_gate_up, ws_down, T, d, E, k, inter,
+                                      scale, out, ws, need, stream);
 }
 
 int moe_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,

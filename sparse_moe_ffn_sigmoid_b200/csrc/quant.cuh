@@ -139,6 +139,75 @@ __device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 v, const Fp8Scale& sc) {
     return out;
 }
 
+// ------------------------------------------------------------ INT4 storage
+// "Kimi K2.5 deep dive", CH7.2: the K2.5 routed experts' weights are 4-bit
+// integers, symmetric, one scale per group of 32 K elements of a row ("Kimi
+// K2.5 Q&A", Q7.1: storage quantized, compute BF16).  Rule (the config gives
+// none): s = bf16(amax / 7), q = clamp(nearest integer to w / s, ties to even,
+// -8, 7) (0 when s = 0); the weight computed with is bf16(q * s).
+// Device layout (this library's packing):
+//   codes  [rows, cols / 2] bytes: 32-bit word j of a row (little-endian) holds
+//          elements 8j .. 8j+7, element 8j + 2i in bits 4i .. 4i+3 and element
+//          8j + 2i + 1 in bits 16 + 4i .. 16 + 4i + 3, each as q + 8 (0 .. 15);
+//   scales [cols / 32, rows] bf16, group-major, so one TMA box brings a K step's
+//          scales of 128 rows.
+constexpr int kInt4Group = 32;
+constexpr int kInt4Warps = 8;             // groups per block of the quantizer
+
+// One warp per (row, group); lane = element of the group.  amax / 7 and w / s
+// are taken in fp32: amax / 7 never lies on a bf16 rounding midpoint and w / s
+// (two bf16 values) is either exactly on a half-integer or at least 2^-9 of
+// its size away from one, so both decisions equal the exact ones.
+__global__ void __launch_bounds__(32 * kInt4Warps) int4_quantize_kernel(
+    const bf16* __restrict__ w, long long rows, int cols, uint32_t* __restrict__ codes,
+    bf16* __restrict__ scale) {
+    const int gpr = cols / kInt4Group;
+    const long long gid = static_cast<long long>(blockIdx.x) * kInt4Warps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gid >= rows * gpr) return;
+    const long long r = gid / gpr;
+    const int g = static_cast<int>(gid - r * gpr);
+    const float v = __bfloat162float(w[r * cols + static_cast<long long>(g) * kInt4Group + lane]);
+    float amax = fabsf(v);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const bf16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+    const float sv = __bfloat162float(sb);
+    int n = 0;
+    if (sv != 0.0f) n = max(-8, min(7, __float2int_rn(__fdiv_rn(v, sv))));
+    const int e = lane & 7;                              // element within the word
+    const int nib = (e & 1) ? (e >> 1) + 4 : (e >> 1);
+    uint32_t bits = static_cast<uint32_t>(n + 8) << (4 * nib);
+    bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
+    bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
+    bits |= __shfl_xor_sync(0xffffffffu, bits, 4);
+    if (e == 0) codes[(r * cols + static_cast<long long>(g) * kInt4Group) / 8 + (lane >> 3)] = bits;
+    if (lane == 0) scale[static_cast<long long>(g) * rows + r] = sb;
+}
+
+// Eight packed codes (one word, layout above) -> eight bf16 weights bf16(q * s):
+// 0x4300 | n is the bf16 value 128 + n, so (128 + n) - 136 = q exactly, and one
+// bf16 multiply rounds q * s to nearest-even.
+__device__ __forceinline__ uint4 int4x8_to_bf16x8(uint32_t wd, __nv_bfloat162 s2) {
+    const uint32_t magic = 0x43004300u;
+    uint32_t v[4];
+    v[0] = (wd & 0x000F000Fu) | magic;
+    v[1] = ((wd >> 4) & 0x000F000Fu) | magic;
+    v[2] = ((wd >> 8) & 0x000F000Fu) | magic;
+    v[3] = ((wd >> 12) & 0x000F000Fu) | magic;
+    const uint32_t off_bits = 0x43084308u;               // 136.0 in both halves
+    const __nv_bfloat162 off = *reinterpret_cast<const __nv_bfloat162*>(&off_bits);
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v[i]), off);
+        const __nv_bfloat162 y = __hmul2(q, s2);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+    }
+    return out;
+}
+
 // ------------------------------------------------------------- FP8 compute
 // Operands of the FP8-compute GEMMs ("Kimi K2.5 Q&A", Q7.1: V3 computes in
 // FP8): E4M3 codes with one power-of-two exponent per ROW (a weight row is an

@@ -146,6 +146,46 @@ def test_quantize_fp8_rejects_bad_shapes():
     assert L.moe_quantize_fp8(FAKE, 128, 128, FAKE, NULL, NULL) == INVALID
 
 
+# ------------------------------------------------------------ INT4 weights
+
+def _layer_w4(T=64, d=7168, E=384, k=8, inter=2048, scale=2.827, ptrs=None, out=FAKE, ws=None):
+    p = ptrs if ptrs is not None else [FAKE] * 9
+    L = moe.lib()
+    if ws is None:
+        return L.moe_layer_forward_w4a16(*p, T, d, E, k, inter, ctypes.c_float(scale), out, NULL)
+    return L.moe_layer_forward_w4a16_ws(*p, T, d, E, k, inter, ctypes.c_float(scale), out, FAKE,
+                                        ws, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=7100), SHAPE), (dict(inter=2000), SHAPE), (dict(E=0), SHAPE), (dict(k=9, E=8), SHAPE),
+    (dict(T=-1), INVALID), (dict(scale=float("nan")), INVALID),
+])
+def test_w4a16_layer_rejects_bad_shapes(kw, code):
+    assert _layer_w4(**kw) == code
+
+
+def test_w4a16_layer_rejects_null_pointers_and_small_workspace():
+    for i in range(9):
+        p = [FAKE] * 9
+        p[i] = NULL
+        assert _layer_w4(ptrs=p) == INVALID
+    assert _layer_w4(out=NULL) == INVALID
+    need = moe.moe_workspace_size(64, 7168, 384, 8, 2048)
+    assert _layer_w4(ws=need - 1) == INVALID
+    assert _layer_w4(T=0) == OK
+
+
+def test_quantize_int4_rejects_bad_shapes():
+    L = moe.lib()
+    assert L.moe_quantize_int4(FAKE, 8, 96, FAKE, FAKE, NULL) == SHAPE     # not a multiple of 64
+    assert L.moe_quantize_int4(FAKE, -1, 128, FAKE, FAKE, NULL) == SHAPE
+    assert L.moe_quantize_int4(FAKE, 0, 128, FAKE, FAKE, NULL) == OK
+    assert L.moe_quantize_int4(NULL, 8, 128, FAKE, FAKE, NULL) == INVALID
+    assert L.moe_quantize_int4(FAKE, 8, 128, FAKE, NULL, NULL) == INVALID
+    assert L.moe_quantize_int4(FAKE, 8, 128, ctypes.c_void_p(0x10004), FAKE, NULL) == INVALID
+
+
 # ------------------------------------------------------------ FP8 compute
 
 def _layer_w8a8(T=64, d=7168, E=384, k=8, inter=2048, scale=2.827, ptrs=None, out=FAKE,

@@ -1,0 +1,158 @@
+"""INT4 storage of the routed experts' weights ("Kimi K2.5 deep dive", CH7.2:
+4-bit symmetric integers in groups of 32 along K; "Kimi K2.5 Q&A", Q7.1:
+storage quantized, compute BF16), CUDA path against the fp64 oracle (B200 only).
+
+- moe_quantize_int4: codes and group scales bit-exact against the oracle's
+  quantizer (the test only re-packs the oracle's codes into the library's
+  layout and transposes its scales: no arithmetic);
+- moe_layer_forward_w4a16: against the oracle's bf16 layer evaluated with the
+  weights the ORACLE's quantizer stands for, bf16(q * s); the bf16 layer's
+  tolerance, since the GPU computes with exactly those weights.
+No expected value comes from the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity as PR
+from moe_inputs import CONFIGS, MoEConfig, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe(cuda_ok):
+    import sparse_moe_ffn_sigmoid_b200 as m
+    m.moe_device_status()
+    return m
+
+
+def _u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def pack_codes(q):
+    """The library's packing of int codes [.., rows, cols] (layout only): word j
+    of a row holds elements 8j + 2i in bits 4i.. and 8j + 2i + 1 in bits 16 + 4i..,
+    each as q + 8; returned as bytes [.., rows, cols / 2]."""
+    n = (q.astype(np.int64) + 8).reshape(q.shape[:-1] + (q.shape[-1] // 8, 8))
+    word = np.zeros(n.shape[:-1], dtype=np.uint64)
+    for i in range(4):
+        word |= (n[..., 2 * i].astype(np.uint64) << np.uint64(4 * i))
+        word |= (n[..., 2 * i + 1].astype(np.uint64) << np.uint64(16 + 4 * i))
+    return word.astype(np.uint32).view(np.uint8).reshape(q.shape[:-1] + (q.shape[-1] // 2,))
+
+
+def _planted(shape, seed):
+    """Groups of many magnitudes, an all-zero group, a negative group maximum,
+    integer values (exact ties of w / s), bf16 subnormals."""
+    rng = np.random.default_rng(seed)
+    cols = shape[-1]
+    w = rng.normal(0, 1, shape)
+    w2 = w.reshape(-1, cols)
+    w2 *= 2.0 ** rng.integers(-30, 12, (w2.shape[0], cols // 32)).repeat(32, 1)
+    w2[0, :32] = 0.0
+    w2[0, 32:64] = rng.normal(0, 1e-3, 32)
+    w2[0, 40] = -3.0
+    w2[1, :32] = np.arange(32) - 16.0
+    w2[1, 32:64] = rng.normal(0, 1e-39, 32)
+    return torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("shape", [(4, 64), (37, 192), (3, 256, 512), (2053, 128)])
+def test_quantize_int4_bit_exact(moe, shape):
+    w = _planted(shape, seed=sum(shape))
+    codes, scales = moe.moe_quantize_int4(w.cuda())
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    q, sc = oracle.quantize_int4(_u16(w))
+    assert np.array_equal(codes.cpu().numpy(), pack_codes(q))
+    cols = shape[-1]
+    want = sc.reshape(-1, cols // 32).T
+    assert np.array_equal(scales.cpu().view(torch.int16).numpy().view(np.uint16), want)
+
+
+W4_CASES = [
+    MoEConfig("w4_small", T=64, d=512, E=16, k=4, inter=256, scale=2.827),
+    MoEConfig("w4_ragged", T=37, d=384, E=7, k=3, inter=192, scale=2.827),
+    MoEConfig("w4_multi_tile", T=600, d=256, E=16, k=4, inter=128, scale=2.827, bias="zipf"),
+    MoEConfig("w4_k2_dims", T=16, d=7168, E=4, k=2, inter=2048, scale=2.827),
+]
+
+
+def _oracle_w4_inputs(inp):
+    """Layer inputs with the routed experts' weights replaced by what the
+    oracle's own INT4 quantizer stands for (shared expert unchanged)."""
+    out = dict(inp)
+    for key in ("w_gate_up", "w_down"):
+        out[key] = oracle.dequantize_int4(*oracle.quantize_int4(_u16(inp[key])))
+    return out
+
+
+def _run(moe, g, cfg, out=None, ws=None):
+    qgu, sgu = moe.moe_quantize_int4(g["w_gate_up"])
+    qdn, sdn = moe.moe_quantize_int4(g["w_down"])
+    if out is None:
+        out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    args = (g["x"], g["w_router"], g["bias"], qgu, sgu, qdn, sdn, g["ws_gate_up"], g["ws_down"],
+            cfg.k, cfg.scale, out)
+    if ws is None:
+        moe.moe_layer_forward_w4a16(*args)
+    else:
+        moe.moe_layer_forward_w4a16_ws(*args, ws)
+    return out, (qgu, sgu, qdn, sdn)
+
+
+@pytest.mark.parametrize("cfg", W4_CASES, ids=lambda c: c.name)
+def test_w4a16_layer_parity(moe, cfg):
+    inp = make_inputs(cfg, seed=61)
+    g = {k: v.cuda() for k, v in inp.items()}
+    out, _ = _run(moe, g, cfg)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    ref, ridx, rw, gap = oracle.moe_forward(_oracle_w4_inputs(inp), cfg.k, cfg.scale)
+    PR.check_output(PR.bf16_np(out), ref, skip_rows=np.nonzero(gap < PR.TIE_EPS)[0])
+
+
+def test_w4a16_layer_deterministic_and_ws(moe):
+    cfg = W4_CASES[0]
+    g = {k: v.cuda() for k, v in make_inputs(cfg, seed=62).items()}
+    o1, _ = _run(moe, g, cfg)
+    o2, _ = _run(moe, g, cfg)
+    ws = torch.empty(moe.moe_workspace_size(cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter),
+                     dtype=torch.uint8, device="cuda")
+    o3, _ = _run(moe, g, cfg, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
+
+
+def test_w4a16_fullsize_decode(moe):
+    """K2 decode shape in the benchmark's launch configuration, sampled rows;
+    the sampled experts' GPU codes and scales equal the oracle quantizer's."""
+    cfg = CONFIGS["k2_decode"]
+    T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
+    g = make_inputs(cfg, seed=0, device="cuda")
+    out, (qgu, sgu, qdn, sdn) = _run(moe, g, cfg)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    x_h = g["x"].cpu()
+    ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
+    sample = [t for t in (0, T // 2, T - 1) if gap[t] >= PR.TIE_EPS]
+    need = sorted(set(ridx[sample].reshape(-1).tolist()))
+    egu = [None] * E
+    edn = [None] * E
+    sgu_h = sgu.cpu().view(torch.int16).numpy().view(np.uint16)
+    for e in need:
+        q, sc = oracle.quantize_int4(_u16(g["w_gate_up"][e]))
+        assert np.array_equal(qgu[e].cpu().numpy(), pack_codes(q))
+        assert np.array_equal(sgu_h[:, e * 2 * I:(e + 1) * 2 * I], sc.T)
+        egu[e] = oracle.dequantize_int4(q, sc)
+        edn[e] = oracle.dequantize_int4(*oracle.quantize_int4(_u16(g["w_down"][e])))
+    ref = oracle.moe_rows(x_h, ridx, rw, egu, edn, g["ws_gate_up"].cpu(), g["ws_down"].cpu(),
+                          tokens=np.array(sample, np.int32))
+    PR.check_output(PR.bf16_np(out[torch.tensor(sample, device="cuda")]), ref)
+    del g, qgu, qdn, out
+    torch.cuda.empty_cache()
