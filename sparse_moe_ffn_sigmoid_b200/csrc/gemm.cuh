@@ -63,7 +63,8 @@ constexpr int kTokenWarp = 10;
 // codes into the bf16 ring (two converter warps per SM sub-partition).
 constexpr int kEpiWarpsFP8 = 4;
 constexpr int kConvWarps = 8;
-constexpr int kConvThreads = 32 * kConvWarps;
+constexpr int kConvGroups = 2;                // converter groups, on alternating K steps
+constexpr int kConvThreads = 32 * kConvWarps / kConvGroups;   // threads per group
 constexpr int kGemmThreadsFP8 = 480;
 constexpr int kSlabBytes8 = kSlabRows * kBK;  // one FP8 slab per K step (128 rows x 64 codes)
 // INT4 slab per K step: 128 rows x 64 codes packed in 32 bytes, then the step's two
@@ -220,41 +221,49 @@ __device__ __forceinline__ bool wait_lane0(uint64_t* bar, uint32_t parity, volat
     return ok;
 }
 
-// FP8-weight mode: the kConvWarps converter warps (thread ct = 0..127) fill
-// the bf16 weight ring for every K step, in step order, all four warps
-// together: at every step each warp waits for the bf16 slot (empty: the MMAs
-// of step q - SA done), and for a routed step also for its codes (full8).
-// Parity waits only tell a phase from the one before it, so every warp waits
-// at every step and the warps meet on a named barrier once per step: none can
-// run a lap ahead of the slot's barrier (and write a slot the MMA still
-// reads) or fall a lap behind it.
-// Routed step: thread ct converts eight codes at a time, units u = ct + 128 i
-// (slab u / 1024, row (u / 8) % 128, chunk u % 8), into the 128-byte-swizzled
-// layout a TMA box would have produced (row r at byte 128 r, 16-byte chunk c
-// at position c ^ (r % 8)); each code times the block's 2^s is exact in bf16.
-// Every thread fences its stores towards the async proxy before the barrier,
-// and thread 0 then publishes the slot (full) and frees the codes (empty8).
-// Shared-expert step (bf16 in HBM): after the barrier thread 0 loads the bf16
-// weights into the slot with TMA (arrive.expect_tx on full).  The weight
-// producer, which runs up to SA8 routed steps ahead, never touches the bf16
-// ring in this mode.
-// OPS = kOpsW8Convert: E4M3 codes (64 bytes per slab row) and one block exponent
-// per slab and step; kOpsW4Convert: packed INT4 codes (32 bytes per slab row,
-// one 32-bit word per unit) and the step's two group scales per row in the slot.
+// Converting modes: the kConvWarps converter warps fill the bf16 weight ring
+// in two groups of four warps (one per SM sub-partition each); group g takes
+// the K steps q = g mod 2, so two steps are converted at once.  At each of its
+// steps every warp of the group waits for the step's code slot (full8: the
+// codes landed, or the producer's plain arrival on a shared-expert step) and
+// for the bf16 slot (empty: the MMAs of step q - SA done), and the group's
+// warps meet on their own named barrier once per step.  The code ring is
+// indexed by the global step like the bf16 ring, so every slot use is waited
+// on by the group that makes it.  A waiter can never be two phases behind a
+// slot's barrier: its previous step needed the MMAs (or codes) of an earlier
+// use of every slot, which run in step order.
+// Routed step: thread ct (0 .. 127 of its group) converts eight codes at a
+// time, units u = ct + 128 i (slab u / 1024, row (u / 8) % 128, chunk u % 8),
+// into the 128-byte-swizzled layout a TMA box would have produced (row r at
+// byte 128 r, 16-byte chunk c at position c ^ (r % 8)).  Every thread fences
+// its stores towards the async proxy before the barrier, and the group's
+// thread 0 then publishes the slot (full) and frees the codes (empty8).
+// Shared-expert step (bf16 in HBM): after the barrier the group's thread 0
+// loads the bf16 weights into the slot with TMA (arrive.expect_tx on full) and
+// frees the (unused) code slot.
 template <int nslab, int OPS>
 __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint8_t* ring8,
                                                 uint8_t* ring_a, int SA, int SA8, uint64_t* full,
                                                 uint64_t* empty, uint64_t* full8,
                                                 uint64_t* empty8, volatile int* abort_flag,
-                                                uint64_t tmo, int ntiles, int ct) {
+                                                uint64_t tmo, int ntiles, int grp, int ct) {
     constexpr bool kInt4 = (OPS == kOpsW4Convert);
     constexpr uint32_t a8_bytes = nslab * code_slab_bytes(OPS);
     constexpr uint32_t a_bytes = nslab * kSlabBytes;
     constexpr int kUnits = nslab * kSlabRows * (kBK / 8) / kConvThreads;   // per thread
+    static_assert(kUnits == 16 && nslab == 2, "unit geometry: 2 slabs x 8 row blocks");
     const int lane = ct & 31;
+    // thread-constant geometry of the units u = ct + 128 j: chunk c = ct % 8,
+    // rows r0 + 16 (j % 8) with r0 = ct / 8, slab j / 8; (r0 + 16 i) % 8 == r0 % 8,
+    // so the 128-byte swizzle of the destination chunk is a thread constant too
+    const int r0 = ct >> 3, cc = ct & 7;
+    const uint32_t dst_off = r0 * (kBK * 2) + ((cc ^ (r0 & 7)) << 4);
+    const uint32_t code_off = kInt4 ? r0 * (kBK / 2) + cc * 4 : r0 * kBK + cc * 8;
+    const uint32_t scale_off = kSlabCodes4 + (cc >> 2) * (kSlabRows * 2) + r0 * 2;
     const uint64_t pol = ptx::policy_evict_first();
     Ring rq{0, 0, SA};          // bf16 slot of step q
-    Ring r8{0, 0, SA8};         // code slot of the routed steps
+    Ring r8{0, 0, SA8};         // code slot of step q
+    uint32_t q = 0;
     bool ok = true;
     uint32_t issued = 0, issued_parity = 0;   // thread 0's bf16 loads, for draining
     for (int i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
@@ -264,32 +273,30 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
             kInt4 ? nullptr : args.a8_scale + (t.a_row0 / kQuantBlock) * args.a8_kblocks;
         const int8_t* sc1 =
             kInt4 ? nullptr : args.a8_scale + (t.a_row1 / kQuantBlock) * args.a8_kblocks;
-        for (int ks = t.ks0; ks < t.ks1; ++ks) {
-            bool w_ok = (!routed || wait_lane0(&full8[r8.stage], r8.phase, abort_flag, tmo, lane)) &&
+        for (int ks = t.ks0; ks < t.ks1; ++ks, ++q) {
+            if (static_cast<int>(q & 1) != grp) {     // the other group's step
+                r8.next();
+                rq.next();
+                continue;
+            }
+            bool w_ok = wait_lane0(&full8[r8.stage], r8.phase, abort_flag, tmo, lane) &&
                         wait_lane0(&empty[rq.stage], rq.phase ^ 1, abort_flag, tmo, lane);
             if (kInt4 && routed && w_ok) {
                 const uint8_t* src = ring8 + r8.stage * a8_bytes;
                 uint8_t* dst = ring_a + rq.stage * a_bytes;
-                // unit u: slab u / 1024, row (u / 8) % 128, 8-code chunk u % 8 (group chunk / 4)
+                // unit j: slab j / 8, row r0 + 16 (j % 8), 8-code chunk c (group c / 4):
+                // every offset is a thread constant plus a compile-time one
                 uint32_t words[kUnits];
 #pragma unroll
-                for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + kConvThreads * j;
-                    const int slab = u / (kSlabRows * 8);
-                    const int r = (u >> 3) & (kSlabRows - 1);
-                    words[j] = *reinterpret_cast<const uint32_t*>(src + slab * kSlabBytes4 +
-                                                                  r * (kBK / 2) + (u & 7) * 4);
-                }
+                for (int j = 0; j < kUnits; ++j)
+                    words[j] = *reinterpret_cast<const uint32_t*>(
+                        src + code_off + (j / 8) * kSlabBytes4 + (j % 8) * 16 * (kBK / 2));
 #pragma unroll
                 for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + kConvThreads * j;
-                    const int slab = u / (kSlabRows * 8);
-                    const int r = (u >> 3) & (kSlabRows - 1);
-                    const int c = u & 7;
                     const bf16 sc = *reinterpret_cast<const bf16*>(
-                        src + slab * kSlabBytes4 + kSlabCodes4 + (c >> 2) * (kSlabRows * 2) + r * 2);
-                    *reinterpret_cast<uint4*>(dst + slab * kSlabBytes + r * (kBK * 2) +
-                                              ((c ^ (r & 7)) << 4)) =
+                        src + scale_off + (j / 8) * kSlabBytes4 + (j % 8) * 16 * 2);
+                    *reinterpret_cast<uint4*>(dst + dst_off + (j / 8) * kSlabBytes +
+                                              (j % 8) * 16 * (kBK * 2)) =
                         int4x8_to_bf16x8(words[j], __bfloat162bfloat162(sc));
                 }
                 ptx::fence_proxy_async_smem();
@@ -302,32 +309,23 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 // the kUnits chains are independent, so their latencies overlap
                 uint2 codes[kUnits];
 #pragma unroll
-                for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + kConvThreads * j;
-                    const int slab = u / (kSlabRows * 8);
-                    const int r = (u >> 3) & (kSlabRows - 1);
-                    codes[j] = *reinterpret_cast<const uint2*>(src + slab * kSlabBytes8 + r * kBK +
-                                                               (u & 7) * 8);
-                }
+                for (int j = 0; j < kUnits; ++j)
+                    codes[j] = *reinterpret_cast<const uint2*>(
+                        src + code_off + (j / 8) * kSlabBytes8 + (j % 8) * 16 * kBK);
 #pragma unroll
-                for (int j = 0; j < kUnits; ++j) {
-                    const int u = ct + kConvThreads * j;
-                    const int slab = u / (kSlabRows * 8);
-                    const int r = (u >> 3) & (kSlabRows - 1);
-                    const int c = u & 7;
-                    *reinterpret_cast<uint4*>(dst + slab * kSlabBytes + r * (kBK * 2) +
-                                              ((c ^ (r & 7)) << 4)) =
-                        fp8x8_to_bf16x8(codes[j], slab == 0 ? s0 : s1);
-                }
+                for (int j = 0; j < kUnits; ++j)
+                    *reinterpret_cast<uint4*>(dst + dst_off + (j / 8) * kSlabBytes +
+                                              (j % 8) * 16 * (kBK * 2)) =
+                        fp8x8_to_bf16x8(codes[j], j < 8 ? s0 : s1);
                 ptx::fence_proxy_async_smem();
             }
-            // every converter thread reaches this barrier once per step
-            ok = ptx::bar_red_and(1, kConvThreads, w_ok);
+            // every thread of the group reaches its barrier once per step of the group
+            ok = ptx::bar_red_and(1 + grp, kConvThreads, w_ok);
             if (!ok) break;
             if (ct == 0) {
+                ptx::mbar_arrive(&empty8[r8.stage]);
                 if (routed) {
                     ptx::mbar_arrive(&full[rq.stage]);
-                    ptx::mbar_arrive(&empty8[r8.stage]);
                 } else {
                     uint64_t* bar = &full[rq.stage];
                     uint8_t* sa = ring_a + rq.stage * a_bytes;
@@ -340,7 +338,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                     issued_parity = (issued_parity & ~(1u << rq.stage)) | (rq.phase << rq.stage);
                 }
             }
-            if (routed) r8.next();
+            r8.next();
             rq.next();
         }
     }
@@ -451,21 +449,21 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
                 const int npad = pad16(t.n);
                 const uint32_t tx = weights ? a_bytes : npad * kBK * 2;
                 for (int ks = t.ks0; ks < t.ks1; ++ks, ++q) {
-                    if (FP8A && weights && t.map != 0) {
-                        // shared-expert step: the converter warps load its bf16
-                        // weights (they track the bf16 ring step by step; this
-                        // thread runs up to SA8 routed steps ahead of it and must
-                        // not wait on its barriers)
-                        rq.next();
-                        rb.next();
-                        continue;
-                    }
                     if (FP8A && weights) {
-                        // routed step: E4M3 codes into the code ring; the converter
-                        // warps fill and publish the bf16 slot
+                        // every step takes a code slot: a routed step's codes go
+                        // into it, a shared-expert step only completes its phase
+                        // (the converter group loads that step's bf16 weights); the
+                        // converter warps fill and publish the bf16 slot
                         if (!wait_bounded(&empty8[r8.stage], r8.phase ^ 1, abort_flag, tmo)) {
                             ok = false;
                             break;
+                        }
+                        if (t.map != 0) {
+                            ptx::mbar_arrive(&full8[r8.stage]);
+                            r8.next();
+                            rq.next();
+                            rb.next();
+                            continue;
                         }
                         uint64_t* bar8 = &full8[r8.stage];
                         ptx::mbar_arrive_expect_tx(bar8, a8_bytes);
@@ -619,9 +617,13 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
         }
     } else if (FP8A && warp >= 2 + kEpiWarpsFP8) {
         // ---------------------------------------------------------- converters
-        convert_weights<nslab, OPS>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
-                               abort_flag, tmo, ntiles,
-                               32 * (warp < kTokenWarp ? warp - 6 : warp - 7) + lane);
+        // group 0: warps 6..9, group 1: warps 11..14 (one warp per sub-partition each)
+        if constexpr (FP8A) {
+            const int grp = warp < kTokenWarp ? 0 : 1;
+            convert_weights<nslab, OPS>(args, ring8, ring_a, SA, SA8, full, empty, full8, empty8,
+                                        abort_flag, tmo, ntiles, grp,
+                                        32 * (warp - (grp == 0 ? 6 : 11)) + lane);
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp

@@ -337,7 +337,9 @@ void fill_pipeline_fp8(GemmArgs& a, int n_max, int code_slab = kSlabBytes8) {
     const size_t b_bytes = static_cast<size_t>(n_max) * kBK * 2;
     const size_t budget = kMaxDynSmem - 1024 - kStagingBytes - 1024;
     a.stages_b = (n_max <= 64 || n_max > 128) ? 2 : 3;
-    a.stages_a = std::max(a.stages_b, n_max <= 128 ? 3 : 2);
+    // two converter groups work on alternating steps: at decode each gets two
+    // bf16 slots
+    a.stages_a = std::max(a.stages_b, n_max <= 64 ? 4 : n_max <= 128 ? 3 : 2);
     const size_t left = budget - a.stages_a * a_bytes - a.stages_b * b_bytes;
     a.stages_a8 = static_cast<int>(std::min<size_t>(12, left / a8_bytes));
 }
