@@ -129,10 +129,15 @@ def test_w4a16_layer_deterministic_and_ws(moe):
     assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
 
 
-def test_w4a16_fullsize_decode(moe):
-    """K2 decode shape in the benchmark's launch configuration, sampled rows;
-    the sampled experts' GPU codes and scales equal the oracle quantizer's."""
-    cfg = CONFIGS["k2_decode"]
+FULL = ["k2_decode", "k2_prefill", "k2_skew", "v3"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_w4a16_fullsize(moe, name):
+    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration,
+    sampled rows (token 0, T/2, T-1, the busiest expert's first token); the
+    sampled experts' GPU codes and scales equal the oracle quantizer's."""
+    cfg = CONFIGS[name]
     T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
     g = make_inputs(cfg, seed=0, device="cuda")
     out, (qgu, sgu, qdn, sdn) = _run(moe, g, cfg)
@@ -140,7 +145,9 @@ def test_w4a16_fullsize_decode(moe):
     assert moe.moe_device_status() == 0
     x_h = g["x"].cpu()
     ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
-    sample = [t for t in (0, T // 2, T - 1) if gap[t] >= PR.TIE_EPS]
+    counts, offsets, row_token, _ = oracle.permute(ridx, E)
+    first_of_busiest = int(row_token[offsets[int(np.argmax(counts))]])
+    sample = sorted({0, T // 2, T - 1, first_of_busiest} - set(np.nonzero(gap < PR.TIE_EPS)[0]))
     need = sorted(set(ridx[sample].reshape(-1).tolist()))
     egu = [None] * E
     edn = [None] * E

@@ -126,10 +126,22 @@ def test_w8a8_layer_deterministic_and_ws(moe):
     assert "quantize_h" in names and moe.moe_last_launch_count() == len(names)
 
 
-def test_w8a8_fullsize_decode(moe):
-    """K2 decode shape in the benchmark's launch configuration, sampled rows;
-    the sampled experts' GPU codes equal the oracle quantizer's."""
-    cfg = CONFIGS["k2_decode"]
+FULL = ["k2_decode", "k2_prefill", "k2_skew", "v3"]
+
+
+def _sample_tokens(ridx, gap, E, T):
+    """Token 0, T/2, T-1 and the first token of the busiest expert (near-ties out)."""
+    counts, offsets, row_token, _ = oracle.permute(ridx, E)
+    busiest = int(np.argmax(counts))
+    first_of_busiest = int(row_token[offsets[busiest]])
+    return sorted({0, T // 2, T - 1, first_of_busiest} - set(np.nonzero(gap < PR.TIE_EPS)[0]))
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_w8a8_fullsize(moe, name):
+    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration,
+    sampled rows; the sampled experts' GPU codes equal the oracle quantizer's."""
+    cfg = CONFIGS[name]
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     g = make_inputs(cfg, seed=0, device="cuda")
     wq = _quantize_all(moe, g)
@@ -139,7 +151,7 @@ def test_w8a8_fullsize_decode(moe):
     assert moe.moe_device_status() == 0
     x_h = g["x"].cpu()
     ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
-    sample = [t for t in (0, T // 2, T - 1) if gap[t] >= PR.TIE_EPS]
+    sample = _sample_tokens(ridx, gap, E, T)
     need = sorted(set(ridx[sample].reshape(-1).tolist()))
     host = {"w_gate_up": {e: g["w_gate_up"][e].cpu() for e in need},
             "w_down": {e: g["w_down"][e].cpu() for e in need},
