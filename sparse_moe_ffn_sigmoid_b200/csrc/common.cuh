@@ -26,13 +26,15 @@ constexpr int kStatusTimeout = -4;      // MOE_ERR_TIMEOUT
 
 // Bounded wait on an mbarrier phase.  Returns false (and records a timeout)
 // once `timeout_ns` has passed, or at once if another role of the CTA has
-// already given up (`abort_flag` set).
+// already given up (`abort_flag` set).  After a first plain test the thread
+// sleeps in the barrier (suspend-time hint of 20 us) between checks of the
+// abort flag and the clock, so a waiting role takes few issue slots.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
                                              volatile int* abort_flag, uint64_t timeout_ns) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ptx::mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (abort_flag && *abort_flag) return false;
         if (ptx::globaltimer_ns() - t0 > timeout_ns) {
             if (abort_flag) *abort_flag = 1;
