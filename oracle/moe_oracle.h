@@ -15,7 +15,7 @@
  *     7. out = shared + sum_j w_j * y_j
  *   "Kimi K2.5 Q&A" Q8.3 gives the same order (router -> shared || routed -> add).
  *
- * Readings where the pages are silent or disagree (each listed in the design doc):
+ * Readings where the pages are silent or disagree:
  *   - step 4 uses the UNBIASED sigmoid scores (the bias only picks experts);
  *   - ties in step 3 go to the lower expert index; slot j = j-th largest b;
  *   - no epsilon in the renormalisation (a sum of k sigmoids is > 0);
