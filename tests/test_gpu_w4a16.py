@@ -78,6 +78,7 @@ W4_CASES = [
     MoEConfig("w4_ragged", T=37, d=384, E=7, k=3, inter=192, scale=2.827),
     MoEConfig("w4_multi_tile", T=600, d=256, E=16, k=4, inter=128, scale=2.827, bias="zipf"),
     MoEConfig("w4_k2_dims", T=16, d=7168, E=4, k=2, inter=2048, scale=2.827),
+    MoEConfig("w4_one_token_k_eq_E", T=1, d=128, E=4, k=4, inter=64, scale=2.827),
 ]
 
 
