@@ -76,7 +76,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* scra
 // Tile plan of the grouped SwiGLU FFN.  Expert g (0..G-1) owns rows
 // [row0_g, row0_g + c_g); the shared expert (if present) is g = G-1 and reads
 // its tokens from the unpermuted map.  Each expert's rows are cut into
-// ceil(c/kTileN) token tiles of equal 16-multiple size; tiles are listed expert
+// ceil(c/tile_n) token tiles of equal 16-multiple size; tiles are listed expert
 // by expert, feature tile by feature tile, token tile fastest, so that tiles
 // sharing a weight slab or a token tile run side by side.
 struct PlanArgs {
@@ -88,6 +88,7 @@ struct PlanArgs {
     int4* tiles2;          // down tiles
     int* ntiles;           // [0] = gate|up count, [1] = down count
     int kstep = kBK;       // K elements per GEMM step (FP8 compute: 2 * kBK)
+    int tile_n = kTileN;   // largest token tile (a multiple of 16, <= kTileN)
 };
 
 constexpr int kPlanMaxG = 1025;   // up to 1024 routed experts and the shared one
@@ -124,7 +125,7 @@ __device__ __forceinline__ void plan_counts(const PlanArgs& p, int c, int* n1, i
         *n1 = *n2 = 0;
         return;
     }
-    const int nt = (c + kTileN - 1) / kTileN;
+    const int nt = (c + p.tile_n - 1) / p.tile_n;
     *n1 = nt * ((p.inter + kSlabRows - 1) / kSlabRows);
     *n2 = nt * ((p.d + 2 * kSlabRows - 1) / (2 * kSlabRows));
 }
@@ -181,7 +182,7 @@ __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) 
     for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
         const int cg = s_c[g];
         if (cg <= 0) continue;
-        const int nt = (cg + kTileN - 1) / kTileN;
+        const int nt = (cg + p.tile_n - 1) / p.tile_n;
         const int chunk = pad16((cg + nt - 1) / nt);
         const int row0 = s_row0[g];
         for (int l = lane; l < nt * ft1; l += 32)
