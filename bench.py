@@ -638,7 +638,7 @@ def run_reference(args, cfg, world):
     if args.cpu_sample:
         n = args.cpu_sample
     else:
-        probe = OracleSample(cfg, g, 1)        # one token measures the per-token cost
+        probe = OracleSample(cfg, g, 1, args.weights)   # one token measures the per-token cost
         per_token = probe.run()
         waves = max(1, int(REFERENCE_BUDGET_S / runs / per_token))
         n = max(1, min(cfg.T, waves * host_cores()))
