@@ -151,6 +151,11 @@ int moe_layer_forward(const uint16_t* x, const uint16_t* w_router, const float* 
 /*
  * moe_layer_forward with caller-owned scratch of at least
  * moe_workspace_size(T, d, E, k, inter) bytes (nothing is allocated).
+ * The _ws entries (this one, _fp8_ws, _w4a16_ws, _w8a8_ws) neither allocate nor
+ * synchronise the host, so a call can be captured into a CUDA graph on
+ * `stream` and replayed; make one call on the device outside the capture first
+ * (it sets up the kernels' attributes).  A replay uses the pointers and sizes
+ * of the captured call.
  */
 int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
                          const uint16_t* w_gate_up, const uint16_t* w_down,
