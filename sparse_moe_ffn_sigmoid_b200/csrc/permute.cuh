@@ -320,4 +320,103 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
     for (; v < nv; v += 32) dst[v] = __ldg(src + v);
 }
 
+// The same permuted rows built token by token: x[t] is read once and written to
+// its k rows slot_row[t*k + j] (one warp per token, 16-byte vectors, lane j
+// holding the j-th destination).  At prefill this reads x once instead of k
+// times (the row-by-row gather's re-reads miss L2 behind its write stream).
+// A destination outside [0, rows) records kStatusInvalidArg and is skipped.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const bf16* __restrict__ x,
+                                                           const int* __restrict__ slot_row,
+                                                           int T, int k, int rows, int d,
+                                                           bf16* __restrict__ xperm) {
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    int dst = lane < k ? slot_row[static_cast<long long>(t) * k + lane] : 0;
+    if (lane < k && (dst < 0 || dst >= rows)) {
+        record_status(kStatusInvalidArg);
+        dst = -1;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<long long>(t) * d);
+    const int nv = d / 8;
+    // every lane runs every round (the shuffles need the whole warp); only the
+    // lanes with a vector in the row load and store
+    for (int base = 0; base < nv; base += 32) {
+        const int v = base + lane;
+        const bool has = v < nv;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (has) val = __ldg(src + v);
+        for (int j = 0; j < k; ++j) {
+            const int r = __shfl_sync(0xffffffffu, dst, j);
+            if (has && r >= 0)
+                reinterpret_cast<uint4*>(xperm + static_cast<long long>(r) * d)[v] = val;
+        }
+    }
+}
+
+// Token rows of the FP8-compute layer, token by token: x[t] (bf16, d columns)
+// is quantized once (rule above) and its codes and exponent written to the k
+// permuted rows slot_row[t*k + j] and to row rows_routed + t (token order).
+// One warp per token; the second pass re-reads the row from L1/L2.  A
+// destination outside [0, rows_routed) records kStatusInvalidArg and is skipped.
+__global__ void __launch_bounds__(32 * kRowQuantWarps) fp8_quantize_tokens_kernel(
+    const bf16* __restrict__ x, const int* __restrict__ slot_row, int T, int k,
+    long long rows_routed, int d, uint8_t* __restrict__ q, int8_t* __restrict__ sexp) {
+    const int t = blockIdx.x * kRowQuantWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    const long long tok_row = rows_routed + t;
+    long long dst = lane < k ? static_cast<long long>(slot_row[static_cast<long long>(t) * k + lane])
+                             : -1;
+    if (lane < k && (dst < 0 || dst >= rows_routed)) {
+        record_status(kStatusInvalidArg);
+        dst = -1;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(x + static_cast<long long>(t) * d);
+    const int nv = d / 8;
+    float amax = 0.0f;
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) {
+        const uint4 u = __ldg(s + v);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int e = fp8_block_exponent(amax);
+    if (dst >= 0) sexp[dst] = static_cast<int8_t>(e);
+    if (lane == 0) sexp[tok_row] = static_cast<int8_t>(e);
+    const float m1 = pow2f(-(e / 2));
+    const float m2 = pow2f(-(e - e / 2));
+    // every lane runs every round (the shuffles need the whole warp); only the
+    // lanes with a vector in the row load, convert and store
+    for (int base = 0; base < nv; base += 32) {
+        const int v = base + lane;
+        const bool has = v < nv;
+        uint2 out = make_uint2(0u, 0u);
+        if (has) {
+            const uint4 u = __ldg(s + v);
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+            uint8_t* o = reinterpret_cast<uint8_t*>(&out);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(p[j]);
+                o[2 * j] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.x, m1), m2), __NV_SATFINITE,
+                                                 __NV_E4M3);
+                o[2 * j + 1] = __nv_cvt_float_to_fp8(__fmul_rn(__fmul_rn(f.y, m1), m2),
+                                                     __NV_SATFINITE, __NV_E4M3);
+            }
+        }
+        for (int j = 0; j < k; ++j) {
+            const long long r = __shfl_sync(0xffffffffu, dst, j);
+            if (has && r >= 0) reinterpret_cast<uint2*>(q + r * d)[v] = out;
+        }
+        if (has) reinterpret_cast<uint2*>(q + tok_row * d)[v] = out;
+    }
+}
+
 }  // namespace moe

@@ -210,6 +210,10 @@ LAYER_CASES = [
     MoEConfig("k1", T=45, d=192, E=6, k=1, inter=128, scale=2.5),
     MoEConfig("zipf_multi_tile", T=600, d=256, E=16, k=4, inter=128, scale=2.827, bias="zipf"),
     MoEConfig("max_e_k", T=64, d=128, E=1024, k=32, inter=64, scale=2.827),
+    # T >= 1024: the token rows are permuted token by token; rows of 16 and 48
+    # 16-byte vectors leave part of the warp without a vector in the last round
+    MoEConfig("token_major_d128", T=1100, d=128, E=64, k=8, inter=64, scale=2.827),
+    MoEConfig("token_major_d384_k32", T=1030, d=384, E=48, k=32, inter=64, scale=2.827),
 ]
 
 

@@ -77,6 +77,9 @@ W8A8_CASES = [
     MoEConfig("w8a8_k2_dims", T=16, d=7168, E=4, k=2, inter=2048, scale=2.827),
     MoEConfig("w8a8_v3_scale", T=100, d=384, E=12, k=6, inter=256, scale=2.5),
     MoEConfig("w8a8_one_token_k_eq_E", T=2, d=128, E=8, k=8, inter=128, scale=2.827),
+    # T >= 1024: token rows quantized token by token (rows of 16 and 48 vectors)
+    MoEConfig("w8a8_token_major_d128", T=1100, d=128, E=32, k=8, inter=128, scale=2.827),
+    MoEConfig("w8a8_token_major_d384", T=1030, d=384, E=16, k=4, inter=128, scale=2.827),
 ]
 
 
