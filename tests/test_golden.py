@@ -55,3 +55,27 @@ def test_layer_flops_per_token_equal_the_printed_dense_ffn():
     acc1 = bench.layer_accounting(cfg, touched=1)
     acc0 = bench.layer_accounting(cfg, touched=0)
     assert acc1["weight_bytes"] - acc0["weight_bytes"] == 3 * cfg.d * cfg.inter * 2
+
+
+@pytest.mark.parametrize("weights,per_expert,shared", [
+    # routed bytes per expert (gate|up + down) and the shared expert's, per format
+    ("bf16", 3 * 7168 * 2048 * 2, 3 * 7168 * 2048 * 2),
+    # E4M3 codes + one int8 exponent per 128 x 128 block; shared expert stays bf16
+    ("fp8", 3 * 7168 * 2048 + (4096 // 128) * (7168 // 128) + (7168 // 128) * (2048 // 128),
+     3 * 7168 * 2048 * 2),
+    # INT4: half a byte per weight + one bf16 scale per 32 K elements; shared bf16
+    ("w4a16", 3 * 7168 * 2048 // 2 + (4096 * (7168 // 32) + 7168 * (2048 // 32)) * 2,
+     3 * 7168 * 2048 * 2),
+    # FP8 compute: codes + one int8 exponent per row, shared expert included
+    ("w8a8", 3 * 7168 * 2048 + 4096 + 7168, 3 * 7168 * 2048 + 4096 + 7168),
+])
+def test_weight_bytes_per_format(weights, per_expert, shared):
+    import bench
+    cfg = CONFIGS["k2_decode"]
+    acc0 = bench.layer_accounting(cfg, touched=0, weights=weights)
+    acc1 = bench.layer_accounting(cfg, touched=1, weights=weights)
+    assert acc1["weight_bytes"] - acc0["weight_bytes"] == per_expert
+    router = cfg.E * cfg.d * 2
+    assert acc0["weight_bytes"] == shared + router
+    # the FLOPs do not depend on the weight format
+    assert acc1["flops"] == bench.layer_accounting(cfg, touched=1)["flops"]
