@@ -63,6 +63,9 @@ def parse_args(argv=None):
                    help="tokens in the oracle's timed sample (default: sized from the core count)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="time the decode headline only (the default run also times k2_prefill, "
+                        "k2_skew and v3 on the same weights)")
     p.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                    help="override a workload field (T, d, E, k, inter), e.g. a small case of\n"
                         "the same kernels for profiling: --set E=16")
@@ -100,6 +103,8 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    PERIOD_MS = 20          # a 20-step decode run lasts about 70 ms
+
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
@@ -109,7 +114,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -244,6 +249,122 @@ def layer_accounting(cfg, touched: int, weights: str = "bf16"):
     acc["weight_bytes"] = touched * (r_gu + r_dn) + (w_gu + w_dn) + E * d * 2
     acc["flops"] = acc["gate_up_flops"] + acc["down_flops"] + acc["router_flops"]
     return acc
+
+
+# ------------------------------------------------ other full-size workloads
+
+# Timed after the decode line in the default run, on the decode run's weights.
+EXTRA_WORKLOADS = ("k2_prefill", "k2_skew", "v3")
+EXTRA_TIMED_MS = 1000.0     # device time each one's timed region aims at (clock samples)
+
+
+def extra_inputs(name, g, dev, seed):
+    """Inputs of another full-size workload on the decode run's weight set.
+    The expert shapes are the same (d = 7168, inter = 2048), so the 384 routed
+    experts, the router rows and the shared expert are reused (the first 256
+    experts and router rows for the DeepSeek-V3 shape); x and the selection
+    bias are drawn for the workload with the distributions moe_inputs states."""
+    import torch
+    from moe_inputs import CONFIGS, make_bias
+    cfg = CONFIGS[name]
+    E = cfg.E
+    if cfg.d != g["x"].shape[1] or cfg.inter != g["w_down"].shape[2] or E > g["w_router"].shape[0]:
+        raise ValueError(f"{name}: expert shapes differ from the decode weight set")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    x = torch.randn((cfg.T, cfg.d), generator=gen, device=dev, dtype=torch.float32)
+    inp = dict(x=x.to(torch.bfloat16), w_router=g["w_router"][:E], bias=make_bias(cfg, gen, dev),
+               w_gate_up=g["w_gate_up"][:E], w_down=g["w_down"][:E], ws_gate_up=g["ws_gate_up"],
+               ws_down=g["ws_down"])
+    return cfg, inp
+
+
+def touched_experts(moe, cfg, g, dev) -> int:
+    """Routed experts with at least one token in this batch (our own route and
+    permute kernels)."""
+    import torch
+    T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
+    ws = torch.empty(moe.moe_workspace_size(T, d, E, k, I), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    moe.moe_route(g["x"], g["w_router"], g["bias"], k, cfg.scale, idx, w, ws)
+    i32 = lambda n: torch.empty((n,), dtype=torch.int32, device=dev)
+    counts, offs, rtok, srow = i32(E), i32(E + 1), i32(T * k), i32(T * k)
+    moe.moe_permute(idx, E, counts, offs, rtok, srow, ws)
+    return int((counts > 0).sum().item())
+
+
+def time_extra_workload(moe, cfg, inp, dev, warmup, peaks, peak_src, gpu_index):
+    """One bf16 layer workload, device-timed like the headline (CUDA events on
+    the launching stream, inputs resident, clocks sampled during the timed
+    region), with its tensor fraction against both measured bf16 peaks, its
+    HBM fraction, and its time in SM cycles at the sampled clock."""
+    import torch
+    T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        moe.moe_layer_forward(inp["x"], inp["w_router"], inp["bias"], inp["w_gate_up"],
+                              inp["w_down"], inp["ws_gate_up"], inp["ws_down"], k, cfg.scale, out)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(warmup):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_warm = start.elapsed_time(end) / warmup
+    steps = int(min(400, max(20, math.ceil(EXTRA_TIMED_MS / max(ms_warm, 1e-3)))))
+    touched = touched_experts(moe, cfg, inp, dev)
+
+    moe.moe_profile_begin(steps)
+    with ClockSampler(gpu_index) as clk:
+        torch.cuda.synchronize(dev)
+        t0 = clk.mark()
+        start.record(stream)
+        for _ in range(steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        t1 = clk.mark()
+    ms = start.elapsed_time(end) / steps
+    n_calls, kernel_ms = moe.moe_profile_end()
+    if moe.moe_device_status() != 0:
+        raise SystemExit(f"{cfg.name}: device status not clean after the timed region")
+    clocks = clk.summary(t0, t1)
+
+    acc = layer_accounting(cfg, touched)
+    burst = peaks["bf16_tflops"]
+    sust = peaks.get("bf16_tflops_sustained", burst)
+    hbm_peak = peaks["hbm_gbs"]
+    tflops = acc["flops"] / (ms / 1e3) / 1e12
+    gu_ms = kernel_ms.get("gemm_gate_up_swiglu", 0.0) / max(n_calls, 1)
+    gu_tflops = acc["gate_up_flops"] / (gu_ms / 1e3) / 1e12 if gu_ms > 0 else None
+    hbm = acc["weight_bytes"] / (ms / 1e3) / 1e9
+    mhz = clocks["sm_mhz"]
+    return {
+        "T": T, "E": E, "k": k, "scale": cfg.scale, "bias": cfg.bias, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+        "touched_experts": touched, "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
+        "tensor": {"achieved_tflops": tflops, "frac_of_burst": tflops / burst,
+                   "frac_of_sustained": tflops / sust, "peak_burst_tflops": burst,
+                   "peak_sustained_tflops": sust, "peak_source": f"{peak_src} bf16_tflops / "
+                                                                 "bf16_tflops_sustained"},
+        "gate_up_kernel": {"avg_launch_ms": gu_ms, "achieved_tflops": gu_tflops,
+                           "frac_of_burst": gu_tflops / burst if gu_tflops else None,
+                           "frac_of_sustained": gu_tflops / sust if gu_tflops else None},
+        "hbm": {"achieved_gbs": hbm, "frac": hbm / hbm_peak, "peak_gbs": hbm_peak,
+                "peak_source": f"{peak_src} hbm_gbs"},
+        "ideal_ms": {"tensor_burst": acc["flops"] / (burst * 1e12) * 1e3,
+                     "tensor_sustained": acc["flops"] / (sust * 1e12) * 1e3,
+                     "hbm": acc["weight_bytes"] / (hbm_peak * 1e9) * 1e3},
+        "clocks": clocks,
+        # ms x median SM MHz / 1000: the step in millions of SM cycles, so that a
+        # power-capped clock shows as a lower MHz at an unchanged cycle count
+        "sm_mcycles_per_step": ms * mhz / 1e3 if mhz else None,
+        "kernel_ms_per_step": {kk: v / max(n_calls, 1) for kk, v in kernel_ms.items()},
+    }
 
 
 # ------------------------------------------------------------------- oracle
@@ -408,16 +529,7 @@ def main(argv=None):
         raise SystemExit("device status not clean after warm-up")
     launches_per_step = moe.moe_last_launch_count()
 
-    # touched experts of this batch (our own route + permute kernels)
-    ws = torch.empty(moe.moe_workspace_size(T, d, E, k, I), dtype=torch.uint8, device=dev)
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    moe.moe_route(g["x"], g["w_router"], g["bias"], k, cfg.scale, idx, w, ws)
-    i32 = lambda n: torch.empty((n,), dtype=torch.int32, device=dev)
-    counts, offs, rtok, srow = i32(E), i32(E + 1), i32(T * k), i32(T * k)
-    moe.moe_permute(idx, E, counts, offs, rtok, srow, ws)
-    touched = int((counts > 0).sum().item())
-    del ws
+    touched = touched_experts(moe, cfg, g, dev)
 
     # ---------------------------------------------------------- timed region
     moe.moe_profile_begin(args.steps)
@@ -511,6 +623,22 @@ def main(argv=None):
         args.workload + {"fp8": "_fp8", "w8a8": "_w8a8", "w4a16": "_w4a16"}.get(args.weights, ""),
         kname)
 
+    # ------------------------------------------------ other full-size workloads
+    # The default run (the decode headline in bf16) also times the prefill, the
+    # skewed and the DeepSeek-V3-shaped batch, one GPU, same process, after the
+    # headline's timed region; each has its own steps, clocks and roofline.
+    extra = None
+    if (world == 1 and not args.no_extra and args.workload == "k2_decode" and not args.set
+            and args.weights == "bf16"):
+        extra = {"note": "same process, after the headline; weights: the decode run's 384 "
+                         "experts (the first 256 for v3), x and bias drawn per workload"}
+        for i, name in enumerate(EXTRA_WORKLOADS):
+            cfg2, inp = extra_inputs(name, g, dev, seed=1000 + i)
+            extra[name] = time_extra_workload(moe, cfg2, inp, dev, args.warmup, peaks, peak_src,
+                                              local_rank)
+            del inp
+        torch.cuda.synchronize(dev)
+
     # ---------------------------------------------------------- CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -538,6 +666,8 @@ def main(argv=None):
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
             "kernel_ms_per_step": {kk: v / max(n_calls, 1) for kk, v in kernel_ms.items()},
         }
+        if extra is not None:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

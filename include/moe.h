@@ -187,9 +187,11 @@ int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const floa
  *     call returns MOE_ERR_UNSUPPORTED_SHAPE before launching anything.  With
  *     K2 shapes (d = 7168, E = 384, k = 8, inter = 2048) that allows up to
  *     T = 97 tokens; decode batches fit, prefill batches do not.
- *   - First call on a device: it looks up the array's device address with
- *     cudaGetSymbolAddress, with that device current.  Make that first call
- *     before any stream capture begins.
+ *   - First call in a CUDA context: it looks up the array's device address
+ *     with cudaGetSymbolAddress, in the context current on the calling thread,
+ *     and caches it under that context's unique id (a non-primary context, or
+ *     a context made after cudaDeviceReset, gets a lookup of its own).  Make
+ *     that first call before any stream capture begins.
  *   - Sharing: every call on every stream of a device uses the same array, and
  *     the array keeps the previous call's contents.  No kernel reads scratch it
  *     has not written earlier in the same call, so nothing needs clearing.

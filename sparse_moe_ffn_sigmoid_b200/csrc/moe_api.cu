@@ -809,24 +809,60 @@ int owned_workspace(cudaStream_t st, size_t need, void** out) {
     return MOE_OK;
 }
 
-// Device address of g_moe_noalloc_scratch on the current device, looked up on
-// the first call per device (with that device current) and cached.
+// Device address of g_moe_noalloc_scratch in the current CUDA context.  A
+// __device__ array has its own address in every context that loads the
+// library, so the address is looked up once per context (with that context
+// current) and cached under the context's unique id (cuCtxGetId: ids are never
+// reused in a process, so a context created after cudaDeviceReset, or a
+// non-primary context of the same device, gets its own lookup).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void* ptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
+std::vector<NoallocEntry> g_noalloc;
+
+bool current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 int noalloc_scratch(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_moe_noalloc_scratch) != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return MOE_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = p;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (have_id)
+        for (const NoallocEntry& e : g_noalloc)
+            if (e.ctx_id == id) {
+                *out = e.ptr;
+                return MOE_OK;
+            }
+    // the lookup also makes the device's primary context current when no
+    // context was yet (then the id is read after it)
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[dev];
+    if (have_id || current_context_id(&id)) g_noalloc.push_back({id, p});
+    *out = p;
     return MOE_OK;
 }
 

@@ -35,6 +35,7 @@ int main(void) {
     if (moe_layer_forward(dummy, dummy, (const float*)dummy, dummy, dummy, dummy, dummy,
                           0, 7168, 384, 8, 2048, 2.827f, dummy, NULL) != MOE_OK)
         return 7;
+    printf("noalloc scratch bytes %lu\n", (unsigned long)MOE_NOALLOC_SCRATCH_BYTES);
     printf("c abi ok\n");
     return 0;
 }
@@ -53,3 +54,6 @@ def test_header_is_c99_and_links(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
     assert "c abi ok" in out.stdout
+    # the binding's copy of the scratch array's size is the header's macro
+    line = [ln for ln in out.stdout.splitlines() if ln.startswith("noalloc scratch bytes")][0]
+    assert int(line.split()[-1]) == moe.NOALLOC_SCRATCH_BYTES

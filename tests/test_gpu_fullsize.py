@@ -55,18 +55,18 @@ def test_fullsize_layer(moe, name):
     assert np.array_equal(dr.cpu().numpy(), row_token)
     assert np.array_equal(ds.cpu().numpy(), slot_row)
 
-    # sampled output rows
-    busiest = int(np.argmax(counts))
-    first_of_busiest = int(row_token[offsets[busiest]])
-    sample = sorted({0, T // 2, T - 1, first_of_busiest} - set(np.nonzero(gap < PR.TIE_EPS)[0]))
-    need = sorted(set(ridx[sample].reshape(-1).tolist()))
-    egu = [None] * E
-    edn = [None] * E
-    for e in need:
-        egu[e] = g["w_gate_up"][e].cpu()
-        edn[e] = g["w_down"][e].cpu()
-    ref = oracle.moe_rows(x_h, ridx, rw, egu, edn, g["ws_gate_up"].cpu(), g["ws_down"].cpu(),
-                          tokens=np.array(sample, np.int32))
+    # output rows at the tiles' edges: the busiest expert's last two token
+    # tiles, the shared expert's last tile, a ragged multi-tile expert's last
+    # tile, element by element against the oracle (one batch of experts on the
+    # host at a time)
+    sample, parts = PR.wide_sample(ridx, gap, E, T, k)
+    print(f"{name}: {len(sample)} rows compared: {parts}")
+    assert len(sample) >= min(T, 128) - 8, parts
+    ref = PR.oracle_rows_by_expert(
+        x_h, ridx, rw, sample,
+        load_expert=lambda e: (PR.u16(g["w_gate_up"][e]), PR.u16(g["w_down"][e])),
+        load_shared=lambda: (PR.u16(g["ws_gate_up"]), PR.u16(g["ws_down"])),
+        row_fn=lambda xr, wts: oracle.swiglu_row(xr, *wts))
     got = PR.bf16_np(out[torch.tensor(sample, device="cuda")])
     PR.check_output(got, ref)
     del g, out, ws

@@ -135,9 +135,12 @@ FULL = ["k2_decode", "k2_prefill", "k2_skew", "v3"]
 
 @pytest.mark.parametrize("name", FULL)
 def test_w4a16_fullsize(moe, name):
-    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration,
-    sampled rows (token 0, T/2, T-1, the busiest expert's first token); the
-    sampled experts' GPU codes and scales equal the oracle quantizer's."""
+    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration: the
+    output rows at the GEMM tiles' ends (the last 64 rows of the busiest
+    expert's segment, of the shared expert's last tile and of a ragged
+    multi-tile expert's last tile) against the oracle with its own INT4
+    quantizer; the GPU codes and scales of every expert those rows select equal
+    the oracle quantizer's."""
     cfg = CONFIGS[name]
     T, d, E, k, I = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter
     g = make_inputs(cfg, seed=0, device="cuda")
@@ -146,21 +149,27 @@ def test_w4a16_fullsize(moe, name):
     assert moe.moe_device_status() == 0
     x_h = g["x"].cpu()
     ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
-    counts, offsets, row_token, _ = oracle.permute(ridx, E)
-    first_of_busiest = int(row_token[offsets[int(np.argmax(counts))]])
-    sample = sorted({0, T // 2, T - 1, first_of_busiest} - set(np.nonzero(gap < PR.TIE_EPS)[0]))
-    need = sorted(set(ridx[sample].reshape(-1).tolist()))
-    egu = [None] * E
-    edn = [None] * E
-    sgu_h = sgu.cpu().view(torch.int16).numpy().view(np.uint16)
-    for e in need:
+    # each tile part's last 64 rows (the tiles' ends): the oracle's FP8 / INT4
+    # rows cost more than bf16 ones
+    sample, parts = PR.wide_sample(ridx, gap, E, T, k, tail=64)
+    print(f"{name}: {len(sample)} rows compared: {parts}")
+    assert len(sample) >= min(T, 128) - 8, parts
+    sgu_h = PR.u16(sgu)
+    sdn_h = PR.u16(sdn)
+
+    def load_expert(e):
         q, sc = oracle.quantize_int4(_u16(g["w_gate_up"][e]))
-        assert np.array_equal(qgu[e].cpu().numpy(), pack_codes(q))
-        assert np.array_equal(sgu_h[:, e * 2 * I:(e + 1) * 2 * I], sc.T)
-        egu[e] = oracle.dequantize_int4(q, sc)
-        edn[e] = oracle.dequantize_int4(*oracle.quantize_int4(_u16(g["w_down"][e])))
-    ref = oracle.moe_rows(x_h, ridx, rw, egu, edn, g["ws_gate_up"].cpu(), g["ws_down"].cpu(),
-                          tokens=np.array(sample, np.int32))
+        assert np.array_equal(qgu[e].cpu().numpy(), pack_codes(q)), f"expert {e} codes"
+        assert np.array_equal(sgu_h[:, e * 2 * I:(e + 1) * 2 * I], sc.T), f"expert {e} scales"
+        qd, scd = oracle.quantize_int4(_u16(g["w_down"][e]))
+        assert np.array_equal(qdn[e].cpu().numpy(), pack_codes(qd)), f"expert {e} down codes"
+        assert np.array_equal(sdn_h[:, e * d:(e + 1) * d], scd.T), f"expert {e} down scales"
+        return oracle.dequantize_int4(q, sc), oracle.dequantize_int4(qd, scd)
+
+    ref = PR.oracle_rows_by_expert(
+        x_h, ridx, rw, sample, load_expert=load_expert,
+        load_shared=lambda: (PR.u16(g["ws_gate_up"]), PR.u16(g["ws_down"])),
+        row_fn=lambda xr, wts: oracle.swiglu_row(xr, *wts))
     PR.check_output(PR.bf16_np(out[torch.tensor(sample, device="cuda")]), ref)
     del g, qgu, qdn, out
     torch.cuda.empty_cache()

@@ -143,8 +143,12 @@ def _sample_tokens(ridx, gap, E, T):
 
 @pytest.mark.parametrize("name", FULL)
 def test_w8a8_fullsize(moe, name):
-    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration,
-    sampled rows; the sampled experts' GPU codes equal the oracle quantizer's."""
+    """Full K2 / DeepSeek-V3 shapes in the benchmark's launch configuration: the
+    output rows at the GEMM tiles' ends (the last 64 rows of the busiest
+    expert's segment, of the shared expert's last tile and of a ragged
+    multi-tile expert's last tile) against the oracle with its own row
+    quantizer; the GPU codes and exponents of every expert those rows select
+    equal the oracle quantizer's."""
     cfg = CONFIGS[name]
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     g = make_inputs(cfg, seed=0, device="cuda")
@@ -155,18 +159,24 @@ def test_w8a8_fullsize(moe, name):
     assert moe.moe_device_status() == 0
     x_h = g["x"].cpu()
     ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
-    sample = _sample_tokens(ridx, gap, E, T)
-    need = sorted(set(ridx[sample].reshape(-1).tolist()))
-    host = {"w_gate_up": {e: g["w_gate_up"][e].cpu() for e in need},
-            "w_down": {e: g["w_down"][e].cpu() for e in need},
-            "ws_gate_up": g["ws_gate_up"].cpu(), "ws_down": g["ws_down"].cpu()}
-    qe, qs = oracle.quantize_expert_rows(host, need)
-    for e in need:
-        assert np.array_equal(wq[0][e].cpu().numpy(), qe[e][0])
-        assert np.array_equal(wq[1][e].cpu().numpy(), qe[e][1])
-        assert np.array_equal(wq[3][e].cpu().numpy(), qe[e][3])
-    ref = oracle.moe_rows_fp8(x_h, ridx, rw, [qe.get(e) for e in range(E)], qs,
-                              tokens=np.array(sample, np.int32))
+    # each tile part's last 64 rows (the tiles' ends): the oracle's FP8 / INT4
+    # rows cost more than bf16 ones
+    sample, parts = PR.wide_sample(ridx, gap, E, T, k, tail=64)
+    print(f"{name}: {len(sample)} rows compared: {parts}")
+    assert len(sample) >= min(T, 128) - 8, parts
+
+    def load_expert(e):
+        q = oracle.quantize_fp8_rows(PR.u16(g["w_gate_up"][e])) + \
+            oracle.quantize_fp8_rows(PR.u16(g["w_down"][e]))
+        for got, want in zip((wq[0][e], wq[1][e], wq[2][e], wq[3][e]), q):
+            assert np.array_equal(got.cpu().numpy(), want), f"expert {e} codes"
+        return q
+
+    ref = PR.oracle_rows_by_expert(
+        x_h, ridx, rw, sample, load_expert=load_expert,
+        load_shared=lambda: oracle.quantize_fp8_rows(PR.u16(g["ws_gate_up"])) +
+        oracle.quantize_fp8_rows(PR.u16(g["ws_down"])),
+        row_fn=lambda xr, q: oracle.swiglu_row_fp8(xr, *q))
     PR.check_output(PR.bf16_np(out[torch.tensor(sample, device="cuda")]), ref)
     del g, wq, out
     torch.cuda.empty_cache()

@@ -68,13 +68,61 @@ def test_noalloc_size_limit(moe):
     fits = max(T for T in range(1, 200)
                if moe.moe_workspace_size(T, cfg.d, cfg.E, cfg.k, cfg.inter) <= limit)
     assert fits >= cfg.T            # the K2 decode batch fits
-    g = make_inputs(cfg.__class__(**{**cfg.as_dict(), "T": fits + 1}), seed=13, device="cuda")
+    # one weight set; only the token rows change with T
+    g = make_inputs(cfg, seed=13, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(14)
+    x_big = torch.randn((fits + 1, cfg.d), generator=gen, device="cuda").to(torch.bfloat16)
     out = torch.empty((fits + 1, cfg.d), dtype=torch.bfloat16, device="cuda")
     # one token more than the array holds: refused before any launch
-    assert _noalloc_raw(moe, g, g["x"], cfg, out) == -2      # MOE_ERR_UNSUPPORTED_SHAPE
-    # the largest batch that fits runs
-    out2 = torch.empty((fits, cfg.d), dtype=torch.bfloat16, device="cuda")
-    assert _noalloc_raw(moe, g, g["x"][:fits], cfg, out2) == 0
+    assert _noalloc_raw(moe, g, x_big, cfg, out) == -2      # MOE_ERR_UNSUPPORTED_SHAPE
+    # the largest batch that fits runs, and its scratch reaches the array's
+    # last bytes: compare it with the allocating entry point
+    x_fit = x_big[:fits].contiguous()
+    out2 = torch.full((fits, cfg.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc_raw(moe, g, x_fit, cfg, out2) == 0
+    ref = torch.empty((fits, cfg.d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward(x_fit, g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                          g["ws_gate_up"], g["ws_down"], cfg.k, cfg.scale, ref)
     torch.cuda.synchronize()
     assert moe.moe_device_status() == 0
-    assert torch.isfinite(out2.float()).all()
+    PR.check_output(PR.bf16_np(out2), PR.bf16_np(ref))
+
+
+def _pool_bytes():
+    """(used, reserved) bytes of the device's default CUDA memory pool, the pool
+    cudaMallocAsync draws from, or None without the cuda-python bindings."""
+    try:
+        from cuda.bindings import runtime as rt
+    except ImportError:
+        return None
+    err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
+    assert err == rt.cudaError_t.cudaSuccess, err
+    vals = []
+    for attr in (rt.cudaMemPoolAttr.cudaMemPoolAttrUsedMemCurrent,
+                 rt.cudaMemPoolAttr.cudaMemPoolAttrReservedMemCurrent):
+        err, v = rt.cudaMemPoolGetAttribute(pool, attr)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        vals.append(int(v))
+    return tuple(vals)
+
+
+def test_noalloc_allocates_nothing(moe):
+    """The point of the entry point: two calls on a stream the library has never
+    seen leave the device's free memory and the stream-ordered pool unchanged
+    (the allocating entry point would take a new scratch buffer for a new
+    stream)."""
+    cfg = CONFIGS["tiny"]
+    g = make_inputs(cfg, seed=15, device="cuda")
+    out = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc_raw(moe, g, g["x"], cfg, out) == 0      # warm-up (symbol lookup)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    free0 = torch.cuda.mem_get_info()[0]
+    pool0 = _pool_bytes()
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            assert _noalloc_raw(moe, g, g["x"], cfg, out) == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert _pool_bytes() == pool0
+    assert moe.moe_device_status() == 0
