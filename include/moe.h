@@ -49,6 +49,11 @@ typedef enum {
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(int status);
 
+/* What the last MOE_ERR_CUDA returned on the calling thread came from: the
+ * failing CUDA call or tensor-map encoding and its error (a thread-local string,
+ * valid until the thread's next failing call; "no error" before any). */
+const char* moe_last_error_string(void);
+
 /*
  * Bytes of device scratch that any staged call below needs for a layer of
  * this size (the largest of their needs).  Routing, permutation and expert
@@ -443,6 +448,74 @@ int moe_profile_end(float* total_ms, int max_kernels, int* n_calls);
 
 /* Name of kernel slot i of a layer call ("" if out of range). */
 const char* moe_kernel_name(int i);
+
+/*
+ * Expert parallelism ("K2 inference engineer's answer", 2.1: the deployment
+ * spreads the routed experts over many GPUs, EP = 128, two or three experts per
+ * rank for DeepSeek-V3 and about 10 GB of expert weights per rank for K2, with
+ * data parallelism over tokens; 2.4: n_group = 1, so any token may select any
+ * rank's experts).  R ranks; rank q owns the E_l = E / R routed experts
+ * [q E_l, (q + 1) E_l) (E a multiple of R); the router, the bias and the shared
+ * expert are replicated; every rank routes its own T tokens.  One layer call on
+ * every rank is:
+ *   1. moe_ep_dispatch: route, permute and gather the rank's token rows into
+ *      send_rows [T*k, d], expert-major (expert e's rows from offsets of
+ *      `counts`), so the rows for rank q are the contiguous block of experts
+ *      [q E_l, (q + 1) E_l);
+ *   2. the caller exchanges the per-expert counts ([R][E_l] ints, all-to-all)
+ *      and the rows (all-to-all with those splits), e.g. NCCL over NVLink;
+ *      the received rows are source-major: source 0's rows grouped by local
+ *      expert, then source 1's, ...;
+ *   3. moe_ep_expert_ffn: the rank's experts on the received rows, outputs in
+ *      the received order;
+ *   4. the caller returns the outputs to their sources (the reverse all-to-all);
+ *      each source gets back exactly its send_rows' order;
+ *   5. moe_ep_combine: the shared expert on the rank's own tokens plus
+ *      out[t] = y_shared[t] + sum_j topk_w[t, j] * y_back[slot_row[t*k + j]].
+ * Each row's arithmetic is that of moe_layer_forward (same kernels, same K
+ * order), so a rank's output equals moe_layer_forward on its own tokens bit
+ * for bit.  All pointers are device memory owned by the caller, every call is
+ * asynchronous on `stream`, errors as in moe_layer_forward; workspaces are sized
+ * by the matching *_workspace_size function (0 for unsupported shapes).
+ *
+ * moe_ep_dispatch: x [T, d], router and bias as in moe_route -> topk_idx [T, k],
+ * topk_w [T, k], counts [E] (rows per expert), slot_row [T*k] (as in
+ * moe_permute), send_rows [T*k, d] bf16.
+ */
+size_t moe_ep_dispatch_workspace_size(int T, int d, int E, int k);
+int moe_ep_dispatch(const uint16_t* x, const uint16_t* w_router, const float* bias, int T, int d,
+                    int E, int k, float scale, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                    int32_t* slot_row, uint16_t* send_rows, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * moe_ep_expert_ffn: recv_rows [rows, d] bf16 as received (source-major) with
+ * recv_counts [R, E_l] int32 (device; row counts per source and local expert,
+ * summing to `rows`; R * E_l <= 1024), the rank's experts' weights
+ * w_gate_up [E_l, 2*inter, d] and w_down [E_l, d, inter] (layouts of
+ * moe_layer_forward) -> y [rows, d] bf16, row i = its expert applied to
+ * received row i.  Inside: the rows are regrouped expert-major (expert e's rows
+ * from source 0, then source 1, ... each in its source's order), run through
+ * the grouped SwiGLU GEMMs and put back in the received order.  A count total
+ * other than `rows` is recorded in the device status word (MOE_ERR_INVALID_ARG)
+ * and y is all zeros.
+ */
+size_t moe_ep_expert_ffn_workspace_size(int rows, int d, int R, int E_local, int inter);
+int moe_ep_expert_ffn(const uint16_t* recv_rows, const int32_t* recv_counts, int rows, int d, int R,
+                      int E_local, int inter, const uint16_t* w_gate_up, const uint16_t* w_down,
+                      uint16_t* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_ep_combine: y_back [T*k, d] bf16 (the expert outputs of this rank's
+ * send_rows, in send_rows' order), x [T, d], the shared expert's ws_gate_up
+ * [2*inter, d] and ws_down [d, inter], topk_w and slot_row from
+ * moe_ep_dispatch -> out [T, d] bf16.
+ */
+size_t moe_ep_combine_workspace_size(int T, int d, int inter);
+int moe_ep_combine(const uint16_t* y_back, const uint16_t* x, const uint16_t* ws_gate_up,
+                   const uint16_t* ws_down, const float* topk_w, const int32_t* slot_row, int T,
+                   int d, int k, int inter, uint16_t* out, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 #ifdef __cplusplus
 }

@@ -16,7 +16,7 @@ import torch
 from . import build as _build
 
 __all__ = [
-    "MoeError", "lib", "moe_status_string", "moe_workspace_size", "moe_route", "moe_permute",
+    "MoeError", "lib", "moe_status_string", "moe_last_error_string", "moe_workspace_size", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_ws",
     "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
@@ -24,12 +24,15 @@ __all__ = [
     "moe_layer_forward_fp8_ws", "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
     "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
     "moe_layer_forward_w8a8_ws", "moe_quantize_int4", "moe_layer_forward_w4a16",
-    "moe_layer_forward_w4a16_ws", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "moe_layer_forward_w4a16_ws", "moe_ep_dispatch", "moe_ep_expert_ffn", "moe_ep_combine",
+    "moe_ep_dispatch_workspace_size", "moe_ep_expert_ffn_workspace_size",
+    "moe_ep_combine_workspace_size", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 # Every function declared in include/moe.h.
 EXPORTED_SYMBOLS = [
-    "moe_status_string", "moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn",
+    "moe_status_string", "moe_last_error_string", "moe_workspace_size", "moe_route",
+    "moe_permute", "moe_expert_ffn",
     "moe_combine", "moe_layer_forward", "moe_layer_forward_ws", "moe_device_status",
     "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
@@ -37,7 +40,9 @@ EXPORTED_SYMBOLS = [
     "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss", "moe_seq_aux_workspace_size",
     "moe_quantize_fp8_rows", "moe_workspace_size_w8a8", "moe_layer_forward_w8a8",
     "moe_layer_forward_w8a8_ws", "moe_quantize_int4", "moe_layer_forward_w4a16",
-    "moe_layer_forward_w4a16_ws",
+    "moe_layer_forward_w4a16_ws", "moe_ep_dispatch_workspace_size", "moe_ep_dispatch",
+    "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_ep_combine_workspace_size",
+    "moe_ep_combine",
 ]
 
 MOE_OK = 0
@@ -47,7 +52,8 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024    # MOE_NOALLOC_SCRATCH_BYTES in inclu
 class MoeError(RuntimeError):
     def __init__(self, fn: str, code: int):
         self.code = code
-        super().__init__(f"{fn} failed: {moe_status_string(code)} ({code})")
+        detail = f": {moe_last_error_string()}" if code == -3 else ""    # MOE_ERR_CUDA
+        super().__init__(f"{fn} failed: {moe_status_string(code)} ({code}){detail}")
 
 
 def _load():
@@ -57,6 +63,7 @@ def _load():
     SZ, U64, I64 = ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int64
     sig = {
         "moe_status_string": ([I], ctypes.c_char_p),
+        "moe_last_error_string": ([], ctypes.c_char_p),
         "moe_workspace_size": ([I, I, I, I, I], SZ),
         "moe_route": ([P, P, P, I, I, I, I, F, P, P, P, SZ, P], I),
         "moe_permute": ([P, I, I, I, P, P, P, P, P, SZ, P], I),
@@ -87,6 +94,12 @@ def _load():
         "moe_workspace_size_w8a8": ([I, I, I, I, I], SZ),
         "moe_layer_forward_w8a8": ([P] * 11 + [I, I, I, I, I, F, P, P], I),
         "moe_layer_forward_w8a8_ws": ([P] * 11 + [I, I, I, I, I, F, P, P, SZ, P], I),
+        "moe_ep_dispatch_workspace_size": ([I, I, I, I], SZ),
+        "moe_ep_dispatch": ([P, P, P, I, I, I, I, F, P, P, P, P, P, P, SZ, P], I),
+        "moe_ep_expert_ffn_workspace_size": ([I, I, I, I, I], SZ),
+        "moe_ep_expert_ffn": ([P, P, I, I, I, I, I, P, P, P, P, SZ, P], I),
+        "moe_ep_combine_workspace_size": ([I, I, I], SZ),
+        "moe_ep_combine": ([P] * 6 + [I, I, I, I, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -137,6 +150,10 @@ BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
 
 def moe_status_string(code: int) -> str:
     return _LIB.moe_status_string(int(code)).decode()
+
+
+def moe_last_error_string() -> str:
+    return _LIB.moe_last_error_string().decode()
 
 
 def moe_workspace_size(T: int, d: int, E: int, k: int, inter: int) -> int:
@@ -465,3 +482,57 @@ def moe_profile_end():
 
 def moe_kernel_name(i: int) -> str:
     return _LIB.moe_kernel_name(int(i)).decode()
+
+
+# ------------------------------------------------------ expert parallelism
+
+def moe_ep_dispatch_workspace_size(T: int, d: int, E: int, k: int) -> int:
+    return int(_LIB.moe_ep_dispatch_workspace_size(T, d, E, k))
+
+
+def moe_ep_dispatch(x, w_router, bias, k: int, scale: float, topk_idx, topk_w, counts, slot_row,
+                    send_rows, workspace, stream=None):
+    T, d = x.shape
+    E = w_router.shape[0]
+    rc = _LIB.moe_ep_dispatch(_ptr(x, BF16, "x"), _ptr(w_router, BF16, "w_router"),
+                              _ptr(bias, F32, "bias"), T, d, E, k, float(scale),
+                              _ptr(topk_idx, I32, "topk_idx"), _ptr(topk_w, F32, "topk_w"),
+                              _ptr(counts, I32, "counts"), _ptr(slot_row, I32, "slot_row"),
+                              _ptr(send_rows, BF16, "send_rows"),
+                              _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                              _stream(stream))
+    _check("moe_ep_dispatch", rc)
+
+
+def moe_ep_expert_ffn_workspace_size(rows: int, d: int, R: int, E_local: int, inter: int) -> int:
+    return int(_LIB.moe_ep_expert_ffn_workspace_size(rows, d, R, E_local, inter))
+
+
+def moe_ep_expert_ffn(recv_rows, recv_counts, w_gate_up, w_down, y, workspace, stream=None):
+    rows, d = recv_rows.shape
+    R, E_local = recv_counts.shape
+    inter = w_gate_up.shape[1] // 2
+    rc = _LIB.moe_ep_expert_ffn(_ptr(recv_rows, BF16, "recv_rows"),
+                                _ptr(recv_counts, I32, "recv_counts"), rows, d, R, E_local, inter,
+                                _ptr(w_gate_up, BF16, "w_gate_up"), _ptr(w_down, BF16, "w_down"),
+                                _ptr(y, BF16, "y"), _ptr(workspace, torch.uint8, "workspace"),
+                                workspace.numel(), _stream(stream))
+    _check("moe_ep_expert_ffn", rc)
+
+
+def moe_ep_combine_workspace_size(T: int, d: int, inter: int) -> int:
+    return int(_LIB.moe_ep_combine_workspace_size(T, d, inter))
+
+
+def moe_ep_combine(y_back, x, ws_gate_up, ws_down, topk_w, slot_row, out, workspace,
+                   stream=None):
+    T, d = x.shape
+    k = topk_w.shape[1]
+    inter = ws_gate_up.shape[0] // 2
+    rc = _LIB.moe_ep_combine(_ptr(y_back, BF16, "y_back"), _ptr(x, BF16, "x"),
+                             _ptr(ws_gate_up, BF16, "ws_gate_up"), _ptr(ws_down, BF16, "ws_down"),
+                             _ptr(topk_w, F32, "topk_w"), _ptr(slot_row, I32, "slot_row"), T, d, k,
+                             inter, _ptr(out, BF16, "out"),
+                             _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                             _stream(stream))
+    _check("moe_ep_combine", rc)

@@ -138,20 +138,27 @@ struct __align__(64) GemmArgs {
     const int8_t* b_exp[2];
 };
 
+// Tile i of a grouped tile list.
+__device__ __forceinline__ Tile tile_at(const int4* tiles, int i) {
+    Tile t;
+    const int4 v0 = tiles[2 * i];
+    const int4 v1 = tiles[2 * i + 1];
+    t.a_row0 = v0.x;
+    t.a_row1 = v0.y;
+    t.b_row0 = v0.z;
+    t.n = v0.w & 0xFFFF;
+    t.map = (v0.w >> 16) & 1;
+    t.out_row0 = v1.x;
+    t.out_col0 = v1.y;
+    t.ks0 = v1.z;
+    t.ks1 = v1.w;
+    return t;
+}
+
 __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int i) {
     Tile t;
     if (a.tiles != nullptr) {
-        const int4 v0 = a.tiles[2 * i];
-        const int4 v1 = a.tiles[2 * i + 1];
-        t.a_row0 = v0.x;
-        t.a_row1 = v0.y;
-        t.b_row0 = v0.z;
-        t.n = v0.w & 0xFFFF;
-        t.map = (v0.w >> 16) & 1;
-        t.out_row0 = v1.x;
-        t.out_col0 = v1.y;
-        t.ks0 = v1.z;
-        t.ks1 = v1.w;
+        t = tile_at(a.tiles, i);
     } else {
         const int m = i % a.dense_mslabs;
         const int r = i / a.dense_mslabs;

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -17,7 +18,9 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemv.cuh"
 #include "balance.cuh"
+#include "ep.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -44,6 +47,20 @@ constexpr int kTokenMajorMinT = 1024;
 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 std::atomic<int> g_last_launches{0};
+
+// The last CUDA failure this thread met inside the library (moe_last_error_string).
+thread_local char t_last_error[256] = "no error";
+
+int record_cuda_failure(const char* where, const char* what) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "%s: %s", where, what);
+    return MOE_ERR_CUDA;
+}
+
+// MOE_OK, or MOE_ERR_CUDA with the launch error recorded, after kernel launches.
+int launch_rc(const char* where) {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : record_cuda_failure(where, cudaGetErrorString(e));
+}
 
 // Kernels of one layer call, in launch order (moe_kernel_name).  gather_rows
 // also quantizes the rows in FP8 compute; quantize_h (the activation rows'
@@ -74,6 +91,8 @@ struct Recorder {
         ++launches;
         skip(st);
     }
+    // a kernel launched inside a slot that a later mark() closes
+    void count() { ++launches; }
     // a slot this call has no kernel for (it times as zero)
     void skip(cudaStream_t st) {
         ++n;
@@ -151,9 +170,21 @@ int tile_rows(int T, int E, int k) {
     return (T > kTileN && static_cast<long long>(T) * k <= 64ll * E) ? 192 : kTileN;
 }
 
+// Decode-sized batches with INT4 or E4M3 routed weights run the register-
+// dequantizing GEMMs of gemv.cuh (token tiles of 16 rows) when the routed experts
+// average at most 4 rows and both contraction lengths are multiples of the
+// format's step (256 for INT4, 128 for E4M3).
+bool gemv_shape(int T, int E, int k) { return static_cast<long long>(T) * k <= 4ll * E; }
+
+bool gemv_ok(int T, int d, int E, int k, int inter, bool int4) {
+    const int step = gemv_step_k(int4 ? kGemvInt4 : kGemvFp8);
+    return gemv_shape(T, E, k) && d % step == 0 && inter % step == 0;
+}
+
 Layout make_layout(int T, int d, int E, int k, int inter, bool fp8_compute = false) {
     Layout L{};
-    const int tn = tile_rows(T, E, k);
+    // tile lists sized for the smallest token tiles any plan of this shape uses
+    const int tn = gemv_shape(T, E, k) ? kGemvTileN : tile_rows(T, E, k);
     const size_t Tk = static_cast<size_t>(T) * k;
     const size_t rows = Tk + T;   // routed rows, then the shared expert's rows
     L.splits = router_splits(T, d, E);
@@ -201,14 +232,42 @@ struct DeviceInfo {
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// Makes sure the calling thread has a current CUDA context before the
+// library's driver calls (tensor-map encoding needs one): a thread whose first
+// CUDA work is a call into this library may have none yet, and then the
+// device's primary context is made current, as the runtime would on its first
+// kernel launch.  A context the caller made current is left alone.
+int bind_context(int dev) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    if (get_current == nullptr) return record_cuda_failure("cuCtxGetCurrent", "entry point not found");
+    if (get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr) return MOE_OK;
+    const cudaError_t e = cudaSetDevice(dev);
+    return e == cudaSuccess ? MOE_OK : record_cuda_failure("cudaSetDevice", cudaGetErrorString(e));
+}
+
 int device_info(DeviceInfo* out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return record_cuda_failure("cudaGetDevice", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return record_cuda_failure("cudaGetDevice", "device index >= 64");
+    const int brc = bind_context(dev);
+    if (brc != MOE_OK) return brc;
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DeviceInfo& di = g_dev[dev];
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return MOE_ERR_CUDA;
+            return launch_rc("cudaDeviceGetAttribute");
         const int smem = static_cast<int>(kMaxDynSmem);
         const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
         if (cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsBF16>, dyn, smem) != cudaSuccess ||
@@ -225,8 +284,20 @@ int device_info(DeviceInfo* out) {
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiSwiGLU, kOpsFP8>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(moe_gemm_kernel<kEpiStoreBF16, kOpsFP8>, dyn, smem) != cudaSuccess ||
             cudaFuncSetAttribute(scan_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kScanSmem)) != cudaSuccess)
-            return MOE_ERR_CUDA;
+                                 static_cast<int>(kScanSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>, dyn,
+                                 gemv_smem_bytes(kGemvInt4)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>, dyn,
+                                 gemv_smem_bytes(kGemvInt4)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>, dyn,
+                                 gemv_smem_bytes(kGemvFp8)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>, dyn,
+                                 gemv_smem_bytes(kGemvFp8)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, dyn,
+                                 gemv_smem_bytes(kGemvBF16)) != cudaSuccess ||
+            cudaFuncSetAttribute(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, dyn,
+                                 gemv_smem_bytes(kGemvBF16)) != cudaSuccess)
+            return launch_rc("cudaFuncSetAttribute");
         di.ready = true;
     }
     *out = di;
@@ -240,8 +311,26 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn g_encode_driver = nullptr;
+
+// cuTensorMapEncodeTiled, recording a failure for moe_last_error_string.
+CUresult encode_recording(CUtensorMap* m, CUtensorMapDataType type, cuuint32_t rank, void* base,
+                          const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                          const cuuint32_t* estr, CUtensorMapInterleave il, CUtensorMapSwizzle sw,
+                          CUtensorMapL2promotion l2, CUtensorMapFloatOOBfill oob) {
+    const CUresult r = g_encode_driver(m, type, rank, base, dims, strides, box, estr, il, sw, l2, oob);
+    if (r != CUDA_SUCCESS) {
+        char what[192];
+        std::snprintf(what, sizeof(what), "CUresult %d (base %p, dims %llu x %llu, box %u x %u)",
+                      static_cast<int>(r), base, static_cast<unsigned long long>(dims[0]),
+                      static_cast<unsigned long long>(rank > 1 ? dims[1] : 1), box[0],
+                      rank > 1 ? box[1] : 1u);
+        record_cuda_failure("cuTensorMapEncodeTiled", what);
+    }
+    return r;
+}
+
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
         void* p = nullptr;
@@ -249,9 +338,13 @@ EncodeTiledFn encode_fn() {
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
+            g_encode_driver = reinterpret_cast<EncodeTiledFn>(p);
     });
-    return fn;
+    if (g_encode_driver == nullptr) {
+        record_cuda_failure("cuTensorMapEncodeTiled", "driver entry point not found");
+        return nullptr;
+    }
+    return encode_recording;
 }
 
 // Row-major E4M3 code matrix [rows, cols] (uint8) read in boxes of 128 rows x
@@ -326,6 +419,46 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Maps of the decode-sized GEMMs (gemv.cuh): weight rows in boxes of 128 bytes x
+// 16 rows with the 128-byte swizzle, as uint8 codes [rows, row_bytes] or bf16
+// [rows, cols]; INT4 group scales [cols / 32, rows] bf16 in boxes of 16 rows x
+// 8 groups (one 256-element step), unswizzled.
+bool make_map_gemv_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemvRowBytes), 16};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_gemv_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * sizeof(bf16)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemvRowBytes / sizeof(bf16)), 16};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_gemv_scales(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {rows, cols / kInt4Group};
+    const cuuint64_t strides[1] = {rows * sizeof(bf16)};
+    const cuuint32_t box[2] = {16, static_cast<cuuint32_t>(gemv_step_k(kGemvInt4) / kInt4Group)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ----------------------------------------------------------------- launches
 
 // Ring depths: the token ring gets 3 slots (2 for tiles of <= 64 tokens, whose
@@ -370,7 +503,7 @@ int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
                                         FP8A ? a.stages_a8 : 0, code_slab_bytes(OPS));
     if (smem > kMaxDynSmem || (FP8A && a.stages_a8 < 2)) return MOE_ERR_UNSUPPORTED_SHAPE;
     moe_gemm_kernel<EPI, OPS><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 // Router GEMM: fp32 logit partials [splits, T, E] (split-K over d).
@@ -431,7 +564,7 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
     else MOE_TOPK(32);
 #undef MOE_TOPK
     rec.mark(st);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offsets, int* row_token,
@@ -448,7 +581,7 @@ int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offset
     permute_scatter_kernel<<<nblk, kPermTokens, 8 * E * sizeof(uint32_t), st>>>(
         idx, T, E, k, blk, row_token, slot_row);
     rec.mark(st);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 // Routed experts' weights stored as E4M3 codes with one int8 exponent per
@@ -481,8 +614,9 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
                bf16* y, const int4* tiles1, const int4* tiles2, const int* ntiles,
                int max_tiles1, int max_tiles2, cudaStream_t st, Recorder& rec,
                const Fp8Experts* f8 = nullptr, const Int4Experts* i4 = nullptr,
-               int tile_n = kTileN) {
+               int tile_n = kTileN, bool use_gemv = false) {
     if ((f8 != nullptr || i4 != nullptr) && !shared) return MOE_ERR_INVALID_ARG;
+    if (use_gemv && i4 == nullptr && f8 == nullptr) return MOE_ERR_INVALID_ARG;
     const int rows_routed = T * k;
     const int rows_all = rows_routed + (shared ? T : 0);
     if (rows_routed > 0) {
@@ -494,6 +628,74 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
                                                                       d, xperm);
         rec.mark(st);
     }
+    if (use_gemv) {
+        // register-dequantizing GEMMs (gemv.cuh) over the plan's 16-row token
+        // tiles: the routed experts' tiles (INT4 or E4M3 codes), then the shared
+        // expert's (bf16), whose tile range starts at ntiles[2] / ntiles[3]
+        const int shared_tiles1 = ((T + kGemvTileN - 1) / kGemvTileN) * (inter / kSlabRows);
+        const int shared_tiles2 = ((T + kGemvTileN - 1) / kGemvTileN) * (d / (2 * kSlabRows));
+        const int wf = i4 ? kGemvInt4 : kGemvFp8;
+        const int grid_r = kGemvCtasPerSm * di.sms;
+        for (int gemm = 0; gemm < 2; ++gemm) {
+            const bool gu = (gemm == 0);
+            const uint64_t rows = gu ? static_cast<uint64_t>(E) * 2 * inter
+                                     : static_cast<uint64_t>(E) * d;
+            const int K = gu ? d : inter;
+            GemvArgs v{};
+            v.tiles = gu ? tiles1 : tiles2;
+            v.first = nullptr;
+            v.last = ntiles + (gu ? 2 : 3);
+            v.exps = i4 ? nullptr : (gu ? f8->gate_up_exp : f8->down_exp);
+            v.b[0] = gu ? (rows_routed > 0 ? xperm : x) : h;
+            v.b[1] = gu ? x : h;
+            v.out = gu ? h : y;
+            v.out_ld = gu ? inter : d;
+            v.K = K;
+            v.col_limit = gu ? inter : d;
+            v.timeout_ns = g_timeout_ns.load();
+            // routed tiles: codes (and INT4 scales)
+            const bool maps_ok =
+                i4 ? make_map_gemv_u8(&v.a_map, gu ? i4->gate_up : i4->down, rows, K / 2) &&
+                         make_map_gemv_scales(&v.s_map, gu ? i4->gate_up_scale : i4->down_scale,
+                                              rows, K)
+                   : make_map_gemv_u8(&v.a_map, gu ? f8->gate_up : f8->down, rows, K);
+            if (!maps_ok) return record_cuda_failure(__func__, "tensor map encoding failed");
+            const int grid1 = std::max(1, std::min(gu ? max_tiles1 : max_tiles2, grid_r));
+            if (wf == kGemvInt4) {
+                if (gu)
+                    moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>
+                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st>>>(v);
+                else
+                    moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>
+                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st>>>(v);
+            } else {
+                if (gu)
+                    moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>
+                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st>>>(v);
+                else
+                    moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>
+                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st>>>(v);
+            }
+            rec.count();
+            // the shared expert's tiles: bf16 weights
+            if (!make_map_gemv_bf16(&v.a_map, gu ? ws_gate_up : ws_down, gu ? 2ull * inter : d, K))
+                return MOE_ERR_CUDA;
+            v.first = ntiles + (gu ? 2 : 3);
+            v.last = ntiles + (gu ? 0 : 1);
+            const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_r));
+            if (gu)
+                moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>
+                    <<<grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st>>>(v);
+            else
+                moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>
+                    <<<grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st>>>(v);
+            if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
+            rec.mark(st);
+            if (gu) rec.skip(st);   // no activation quantization
+        }
+        return MOE_OK;
+    }
+
     // largest token tile: an expert never holds more rows than its token count
     const int max_rows = shared ? T : rows_routed;
     const int n_max = std::min(tile_n, (max_rows + 15) & ~15);
@@ -687,7 +889,7 @@ int launch_ffn_fp8(const DeviceInfo& di, const bf16* x, const int* row_token,
     rc = launch_gemm<kEpiStoreBF16, kOpsFP8>(g2, std::min(max_tiles2, di.sms), st);
     if (rc != MOE_OK) return rc;
     rec.mark(st);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* slot_row, int T,
@@ -698,7 +900,7 @@ int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* sl
     combine_kernel<<<grid, kCombineThreads, 0, st>>>(y, ysh, w, slot_row, T, d, k,
                                                      static_cast<long long>(T) * k, out);
     rec.mark(st);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
@@ -749,7 +951,8 @@ int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* 
     if (rc != MOE_OK) return rc;
     PlanArgs plan{E, 1, T, d, inter, T * k, tiles1, tiles2, ntiles};
     if (f8c != nullptr) plan.kstep = 2 * kBK;
-    plan.tile_n = tile_rows(T, E, k);
+    const bool use_gemv = (i4 != nullptr || f8 != nullptr) && gemv_ok(T, d, E, k, inter, i4 != nullptr);
+    plan.tile_n = use_gemv ? kGemvTileN : tile_rows(T, E, k);
     rc = launch_permute(idx, T, E, k, counts, offsets, row_token, slot_row,
                         reinterpret_cast<int*>(P(L.blk)), plan, st, rec);
     if (rc != MOE_OK) return rc;
@@ -762,7 +965,7 @@ int layer_forward(const bf16* x, const bf16* wr, const float* bias, const bf16* 
         rc = launch_ffn(di, x, row_token, slot_row, T, d, E, k, inter, wgu, wdn, sgu, sdn, true,
                         xperm, h,
                         y, tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec, f8, i4,
-                        plan.tile_n);
+                        plan.tile_n, use_gemv);
     if (rc != MOE_OK) return rc;
     rc = launch_combine(y, y + static_cast<size_t>(T) * k * d, w, slot_row, T, d, k, out, st, rec);
     g_last_launches.store(rec.launches);
@@ -815,7 +1018,6 @@ int owned_workspace(cudaStream_t st, size_t need, void** out) {
 // current) and cached under the context's unique id (cuCtxGetId: ids are never
 // reused in a process, so a context created after cudaDeviceReset, or a
 // non-primary context of the same device, gets its own lookup).
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
 using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
 struct NoallocEntry {
@@ -864,6 +1066,83 @@ int noalloc_scratch(void** out) {
     if (have_id || current_context_id(&id)) g_noalloc.push_back({id, p});
     *out = p;
     return MOE_OK;
+}
+
+// ------------------------------------------------------ expert parallelism
+
+// Scratch of moe_ep_dispatch: router partials, permutation block counts,
+// expert offsets and the permuted rows' tokens.
+struct EpDispatchLayout {
+    size_t partials, blk, offsets, row_token, total;
+    int splits;
+};
+
+EpDispatchLayout ep_dispatch_layout(int T, int d, int E, int k) {
+    EpDispatchLayout L{};
+    L.splits = router_splits(T, d, E);
+    const int nblk = (T + kPermTokens - 1) / kPermTokens;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.partials = take(static_cast<size_t>(L.splits) * T * E * sizeof(float));
+    L.blk = take(static_cast<size_t>(std::max(nblk, 1)) * E * sizeof(int));
+    L.offsets = take(static_cast<size_t>(E + 2) * sizeof(int));
+    L.row_token = take(static_cast<size_t>(T) * k * sizeof(int));
+    L.total = off;
+    return L;
+}
+
+// Scratch of moe_ep_expert_ffn: the receive maps and expert offsets, then the
+// grouped FFN's scratch (the layout of `rows` tokens, E_l experts, k = 1).
+struct EpFfnLayout {
+    size_t exp_offsets, src_of_exp, exp_of_src, ffn, total;
+    Layout F;
+};
+
+EpFfnLayout ep_ffn_layout(int rows, int d, int El, int inter) {
+    EpFfnLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.exp_offsets = take(static_cast<size_t>(El + 2) * sizeof(int));
+    L.src_of_exp = take(static_cast<size_t>(rows) * sizeof(int));
+    L.exp_of_src = take(static_cast<size_t>(rows) * sizeof(int));
+    L.ffn = off;
+    L.F = make_layout(rows, d, El, 1, inter);
+    L.total = L.ffn + L.F.total;
+    return L;
+}
+
+// Scratch of moe_ep_combine: the shared expert's tile lists, h and output rows.
+struct EpCombineLayout {
+    size_t tiles1, tiles2, ntiles, h, y, total;
+    int max_tiles1, max_tiles2;
+};
+
+EpCombineLayout ep_combine_layout(int T, int d, int inter) {
+    EpCombineLayout L{};
+    const int nt = (T + kTileN - 1) / kTileN;
+    L.max_tiles1 = nt * ((inter + kSlabRows - 1) / kSlabRows);
+    L.max_tiles2 = nt * ((d + 2 * kSlabRows - 1) / (2 * kSlabRows));
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.tiles1 = take(static_cast<size_t>(L.max_tiles1) * 2 * sizeof(int4));
+    L.tiles2 = take(static_cast<size_t>(L.max_tiles2) * 2 * sizeof(int4));
+    L.ntiles = take(4 * sizeof(int));
+    L.h = take(static_cast<size_t>(T) * inter * sizeof(bf16));
+    L.y = take(static_cast<size_t>(T) * d * sizeof(bf16));
+    L.total = off;
+    return L;
 }
 
 }  // namespace
@@ -949,7 +1228,7 @@ int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* o
     int* ntiles = reinterpret_cast<int*>(base + L.ntiles);
     PlanArgs plan{E, 0, T, d, inter, T * k, tiles1, tiles2, ntiles};
     plan_kernel<<<1, 1024, 0, st>>>(offsets, plan);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
     Recorder rec;
     return launch_ffn(di, reinterpret_cast<const bf16*>(x), row_token, nullptr, T, d, E, k, inter,
                       reinterpret_cast<const bf16*>(w_gate_up), reinterpret_cast<const bf16*>(w_down),
@@ -1044,7 +1323,7 @@ int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, 
     const dim3 grid(static_cast<unsigned>(rows / kQuantBlock), static_cast<unsigned>(cols / kQuantBlock));
     fp8_quantize_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const bf16*>(w), cols, q, exps);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
@@ -1102,7 +1381,7 @@ int moe_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* co
     int4_quantize_kernel<<<blocks, 32 * kInt4Warps, 0, static_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const bf16*>(w), rows, static_cast<int>(cols),
         reinterpret_cast<uint32_t*>(codes), reinterpret_cast<bf16*>(scales));
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int moe_layer_forward_w4a16_ws(const uint16_t* x, const uint16_t* w_router, const float* bias,
@@ -1159,7 +1438,7 @@ int moe_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t
     fp8_quantize_rows_kernel<<<blocks, 32 * kRowQuantWarps, 0, static_cast<cudaStream_t>(stream)>>>(
         reinterpret_cast<const bf16*>(w), cols, nullptr, 0, rows, rows, static_cast<int>(cols), q,
         exps);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 size_t moe_workspace_size_w8a8(int T, int d, int E, int k, int inter) {
@@ -1251,7 +1530,7 @@ int moe_bias_update(const int32_t* counts, int T, int E, int k, float gamma, flo
     bias_update_kernel<<<(E + kBalanceThreads - 1) / kBalanceThreads, kBalanceThreads, 0,
                          static_cast<cudaStream_t>(stream)>>>(
         counts, static_cast<long long>(T) * k, E, gamma, bias);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d, int E,
@@ -1274,7 +1553,7 @@ int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d,
     const long long n = static_cast<long long>(T) * E;
     router_scores_kernel<<<static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads),
                            kBalanceThreads, 0, st>>>(partials, splits, n, n, scores);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
@@ -1306,7 +1585,137 @@ int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S,
                            kBalanceThreads, 0, st>>>(topk_idx, n, S * k, E, cnt);
     seq_aux_finish_kernel<<<B, kBalanceThreads, 0, st>>>(part, cnt, L.nsplit, S, E, k, alpha, loss,
                                                          f, p);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
+}
+
+// ------------------------------------------------------ expert parallelism
+
+size_t moe_ep_dispatch_workspace_size(int T, int d, int E, int k) {
+    if (check_dims(T, d, E, k, 64) != MOE_OK) return 0;
+    return ep_dispatch_layout(T, d, E, k).total;
+}
+
+int moe_ep_dispatch(const uint16_t* x, const uint16_t* w_router, const float* bias, int T, int d,
+                    int E, int k, float scale, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                    int32_t* slot_row, uint16_t* send_rows, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    int rc = check_dims(T, d, E, k, 64);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(x, w_router, bias, topk_idx, topk_w, counts, slot_row, send_rows, workspace) ||
+        !(scale == scale))
+        return MOE_ERR_INVALID_ARG;
+    const EpDispatchLayout L = ep_dispatch_layout(T, d, E, k);
+    if (workspace_bytes < L.total) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    int* row_token = reinterpret_cast<int*>(base + L.row_token);
+    Recorder rec;
+    rc = launch_route(di, reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(w_router),
+                      bias, T, d, E, k, scale, topk_idx, topk_w,
+                      reinterpret_cast<float*>(base + L.partials), L.splits, st, rec);
+    if (rc != MOE_OK) return rc;
+    PlanArgs none{};
+    rc = launch_permute(topk_idx, T, E, k, counts, reinterpret_cast<int*>(base + L.offsets),
+                        row_token, slot_row, reinterpret_cast<int*>(base + L.blk), none, st, rec);
+    if (rc != MOE_OK) return rc;
+    const int rows = T * k;
+    gather_rows_kernel<<<(rows + 7) / 8, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), row_token,
+                                                        T, rows, d,
+                                                        reinterpret_cast<bf16*>(send_rows));
+    return launch_rc(__func__);
+}
+
+size_t moe_ep_expert_ffn_workspace_size(int rows, int d, int R, int E_local, int inter) {
+    if (R < 1 || E_local < 1 || static_cast<long long>(R) * E_local > 1024) return 0;
+    if (check_dims(rows, d, E_local, 1, inter) != MOE_OK) return 0;
+    return ep_ffn_layout(rows, d, E_local, inter).total;
+}
+
+int moe_ep_expert_ffn(const uint16_t* recv_rows, const int32_t* recv_counts, int rows, int d, int R,
+                      int E_local, int inter, const uint16_t* w_gate_up, const uint16_t* w_down,
+                      uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    if (R < 1 || E_local < 1 || static_cast<long long>(R) * E_local > 1024)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    int rc = check_dims(rows, d, E_local, 1, inter);
+    if (rc != MOE_OK) return rc;
+    if (rows == 0) return MOE_OK;
+    if (!all_ok(recv_rows, recv_counts, w_gate_up, w_down, y, workspace)) return MOE_ERR_INVALID_ARG;
+    const EpFfnLayout L = ep_ffn_layout(rows, d, E_local, inter);
+    if (workspace_bytes < L.total) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    int* exp_offsets = reinterpret_cast<int*>(base + L.exp_offsets);
+    int* src_of_exp = reinterpret_cast<int*>(base + L.src_of_exp);
+    int* exp_of_src = reinterpret_cast<int*>(base + L.exp_of_src);
+    uint8_t* fb = base + L.ffn;
+    int4* tiles1 = reinterpret_cast<int4*>(fb + L.F.tiles1);
+    int4* tiles2 = reinterpret_cast<int4*>(fb + L.F.tiles2);
+    int* ntiles = reinterpret_cast<int*>(fb + L.F.ntiles);
+    bf16* y_exp = reinterpret_cast<bf16*>(fb + L.F.y);
+    ep_plan_kernel<<<1, 1024, 0, st>>>(recv_counts, R, E_local, rows, exp_offsets, src_of_exp,
+                                       exp_of_src);
+    PlanArgs plan{E_local, 0, rows, d, inter, rows, tiles1, tiles2, ntiles};
+    plan_kernel<<<1, 1024, 0, st>>>(exp_offsets, plan);
+    if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
+    Recorder rec;
+    rc = launch_ffn(di, reinterpret_cast<const bf16*>(recv_rows), src_of_exp, nullptr, rows, d,
+                    E_local, 1, inter, reinterpret_cast<const bf16*>(w_gate_up),
+                    reinterpret_cast<const bf16*>(w_down), nullptr, nullptr, false,
+                    reinterpret_cast<bf16*>(fb + L.F.xperm), reinterpret_cast<bf16*>(fb + L.F.h),
+                    y_exp, tiles1, tiles2, ntiles, L.F.max_tiles1, L.F.max_tiles2, st, rec);
+    if (rc != MOE_OK) return rc;
+    // expert-major output rows back to the received (source-major) order
+    gather_rows_kernel<<<(rows + 7) / 8, 256, 0, st>>>(y_exp, exp_of_src, rows, rows, d,
+                                                        reinterpret_cast<bf16*>(y));
+    return launch_rc(__func__);
+}
+
+size_t moe_ep_combine_workspace_size(int T, int d, int inter) {
+    if (check_dims(T, d, 1, 1, inter) != MOE_OK) return 0;
+    return ep_combine_layout(T, d, inter).total;
+}
+
+int moe_ep_combine(const uint16_t* y_back, const uint16_t* x, const uint16_t* ws_gate_up,
+                   const uint16_t* ws_down, const float* topk_w, const int32_t* slot_row, int T,
+                   int d, int k, int inter, uint16_t* out, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+    int rc = check_dims(T, d, k, k, inter);
+    if (rc != MOE_OK) return rc;
+    if (T == 0) return MOE_OK;
+    if (!all_ok(y_back, x, ws_gate_up, ws_down, topk_w, slot_row, out, workspace))
+        return MOE_ERR_INVALID_ARG;
+    const EpCombineLayout L = ep_combine_layout(T, d, inter);
+    if (workspace_bytes < L.total) return MOE_ERR_INVALID_ARG;
+    DeviceInfo di;
+    rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    int4* tiles1 = reinterpret_cast<int4*>(base + L.tiles1);
+    int4* tiles2 = reinterpret_cast<int4*>(base + L.tiles2);
+    int* ntiles = reinterpret_cast<int*>(base + L.ntiles);
+    bf16* y_sh = reinterpret_cast<bf16*>(base + L.y);
+    // the shared expert alone: a plan with no routed expert (E = 0) and the T
+    // token rows in order; its weights also stand in for the (unused) routed slot
+    PlanArgs plan{0, 1, T, d, inter, 0, tiles1, tiles2, ntiles};
+    plan_kernel<<<1, 1024, 0, st>>>(nullptr, plan);
+    if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
+    const bf16* sgu = reinterpret_cast<const bf16*>(ws_gate_up);
+    const bf16* sdn = reinterpret_cast<const bf16*>(ws_down);
+    Recorder rec;
+    rc = launch_ffn(di, reinterpret_cast<const bf16*>(x), nullptr, nullptr, T, d, 1, 0, inter, sgu,
+                    sdn, sgu, sdn, true, nullptr, reinterpret_cast<bf16*>(base + L.h), y_sh,
+                    tiles1, tiles2, ntiles, L.max_tiles1, L.max_tiles2, st, rec);
+    if (rc != MOE_OK) return rc;
+    return launch_combine(reinterpret_cast<const bf16*>(y_back), y_sh, topk_w, slot_row, T, d, k,
+                          reinterpret_cast<bf16*>(out), st, rec);
 }
 
 int moe_device_status(void* stream, int* device_status) {
@@ -1326,10 +1735,12 @@ void moe_set_wait_timeout_ns(uint64_t timeout_ns) {
 
 int moe_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
     selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_rc(__func__);
 }
 
 int moe_last_launch_count(void) { return g_last_launches.load(); }
+
+const char* moe_last_error_string(void) { return t_last_error; }
 
 int moe_profile_begin(int max_calls) {
     if (max_calls < 0) return MOE_ERR_INVALID_ARG;

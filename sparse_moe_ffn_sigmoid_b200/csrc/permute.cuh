@@ -86,7 +86,7 @@ struct PlanArgs {
     int rows_routed;       // T*k
     int4* tiles1;          // gate|up tiles
     int4* tiles2;          // down tiles
-    int* ntiles;           // [0] = gate|up count, [1] = down count
+    int* ntiles;           // [0] = gate|up count, [1] = down count, [2], [3]: routed ones
     int kstep = kBK;       // K elements per GEMM step (FP8 compute: 2 * kBK)
     int tile_n = kTileN;   // largest token tile (a multiple of 16, <= kTileN)
 };
@@ -171,10 +171,21 @@ __device__ void plan_tiles(const PlanArgs& p, const int* offsets, int* scratch) 
             s_first2[g] = first2[h];
         }
     }
+    // [0], [1]: tiles of the gate|up and down lists; [2], [3]: how many of them
+    // are routed experts' (the shared expert's tiles come last)
     if (threadIdx.x == 0) {
         p.ntiles[0] = tot1a + tot1b;
         p.ntiles[1] = tot2a + tot2b;
+        if (!p.has_shared) {
+            p.ntiles[2] = tot1a + tot1b;
+            p.ntiles[3] = tot2a + tot2b;
+        }
     }
+    for (int h = 0; h < 2; ++h)
+        if (p.has_shared && threadIdx.x + h * 1024 == p.E) {
+            p.ntiles[2] = first1[h];
+            p.ntiles[3] = first2[h];
+        }
     __syncthreads();
     const int ft1 = (p.inter + kSlabRows - 1) / kSlabRows;
     const int ft2 = (p.d + 2 * kSlabRows - 1) / (2 * kSlabRows);

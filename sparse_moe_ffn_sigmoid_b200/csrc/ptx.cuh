@@ -128,6 +128,21 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
+// Warp-level tensor-core MMA with the A operand in registers:
+// D[16 x 8] += A[16 x 16] * B[16 x 8], bf16 inputs, fp32 accumulators.
+// Fragments (g = lane / 4, c = lane % 4): a0 = A[g][2c, 2c+1], a1 = A[g+8][2c, 2c+1],
+// a2 = A[g][2c+8, 2c+9], a3 = A[g+8][2c+8, 2c+9]; b0 = B[2c, 2c+1][g],
+// b1 = B[2c+8, 2c+9][g]; d0, d1 = D[g][2c, 2c+1], d2, d3 = D[g+8][2c, 2c+1].
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

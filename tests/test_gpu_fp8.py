@@ -70,6 +70,15 @@ FP8_CASES = [
     MoEConfig("fp8_ragged", T=37, d=384, E=7, k=3, inter=128, scale=2.827),
     MoEConfig("fp8_multi_tile", T=600, d=256, E=16, k=4, inter=128, scale=2.827, bias="zipf"),
     MoEConfig("fp8_k2_dims", T=16, d=7168, E=4, k=2, inter=2048, scale=2.827),
+    # decode-sized batches (routed experts average <= 4 rows): the register-
+    # dequantizing GEMMs with 16-row token tiles
+    MoEConfig("fp8v_small", T=16, d=512, E=32, k=4, inter=128, scale=2.827),
+    # experts 0 and 1 take all 32 tokens: two full token tiles each; d = 384
+    # leaves the down tiles' second 128-row block half outside
+    MoEConfig("fp8v_zipf_two_tiles", T=32, d=384, E=32, k=4, inter=256, scale=2.827,
+              bias="zipf"),
+    MoEConfig("fp8v_ragged", T=23, d=640, E=24, k=3, inter=384, scale=2.827),
+    MoEConfig("fp8v_k2_dims", T=8, d=7168, E=16, k=8, inter=2048, scale=2.827),
 ]
 
 
@@ -118,8 +127,33 @@ def test_fp8_layer_deterministic_and_ws(moe):
     assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
 
 
+def test_fp8_decode_path_deterministic_and_ws(moe):
+    """The decode-sized path: identical bits on repeated calls and through the
+    caller-workspace form."""
+    cfg = next(c for c in FP8_CASES if c.name == "fp8v_zipf_two_tiles")
+    g = {k: v.cuda() for k, v in make_inputs(cfg, seed=33).items()}
+    qgu, egu = moe.moe_quantize_fp8(g["w_gate_up"])
+    qdn, edn = moe.moe_quantize_fp8(g["w_down"])
+    args = (g["x"], g["w_router"], g["bias"], qgu, egu, qdn, edn, g["ws_gate_up"], g["ws_down"],
+            cfg.k, cfg.scale)
+    o1 = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    o2, o3 = torch.empty_like(o1), torch.empty_like(o1)
+    moe.moe_layer_forward_fp8(*args, o1)
+    moe.moe_layer_forward_fp8(*args, o2)
+    ws = torch.empty(moe.moe_workspace_size(cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter),
+                     dtype=torch.uint8, device="cuda")
+    moe.moe_layer_forward_fp8_ws(*args, o3, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(o1.view(torch.int16), o3.view(torch.int16))
+
+
 def test_fp8_fullsize_decode(moe):
-    """K2 decode shape in the benchmark's launch configuration, sampled rows."""
+    """K2 decode shape in the benchmark's launch configuration: every token's
+    output row against the oracle evaluated with its own quantizer's weights
+    (one batch of experts on the host at a time); the GPU's stored codes and
+    exponents of every selected expert equal the oracle quantizer's."""
     cfg = CONFIGS["k2_decode"]
     T, d, E, k = cfg.T, cfg.d, cfg.E, cfg.k
     g = make_inputs(cfg, seed=0, device="cuda")
@@ -132,19 +166,21 @@ def test_fp8_fullsize_decode(moe):
     assert moe.moe_device_status() == 0
     x_h = g["x"].cpu()
     ridx, rw, gap = oracle.route(x_h, g["w_router"].cpu(), g["bias"].cpu(), k, cfg.scale)
-    sample = [t for t in (0, T // 2, T - 1) if gap[t] >= PR.TIE_EPS]
-    need = sorted(set(ridx[sample].reshape(-1).tolist()))
-    egq = [None] * E
-    edq = [None] * E
-    for e in need:
-        q, s = oracle.quantize_fp8(_u16(g["w_gate_up"][e]))
-        # the GPU's stored codes of these experts match the oracle's quantizer
-        assert np.array_equal(qgu[e].cpu().numpy(), q) and np.array_equal(egu[e].cpu().numpy(), s)
-        egq[e] = oracle.dequantize_fp8(q, s)
-        q, s = oracle.quantize_fp8(_u16(g["w_down"][e]))
-        edq[e] = oracle.dequantize_fp8(q, s)
-    ref = oracle.moe_rows(x_h, ridx, rw, egq, edq, g["ws_gate_up"].cpu(), g["ws_down"].cpu(),
-                          tokens=np.array(sample, np.int32))
+    sample, parts = PR.wide_sample(ridx, gap, E, T, k)
+
+    def load_expert(e):
+        wts = []
+        for key, q_gpu, s_gpu in (("w_gate_up", qgu, egu), ("w_down", qdn, edn)):
+            q, s = oracle.quantize_fp8(_u16(g[key][e]))
+            assert np.array_equal(q_gpu[e].cpu().numpy(), q), f"expert {e} {key} codes"
+            assert np.array_equal(s_gpu[e].cpu().numpy(), s), f"expert {e} {key} exponents"
+            wts.append(oracle.dequantize_fp8(q, s))
+        return tuple(wts)
+
+    ref = PR.oracle_rows_by_expert(
+        x_h, ridx, rw, sample, load_expert=load_expert,
+        load_shared=lambda: (PR.u16(g["ws_gate_up"]), PR.u16(g["ws_down"])),
+        row_fn=lambda xr, wts: oracle.swiglu_row(xr, *wts))
     PR.check_output(PR.bf16_np(out[torch.tensor(sample, device="cuda")]), ref)
     del g, qgu, qdn, out
     torch.cuda.empty_cache()
