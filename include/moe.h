@@ -421,6 +421,17 @@ int moe_device_status(void* stream, int* device_status);
 void moe_set_wait_timeout_ns(uint64_t timeout_ns);
 
 /*
+ * Programmatic dependent launch (default off).  With enable = 1, every kernel of
+ * a call after its first may be scheduled while the call's previous kernel is
+ * still running; it runs its set-up (barriers, tensor memory, descriptor
+ * prefetch) meanwhile and waits for that kernel before reading any result.
+ * The first kernel of every call waits for whatever the stream held before.
+ * Results are the same either way.  Applies to launches issued after the call
+ * (process-wide).
+ */
+void moe_set_pdl(int enable);
+
+/*
  * Failure-detection self-test: launches one block that waits on an mbarrier
  * nobody arrives on, bounded by `timeout_ns`.  The wait runs out, the kernel
  * records MOE_ERR_TIMEOUT and returns; the context stays usable.

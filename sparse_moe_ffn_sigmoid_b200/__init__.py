@@ -18,7 +18,7 @@ from . import build as _build
 __all__ = [
     "MoeError", "lib", "moe_status_string", "moe_last_error_string", "moe_workspace_size", "moe_route", "moe_permute",
     "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_ws",
-    "moe_device_status", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
+    "moe_device_status", "moe_set_wait_timeout_ns", "moe_set_pdl", "moe_selftest_wait_timeout",
     "moe_last_launch_count", "moe_profile_begin", "moe_profile_end", "moe_kernel_name",
     "moe_layer_forward_noalloc", "moe_quantize_fp8", "moe_layer_forward_fp8",
     "moe_layer_forward_fp8_ws", "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss",
@@ -34,7 +34,7 @@ EXPORTED_SYMBOLS = [
     "moe_status_string", "moe_last_error_string", "moe_workspace_size", "moe_route",
     "moe_permute", "moe_expert_ffn",
     "moe_combine", "moe_layer_forward", "moe_layer_forward_ws", "moe_device_status",
-    "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout", "moe_last_launch_count",
+    "moe_set_wait_timeout_ns", "moe_set_pdl", "moe_selftest_wait_timeout", "moe_last_launch_count",
     "moe_profile_begin", "moe_profile_end", "moe_kernel_name", "moe_layer_forward_noalloc",
     "moe_quantize_fp8", "moe_layer_forward_fp8", "moe_layer_forward_fp8_ws",
     "moe_bias_update", "moe_router_scores", "moe_seq_aux_loss", "moe_seq_aux_workspace_size",
@@ -73,6 +73,7 @@ def _load():
         "moe_layer_forward_ws": ([P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, SZ, P], I),
         "moe_device_status": ([P, ctypes.POINTER(I)], I),
         "moe_set_wait_timeout_ns": ([U64], None),
+        "moe_set_pdl": ([I], None),
         "moe_selftest_wait_timeout": ([U64, P], I),
         "moe_last_launch_count": ([], I),
         "moe_profile_begin": ([I], I),
@@ -456,6 +457,11 @@ def moe_device_status(stream=None) -> int:
 
 def moe_set_wait_timeout_ns(ns: int) -> None:
     _LIB.moe_set_wait_timeout_ns(int(ns))
+
+
+def moe_set_pdl(enable: bool) -> None:
+    """Programmatic dependent launch of the library's kernels on / off (default off)."""
+    _LIB.moe_set_pdl(1 if enable else 0)
 
 
 def moe_selftest_wait_timeout(ns: int, stream=None) -> None:

@@ -22,6 +22,8 @@ constexpr int kBalanceThreads = 256;
 
 __global__ void __launch_bounds__(kBalanceThreads) bias_update_kernel(
     const int* __restrict__ counts, long long total, int E, float gamma, float* __restrict__ bias) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= E) return;
     const long long scaled = static_cast<long long>(counts[e]) * E;
@@ -38,6 +40,8 @@ __global__ void __launch_bounds__(kBalanceThreads) bias_update_kernel(
 __global__ void __launch_bounds__(kBalanceThreads) router_scores_kernel(
     const float* __restrict__ partials, int splits, long long split_stride, long long n,
     float* __restrict__ scores) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= n) return;
     float acc = partials[i];
@@ -52,6 +56,8 @@ constexpr int kAuxWarps = 8;
 // a fixed-shape shuffle sum.
 __global__ void __launch_bounds__(kBalanceThreads) token_totals_kernel(
     const float* __restrict__ scores, long long T, int E, float* __restrict__ inv_tot) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const long long t = static_cast<long long>(blockIdx.x) * (kBalanceThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
@@ -72,6 +78,8 @@ constexpr int kAuxTokens = 256;            // tokens per block of the loss kerne
 __global__ void __launch_bounds__(32 * kAuxWarps) seq_aux_partial_kernel(
     const float* __restrict__ scores, const float* __restrict__ inv_tot, int S, int E,
     float* __restrict__ part) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ float sp[kAuxWarps][kAuxExperts];
     const int b = blockIdx.x, c = blockIdx.y, sblk = blockIdx.z;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -95,6 +103,8 @@ __global__ void __launch_bounds__(32 * kAuxWarps) seq_aux_partial_kernel(
 // cnt[b * E + e] += 1 for every selection of sequence b (integer atomics).
 __global__ void __launch_bounds__(kBalanceThreads) seq_aux_count_kernel(
     const int* __restrict__ topk_idx, long long n, int Sk, int E, int* __restrict__ cnt) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const long long j = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (j >= n) return;
     const int e = topk_idx[j];
@@ -110,6 +120,8 @@ __global__ void __launch_bounds__(kBalanceThreads) seq_aux_count_kernel(
 __global__ void __launch_bounds__(kBalanceThreads) seq_aux_finish_kernel(
     const float* __restrict__ part, const int* __restrict__ cnt, int nsplit, int S, int E, int k,
     float alpha, float* __restrict__ loss, float* __restrict__ f_out, float* __restrict__ p_out) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ float scratch[32];
     const int b = blockIdx.x;
     const float fscale = static_cast<float>(E) / (static_cast<float>(k) * S);

@@ -41,6 +41,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const bf16* __restrict__ y, const bf16* __restrict__ y_shared, const float* __restrict__ topk_w,
     const int* __restrict__ slot_row, int T, int d, int k, long long y_rows,
     bf16* __restrict__ out) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ int s_row[32];
     __shared__ float s_w[32];
     const int t = blockIdx.x;

@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(1024) ep_plan_kernel(const int* __restrict__ r
                                                        int* __restrict__ exp_offsets,
                                                        int* __restrict__ src_of_exp,
                                                        int* __restrict__ exp_of_src) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ int scratch[32];
     __shared__ int s_seg[1024];    // source-major start of segment (s, e), index s * El + e
     __shared__ int s_exp[1024];    // expert-major start of segment (s, e), index s * El + e

@@ -433,6 +433,10 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    // the prologue above touches only this CTA's shared memory and TMEM: it may
+    // overlap the previous kernel on the stream; its results are read below
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
 
     const int ntiles = args.tiles != nullptr ? *args.ntiles_dev : args.ntiles_host;
     const uint64_t tmo = args.timeout_ns;

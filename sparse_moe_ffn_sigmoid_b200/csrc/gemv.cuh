@@ -259,6 +259,12 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                              static_cast<long long>(cu.st) * KS + 8 * P * c
                        : nullptr;
     }
+    // E4M3: the two row sets' multipliers
+    Fp8Scale fs[2];
+    if constexpr (WF == kGemvFp8) {
+#pragma unroll
+        for (int so = 0; so < 2; ++so) fs[so] = fp8_scale(e8[so]);
+    }
     // INT4: scales of the lane's two groups (2c, 2c + 1) for its four rows
     uint32_t sc[2][4];
     if constexpr (WF == kGemvInt4) {
@@ -299,7 +305,7 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                                                 *reinterpret_cast<const __nv_bfloat162*>(&sc[j][i]));
                     } else if constexpr (WF == kGemvFp8) {
                         const uint2 c8 = pm ? make_uint2(av[i].z, av[i].w) : make_uint2(av[i].x, av[i].y);
-                        q[h] = fp8x8_to_bf16x8(c8, fp8_scale(e8[so]));
+                        q[h] = fp8x8_to_bf16x8(c8, fs[so]);
                     } else {
                         q[h] = av[i];
                     }
@@ -344,6 +350,10 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
         if (WF == kGemvInt4) ptx::prefetch_tensormap(&a.s_map);
     }
     __syncwarp();
+    // the set-up above touches only shared memory: it may overlap the previous
+    // kernel on the stream, whose results are read from here on
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
 
     const int first = a.first ? *a.first : 0;
     const int last = *a.last;

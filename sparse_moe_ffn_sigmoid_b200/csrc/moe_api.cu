@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "moe.h"
@@ -60,6 +61,39 @@ int record_cuda_failure(const char* where, const char* what) {
 int launch_rc(const char* where) {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? MOE_OK : record_cuda_failure(where, cudaGetErrorString(e));
+}
+
+// Programmatic dependent launch of the library's kernels (moe_set_pdl): each
+// kernel may be scheduled while the previous kernel on the stream finishes and
+// runs its set-up meanwhile; every kernel waits (griddep_wait) before it reads
+// what earlier kernels wrote.
+std::atomic<int> g_pdl{0};
+
+// Only a kernel whose predecessor on the stream is this library's previous
+// kernel of the same call gets the attribute: the first kernel of every call
+// waits for whatever the stream held before (other libraries' kernels, copies).
+thread_local bool t_after_own_kernel = false;
+
+struct CallScope {
+    CallScope() { t_after_own_kernel = false; }
+};
+
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+            Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (g_pdl.load() && t_after_own_kernel) ? 1 : 0;
+    // a failed launch is left in the thread's error state for launch_rc
+    (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    t_after_own_kernel = true;
 }
 
 // Kernels of one layer call, in launch order (moe_kernel_name).  gather_rows
@@ -502,7 +536,7 @@ int launch_gemm(const GemmArgs& a, int grid, cudaStream_t st) {
     const size_t smem = gemm_smem_bytes(a.stages_a, a.stages_b, a.nslab, a.n_max,
                                         FP8A ? a.stages_a8 : 0, code_slab_bytes(OPS));
     if (smem > kMaxDynSmem || (FP8A && a.stages_a8 < 2)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    moe_gemm_kernel<EPI, OPS><<<grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st>>>(a);
+    launch(moe_gemm_kernel<EPI, OPS>, grid, FP8A ? kGemmThreadsFP8 : kGemmThreads, smem, st, a);
     return launch_rc(__func__);
 }
 
@@ -548,11 +582,11 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
 #define MOE_TOPK(N)                                                                              \
     do {                                                                                         \
         if (per_block)                                                                           \
-            topk_block_kernel<N><<<T, 32 * (N), 0, st>>>(partials, splits, sstride, T, E, k,     \
-                                                         bias, scale, idx, w);                   \
+            launch(topk_block_kernel<N>, T, 32 * (N), 0, st, partials, splits, sstride, T, E, k,  \
+                   bias, scale, idx, w);                                                         \
         else                                                                                     \
-            topk_warp_kernel<N><<<(T + 7) / 8, 256, 0, st>>>(partials, splits, sstride, T, E, k, \
-                                                             bias, scale, idx, w);               \
+            launch(topk_warp_kernel<N>, (T + 7) / 8, 256, 0, st, partials, splits, sstride, T, E, \
+                   k, bias, scale, idx, w);                                                      \
     } while (0)
     if (npl <= 1) MOE_TOPK(1);
     else if (npl <= 2) MOE_TOPK(2);
@@ -570,16 +604,14 @@ int launch_route(const DeviceInfo& di, const bf16* x, const bf16* wr, const floa
 int launch_permute(const int* idx, int T, int E, int k, int* counts, int* offsets, int* row_token,
                    int* slot_row, int* blk, const PlanArgs& plan, cudaStream_t st, Recorder& rec) {
     const int nblk = (T + kPermTokens - 1) / kPermTokens;
-    permute_hist_kernel<<<nblk, kPermTokens, 4 * E * sizeof(uint32_t), st>>>(idx, T, E, k, blk);
+    launch(permute_hist_kernel, nblk, kPermTokens, 4 * E * sizeof(uint32_t), st, idx, T, E, k, blk);
     rec.mark(st);
     // block counts are staged in shared memory when they fit (prefill: 98 KB)
     const long long n = static_cast<long long>(nblk) * E;
     const int smem_counts = n * 4 <= static_cast<long long>(kScanSmem) ? static_cast<int>(n) : 0;
-    scan_plan_kernel<<<1, 1024, smem_counts * 4, st>>>(blk, nblk, E, counts, offsets, plan,
-                                                     smem_counts);
+    launch(scan_plan_kernel, 1, 1024, smem_counts * 4, st, blk, nblk, E, counts, offsets, plan, smem_counts);
     rec.mark(st);
-    permute_scatter_kernel<<<nblk, kPermTokens, 8 * E * sizeof(uint32_t), st>>>(
-        idx, T, E, k, blk, row_token, slot_row);
+    launch(permute_scatter_kernel, nblk, kPermTokens, 8 * E * sizeof(uint32_t), st, idx, T, E, k, blk, row_token, slot_row);
     rec.mark(st);
     return launch_rc(__func__);
 }
@@ -621,11 +653,9 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
     const int rows_all = rows_routed + (shared ? T : 0);
     if (rows_routed > 0) {
         if (slot_row != nullptr && T >= kTokenMajorMinT)   // token by token: x rows read once
-            scatter_rows_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, slot_row, T, k, rows_routed, d,
-                                                            xperm);
+            launch(scatter_rows_kernel, (T + 7) / 8, 256, 0, st, x, slot_row, T, k, rows_routed, d, xperm);
         else
-            gather_rows_kernel<<<(rows_routed + 7) / 8, 256, 0, st>>>(x, row_token, T, rows_routed,
-                                                                      d, xperm);
+            launch(gather_rows_kernel, (rows_routed + 7) / 8, 256, 0, st, x, row_token, T, rows_routed, d, xperm);
         rec.mark(st);
     }
     if (use_gemv) {
@@ -663,18 +693,14 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             const int grid1 = std::max(1, std::min(gu ? max_tiles1 : max_tiles2, grid_r));
             if (wf == kGemvInt4) {
                 if (gu)
-                    moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>
-                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st>>>(v);
+                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>, grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st, v);
                 else
-                    moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>
-                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st>>>(v);
+                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>, grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st, v);
             } else {
                 if (gu)
-                    moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>
-                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st>>>(v);
+                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>, grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st, v);
                 else
-                    moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>
-                        <<<grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st>>>(v);
+                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>, grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st, v);
             }
             rec.count();
             // the shared expert's tiles: bf16 weights
@@ -684,11 +710,9 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             v.last = ntiles + (gu ? 0 : 1);
             const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_r));
             if (gu)
-                moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>
-                    <<<grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st>>>(v);
+                launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st, v);
             else
-                moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>
-                    <<<grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st>>>(v);
+                launch(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st, v);
             if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
             rec.mark(st);
             if (gu) rec.skip(st);   // no activation quantization
@@ -828,12 +852,9 @@ int launch_ffn_fp8(const DeviceInfo& di, const bf16* x, const int* row_token,
     const long long rows_all = rows_routed + T;
     const unsigned qblocks = static_cast<unsigned>((rows_all + kRowQuantWarps - 1) / kRowQuantWarps);
     if (T >= kTokenMajorMinT)
-        fp8_quantize_tokens_kernel<<<(T + kRowQuantWarps - 1) / kRowQuantWarps,
-                                     32 * kRowQuantWarps, 0, st>>>(x, slot_row, T, k, rows_routed,
-                                                                   d, xq, xexp);
+        launch(fp8_quantize_tokens_kernel, (T + kRowQuantWarps - 1) / kRowQuantWarps, 32 * kRowQuantWarps, 0, st, x, slot_row, T, k, rows_routed, d, xq, xexp);
     else
-        fp8_quantize_rows_kernel<<<qblocks, 32 * kRowQuantWarps, 0, st>>>(
-            x, d, row_token, rows_routed, T, rows_all, d, xq, xexp);
+        launch(fp8_quantize_rows_kernel, qblocks, 32 * kRowQuantWarps, 0, st, x, d, row_token, rows_routed, T, rows_all, d, xq, xexp);
     rec.mark(st);
     const int n_max = std::min(tile_n, (T + 15) & ~15);
     const uint8_t* xq_tok = xq + rows_routed * d;
@@ -863,8 +884,7 @@ int launch_ffn_fp8(const DeviceInfo& di, const bf16* x, const int* row_token,
     if (rc != MOE_OK) return rc;
     rec.mark(st);
 
-    fp8_quantize_rows_kernel<<<qblocks, 32 * kRowQuantWarps, 0, st>>>(
-        h, inter, nullptr, 0, rows_all, rows_all, inter, hq, hexp);
+    launch(fp8_quantize_rows_kernel, qblocks, 32 * kRowQuantWarps, 0, st, h, inter, nullptr, 0, rows_all, rows_all, inter, hq, hexp);
     rec.mark(st);
 
     GemmArgs g2;
@@ -897,8 +917,7 @@ int launch_combine(const bf16* y, const bf16* ysh, const float* w, const int* sl
     // split each row over several blocks only while the batch is small
     const int chunks = (d / 8 + kCombineThreads - 1) / kCombineThreads;
     const dim3 grid(T, std::max(1, std::min(chunks, (2048 + T - 1) / T)));
-    combine_kernel<<<grid, kCombineThreads, 0, st>>>(y, ysh, w, slot_row, T, d, k,
-                                                     static_cast<long long>(T) * k, out);
+    launch(combine_kernel, grid, kCombineThreads, 0, st, y, ysh, w, slot_row, T, d, k, static_cast<long long>(T) * k, out);
     rec.mark(st);
     return launch_rc(__func__);
 }
@@ -1172,6 +1191,7 @@ size_t moe_workspace_size(int T, int d, int E, int k, int inter) {
 int moe_route(const uint16_t* x, const uint16_t* w_router, const float* bias, int T, int d, int E,
               int k, float scale, int32_t* topk_idx, float* topk_w, void* workspace,
               size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, 64);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1192,6 +1212,7 @@ int moe_route(const uint16_t* x, const uint16_t* w_router, const float* bias, in
 int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, int32_t* offsets,
                 int32_t* row_token, int32_t* slot_row, void* workspace, size_t workspace_bytes,
                 void* stream) {
+    CallScope scope;
     int rc = check_dims(T, 64, E, k, 64);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1212,6 +1233,7 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* counts, i
 int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* offsets,
                    const uint16_t* w_gate_up, const uint16_t* w_down, int T, int d, int E, int k,
                    int inter, uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1227,7 +1249,7 @@ int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* o
     int4* tiles2 = reinterpret_cast<int4*>(base + L.tiles2);
     int* ntiles = reinterpret_cast<int*>(base + L.ntiles);
     PlanArgs plan{E, 0, T, d, inter, T * k, tiles1, tiles2, ntiles};
-    plan_kernel<<<1, 1024, 0, st>>>(offsets, plan);
+    launch(plan_kernel, 1, 1024, 0, st, offsets, plan);
     if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
     Recorder rec;
     return launch_ffn(di, reinterpret_cast<const bf16*>(x), row_token, nullptr, T, d, E, k, inter,
@@ -1239,6 +1261,7 @@ int moe_expert_ffn(const uint16_t* x, const int32_t* row_token, const int32_t* o
 
 int moe_combine(const uint16_t* y, const uint16_t* y_shared, const float* topk_w,
                 const int32_t* slot_row, int T, int d, int k, uint16_t* out, void* stream) {
+    CallScope scope;
     if (T < 0 || k < 1 || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (d < 8 || d % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return MOE_OK;
@@ -1255,6 +1278,7 @@ int moe_layer_forward_ws(const uint16_t* x, const uint16_t* w_router, const floa
                          const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                          int E, int k, int inter, float scale, uint16_t* out, void* workspace,
                          size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1274,6 +1298,7 @@ int moe_layer_forward(const uint16_t* x, const uint16_t* w_router, const float* 
                       const uint16_t* w_gate_up, const uint16_t* w_down,
                       const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d, int E,
                       int k, int inter, float scale, uint16_t* out, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1293,6 +1318,7 @@ int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const
                               const uint16_t* w_gate_up, const uint16_t* w_down,
                               const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                               int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1315,14 +1341,14 @@ int moe_layer_forward_noalloc(const uint16_t* x, const uint16_t* w_router, const
 
 int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, int8_t* exps,
                      void* stream) {
+    CallScope scope;
     if (rows < 0 || cols < 0 || rows % kQuantBlock != 0 || cols % kQuantBlock != 0 ||
         rows / kQuantBlock > 0x7FFFFFFF || cols / kQuantBlock > 65535)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (rows == 0 || cols == 0) return MOE_OK;
     if (!all_ok(w, q) || exps == nullptr) return MOE_ERR_INVALID_ARG;
     const dim3 grid(static_cast<unsigned>(rows / kQuantBlock), static_cast<unsigned>(cols / kQuantBlock));
-    fp8_quantize_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const bf16*>(w), cols, q, exps);
+    launch(fp8_quantize_kernel, grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const bf16*>(w), cols, q, exps);
     return launch_rc(__func__);
 }
 
@@ -1332,6 +1358,7 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
                              const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                              int E, int k, int inter, float scale, uint16_t* out,
                              void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (d % kQuantBlock != 0 || inter % kQuantBlock != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1353,6 +1380,7 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
                           const uint8_t* wq_down, const int8_t* wq_down_exp,
                           const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                           int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (d % kQuantBlock != 0 || inter % kQuantBlock != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1371,6 +1399,7 @@ int moe_layer_forward_fp8(const uint16_t* x, const uint16_t* w_router, const flo
 
 int moe_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* codes,
                       uint16_t* scales, void* stream) {
+    CallScope scope;
     if (rows < 0 || cols < 0 || cols % kBK != 0 || cols > 0x7FFFFFFF ||
         rows * (cols / kInt4Group) > 0x7FFFFFFFll * kInt4Warps)
         return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1378,9 +1407,7 @@ int moe_quantize_int4(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* co
     if (!all_ok(w, codes, scales)) return MOE_ERR_INVALID_ARG;
     const long long groups = rows * (cols / kInt4Group);
     const unsigned blocks = static_cast<unsigned>((groups + kInt4Warps - 1) / kInt4Warps);
-    int4_quantize_kernel<<<blocks, 32 * kInt4Warps, 0, static_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const bf16*>(w), rows, static_cast<int>(cols),
-        reinterpret_cast<uint32_t*>(codes), reinterpret_cast<bf16*>(scales));
+    launch(int4_quantize_kernel, blocks, 32 * kInt4Warps, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const bf16*>(w), rows, static_cast<int>(cols), reinterpret_cast<uint32_t*>(codes), reinterpret_cast<bf16*>(scales));
     return launch_rc(__func__);
 }
 
@@ -1390,6 +1417,7 @@ int moe_layer_forward_w4a16_ws(const uint16_t* x, const uint16_t* w_router, cons
                                const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                                int E, int k, int inter, float scale, uint16_t* out,
                                void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1411,6 +1439,7 @@ int moe_layer_forward_w4a16(const uint16_t* x, const uint16_t* w_router, const f
                             const uint8_t* wq_down, const uint16_t* wq_down_scale,
                             const uint16_t* ws_gate_up, const uint16_t* ws_down, int T, int d,
                             int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1429,15 +1458,14 @@ int moe_layer_forward_w4a16(const uint16_t* x, const uint16_t* w_router, const f
 
 int moe_quantize_fp8_rows(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q,
                           int8_t* exps, void* stream) {
+    CallScope scope;
     if (rows < 0 || cols < 0 || cols % 16 != 0 || cols > 0x7FFFFFFF ||
         rows > 0x7FFFFFFFll * kRowQuantWarps)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (rows == 0 || cols == 0) return MOE_OK;
     if (!all_ok(w, q) || exps == nullptr) return MOE_ERR_INVALID_ARG;
     const unsigned blocks = static_cast<unsigned>((rows + kRowQuantWarps - 1) / kRowQuantWarps);
-    fp8_quantize_rows_kernel<<<blocks, 32 * kRowQuantWarps, 0, static_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const bf16*>(w), cols, nullptr, 0, rows, rows, static_cast<int>(cols), q,
-        exps);
+    launch(fp8_quantize_rows_kernel, blocks, 32 * kRowQuantWarps, 0, static_cast<cudaStream_t>(stream), reinterpret_cast<const bf16*>(w), cols, nullptr, 0, rows, rows, static_cast<int>(cols), q, exps);
     return launch_rc(__func__);
 }
 
@@ -1453,6 +1481,7 @@ int moe_layer_forward_w8a8_ws(const uint16_t* x, const uint16_t* w_router, const
                               const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
                               int E, int k, int inter, float scale, uint16_t* out,
                               void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (d % (2 * kBK) != 0 || inter % (2 * kBK) != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1476,6 +1505,7 @@ int moe_layer_forward_w8a8(const uint16_t* x, const uint16_t* w_router, const fl
                            const uint8_t* wsq_gate_up, const int8_t* wsq_gate_up_exp,
                            const uint8_t* wsq_down, const int8_t* wsq_down_exp, int T, int d,
                            int E, int k, int inter, float scale, uint16_t* out, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, inter);
     if (rc != MOE_OK) return rc;
     if (d % (2 * kBK) != 0 || inter % (2 * kBK) != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1523,18 +1553,18 @@ size_t moe_seq_aux_workspace_size(int B, int S, int E) {
 
 int moe_bias_update(const int32_t* counts, int T, int E, int k, float gamma, float* bias,
                     void* stream) {
+    CallScope scope;
     if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (T < 0) return MOE_ERR_INVALID_ARG;
     if (counts == nullptr || bias == nullptr || !(gamma == gamma)) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;           // no rows routed: every expert sits at the mean
-    bias_update_kernel<<<(E + kBalanceThreads - 1) / kBalanceThreads, kBalanceThreads, 0,
-                         static_cast<cudaStream_t>(stream)>>>(
-        counts, static_cast<long long>(T) * k, E, gamma, bias);
+    launch(bias_update_kernel, (E + kBalanceThreads - 1) / kBalanceThreads, kBalanceThreads, 0, static_cast<cudaStream_t>(stream), counts, static_cast<long long>(T) * k, E, gamma, bias);
     return launch_rc(__func__);
 }
 
 int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d, int E,
                       float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, 1, 64);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1551,14 +1581,14 @@ int moe_router_scores(const uint16_t* x, const uint16_t* w_router, int T, int d,
                             reinterpret_cast<const bf16*>(w_router), T, d, E, partials, splits, st);
     if (rc != MOE_OK) return rc;
     const long long n = static_cast<long long>(T) * E;
-    router_scores_kernel<<<static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads),
-                           kBalanceThreads, 0, st>>>(partials, splits, n, n, scores);
+    launch(router_scores_kernel, static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads), kBalanceThreads, 0, st, partials, splits, n, n, scores);
     return launch_rc(__func__);
 }
 
 int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S, int E, int k,
                      float alpha, float* loss, float* f, float* p, void* workspace,
                      size_t workspace_bytes, void* stream) {
+    CallScope scope;
     if (E < 1 || E > 1024 || k < 1 || k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (B < 0 || S < 1) return MOE_ERR_INVALID_ARG;
     if (B == 0) return MOE_OK;
@@ -1575,16 +1605,13 @@ int moe_seq_aux_loss(const float* scores, const int32_t* topk_idx, int B, int S,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(cnt, 0, static_cast<size_t>(B) * E * sizeof(int), st) != cudaSuccess)
         return MOE_ERR_CUDA;
-    token_totals_kernel<<<static_cast<unsigned>((T + 7) / 8), kBalanceThreads, 0, st>>>(
-        scores, T, E, inv_tot);
+    launch(token_totals_kernel, static_cast<unsigned>((T + 7) / 8), kBalanceThreads, 0, st, scores, T, E, inv_tot);
     const int nchunk = (E + kAuxExperts - 1) / kAuxExperts;
-    seq_aux_partial_kernel<<<dim3(B, nchunk, L.nsplit), 32 * kAuxWarps, 0, st>>>(scores, inv_tot,
-                                                                                S, E, part);
+    launch(seq_aux_partial_kernel, dim3(B, nchunk, L.nsplit), 32 * kAuxWarps, 0, st, scores,
+           inv_tot, S, E, part);
     const long long n = T * k;
-    seq_aux_count_kernel<<<static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads),
-                           kBalanceThreads, 0, st>>>(topk_idx, n, S * k, E, cnt);
-    seq_aux_finish_kernel<<<B, kBalanceThreads, 0, st>>>(part, cnt, L.nsplit, S, E, k, alpha, loss,
-                                                         f, p);
+    launch(seq_aux_count_kernel, static_cast<unsigned>((n + kBalanceThreads - 1) / kBalanceThreads), kBalanceThreads, 0, st, topk_idx, n, S * k, E, cnt);
+    launch(seq_aux_finish_kernel, B, kBalanceThreads, 0, st, part, cnt, L.nsplit, S, E, k, alpha, loss, f, p);
     return launch_rc(__func__);
 }
 
@@ -1599,6 +1626,7 @@ int moe_ep_dispatch(const uint16_t* x, const uint16_t* w_router, const float* bi
                     int E, int k, float scale, int32_t* topk_idx, float* topk_w, int32_t* counts,
                     int32_t* slot_row, uint16_t* send_rows, void* workspace,
                     size_t workspace_bytes, void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, E, k, 64);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1623,9 +1651,7 @@ int moe_ep_dispatch(const uint16_t* x, const uint16_t* w_router, const float* bi
                         row_token, slot_row, reinterpret_cast<int*>(base + L.blk), none, st, rec);
     if (rc != MOE_OK) return rc;
     const int rows = T * k;
-    gather_rows_kernel<<<(rows + 7) / 8, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), row_token,
-                                                        T, rows, d,
-                                                        reinterpret_cast<bf16*>(send_rows));
+    launch(gather_rows_kernel, (rows + 7) / 8, 256, 0, st, reinterpret_cast<const bf16*>(x), row_token, T, rows, d, reinterpret_cast<bf16*>(send_rows));
     return launch_rc(__func__);
 }
 
@@ -1638,6 +1664,7 @@ size_t moe_ep_expert_ffn_workspace_size(int rows, int d, int R, int E_local, int
 int moe_ep_expert_ffn(const uint16_t* recv_rows, const int32_t* recv_counts, int rows, int d, int R,
                       int E_local, int inter, const uint16_t* w_gate_up, const uint16_t* w_down,
                       uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    CallScope scope;
     if (R < 1 || E_local < 1 || static_cast<long long>(R) * E_local > 1024)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     int rc = check_dims(rows, d, E_local, 1, inter);
@@ -1659,10 +1686,9 @@ int moe_ep_expert_ffn(const uint16_t* recv_rows, const int32_t* recv_counts, int
     int4* tiles2 = reinterpret_cast<int4*>(fb + L.F.tiles2);
     int* ntiles = reinterpret_cast<int*>(fb + L.F.ntiles);
     bf16* y_exp = reinterpret_cast<bf16*>(fb + L.F.y);
-    ep_plan_kernel<<<1, 1024, 0, st>>>(recv_counts, R, E_local, rows, exp_offsets, src_of_exp,
-                                       exp_of_src);
+    launch(ep_plan_kernel, 1, 1024, 0, st, recv_counts, R, E_local, rows, exp_offsets, src_of_exp, exp_of_src);
     PlanArgs plan{E_local, 0, rows, d, inter, rows, tiles1, tiles2, ntiles};
-    plan_kernel<<<1, 1024, 0, st>>>(exp_offsets, plan);
+    launch(plan_kernel, 1, 1024, 0, st, exp_offsets, plan);
     if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
     Recorder rec;
     rc = launch_ffn(di, reinterpret_cast<const bf16*>(recv_rows), src_of_exp, nullptr, rows, d,
@@ -1672,8 +1698,7 @@ int moe_ep_expert_ffn(const uint16_t* recv_rows, const int32_t* recv_counts, int
                     y_exp, tiles1, tiles2, ntiles, L.F.max_tiles1, L.F.max_tiles2, st, rec);
     if (rc != MOE_OK) return rc;
     // expert-major output rows back to the received (source-major) order
-    gather_rows_kernel<<<(rows + 7) / 8, 256, 0, st>>>(y_exp, exp_of_src, rows, rows, d,
-                                                        reinterpret_cast<bf16*>(y));
+    launch(gather_rows_kernel, (rows + 7) / 8, 256, 0, st, y_exp, exp_of_src, rows, rows, d, reinterpret_cast<bf16*>(y));
     return launch_rc(__func__);
 }
 
@@ -1686,6 +1711,7 @@ int moe_ep_combine(const uint16_t* y_back, const uint16_t* x, const uint16_t* ws
                    const uint16_t* ws_down, const float* topk_w, const int32_t* slot_row, int T,
                    int d, int k, int inter, uint16_t* out, void* workspace, size_t workspace_bytes,
                    void* stream) {
+    CallScope scope;
     int rc = check_dims(T, d, k, k, inter);
     if (rc != MOE_OK) return rc;
     if (T == 0) return MOE_OK;
@@ -1705,7 +1731,7 @@ int moe_ep_combine(const uint16_t* y_back, const uint16_t* x, const uint16_t* ws
     // the shared expert alone: a plan with no routed expert (E = 0) and the T
     // token rows in order; its weights also stand in for the (unused) routed slot
     PlanArgs plan{0, 1, T, d, inter, 0, tiles1, tiles2, ntiles};
-    plan_kernel<<<1, 1024, 0, st>>>(nullptr, plan);
+    launch(plan_kernel, 1, 1024, 0, st, nullptr, plan);
     if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
     const bf16* sgu = reinterpret_cast<const bf16*>(ws_gate_up);
     const bf16* sdn = reinterpret_cast<const bf16*>(ws_down);
@@ -1728,6 +1754,8 @@ int moe_device_status(void* stream, int* device_status) {
     *device_status = v;
     return MOE_OK;
 }
+
+void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
 
 void moe_set_wait_timeout_ns(uint64_t timeout_ns) {
     g_timeout_ns.store(timeout_ns == 0 ? 1 : timeout_ns);

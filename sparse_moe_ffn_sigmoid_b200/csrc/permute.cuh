@@ -23,6 +23,8 @@ constexpr int kPermTokens = 128;   // tokens per block (4 warps)
 
 __global__ void __launch_bounds__(kPermTokens) permute_hist_kernel(
     const int* __restrict__ topk_idx, int T, int E, int k, int* __restrict__ blk_counts) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     extern __shared__ uint32_t mask[];   // [4][E]
     for (int i = threadIdx.x; i < 4 * E; i += blockDim.x) mask[i] = 0;
     __syncthreads();
@@ -211,6 +213,10 @@ __global__ void __launch_bounds__(1024) scan_plan_kernel(int* __restrict__ blk_c
                                                          int E, int* __restrict__ counts,
                                                          int* __restrict__ offsets, PlanArgs plan,
                                                          int smem_counts) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     extern __shared__ int sc[];
     __shared__ int scratch[32];
     __shared__ int s_total[2];
@@ -268,6 +274,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ offs
 __global__ void __launch_bounds__(kPermTokens) permute_scatter_kernel(
     const int* __restrict__ topk_idx, int T, int E, int k, const int* __restrict__ blk_base,
     int* __restrict__ row_token, int* __restrict__ slot_row) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     extern __shared__ uint32_t sm[];
     uint32_t* mask = sm;                                  // [4][E]
     int* wbase = reinterpret_cast<int*>(sm + 4 * E);      // [4][E]
@@ -307,6 +315,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const bf16* __restrict
                                                           const int* __restrict__ row_token,
                                                           int T, int rows, int d,
                                                           bf16* __restrict__ xperm) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
@@ -340,6 +350,8 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const bf16* __restric
                                                            const int* __restrict__ slot_row,
                                                            int T, int k, int rows, int d,
                                                            bf16* __restrict__ xperm) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= T) return;
@@ -373,6 +385,8 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const bf16* __restric
 __global__ void __launch_bounds__(32 * kRowQuantWarps) fp8_quantize_tokens_kernel(
     const bf16* __restrict__ x, const int* __restrict__ slot_row, int T, int k,
     long long rows_routed, int d, uint8_t* __restrict__ q, int8_t* __restrict__ sexp) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int t = blockIdx.x * kRowQuantWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (t >= T) return;

@@ -128,6 +128,18 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on its stream is still
+// running: griddep_wait() returns once that kernel has completed and its
+// memory writes are visible (at once when there is no such dependency), and
+// griddep_launch_dependents() lets the next kernel on the stream be scheduled
+// (it will wait itself before touching this kernel's results).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Warp-level tensor-core MMA with the A operand in registers:
 // D[16 x 8] += A[16 x 16] * B[16 x 8], bf16 inputs, fp32 accumulators.
 // Fragments (g = lane / 4, c = lane % 4): a0 = A[g][2c, 2c+1], a1 = A[g+8][2c, 2c+1],

@@ -41,6 +41,8 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(const bf16*
                                                                      long long cols,
                                                                      uint8_t* __restrict__ q,
                                                                      int8_t* __restrict__ sexp) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ float s_max[kQuantThreads / 32];
     const long long r0 = static_cast<long long>(blockIdx.x) * kQuantBlock;
     const long long c0 = static_cast<long long>(blockIdx.y) * kQuantBlock;
@@ -161,6 +163,8 @@ constexpr int kInt4Warps = 8;             // groups per block of the quantizer
 __global__ void __launch_bounds__(32 * kInt4Warps) int4_quantize_kernel(
     const bf16* __restrict__ w, long long rows, int cols, uint32_t* __restrict__ codes,
     bf16* __restrict__ scale) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int gpr = cols / kInt4Group;
     const long long gid = static_cast<long long>(blockIdx.x) * kInt4Warps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -225,6 +229,8 @@ __global__ void __launch_bounds__(32 * kRowQuantWarps) fp8_quantize_rows_kernel(
     const bf16* __restrict__ src, long long ld, const int* __restrict__ row_map, long long n_map,
     long long src_rows, long long rows, int cols, uint8_t* __restrict__ q,
     int8_t* __restrict__ sexp) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const long long r = static_cast<long long>(blockIdx.x) * kRowQuantWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;

@@ -109,6 +109,8 @@ __global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict_
                                                         const float* __restrict__ bias,
                                                         float scale, int* __restrict__ topk_idx,
                                                         float* __restrict__ topk_w) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -144,6 +146,8 @@ __global__ void __launch_bounds__(32 * NPL) topk_block_kernel(const float* __res
                                                               float scale,
                                                               int* __restrict__ topk_idx,
                                                               float* __restrict__ topk_w) {
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
     __shared__ float sh_s[32 * NPL], sh_b[32 * NPL];
     const int t = blockIdx.x;
     if (t >= T) return;
