@@ -235,28 +235,26 @@ __device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, const GemvCurso
 }
 
 // One step of a unit: the MMAs of its P pairs on both row sets and the unit's
-// (one or two) token n-tiles, accumulating into acc (first MMA of each pair)
-// and acc2 (second).
+// (one or two) token n-tiles, accumulating into acc.
 template <int WF>
 __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& cu,
                                           const uint8_t* codes, const uint8_t* scales,
-                                          const int (&e8)[2], float (&acc)[2][2][4],
-                                          float (&acc2)[2][2][4], int lane) {
+                                          const int (&e8)[2], float (&acc)[2][2][4], int lane) {
     constexpr int KS = gemv_step_k(WF);
     constexpr int P = KS / 32;                        // MMA pairs per step
     constexpr int PJ = P / 2;                         // pairs per 16-byte chunk of a lane
     const int g = lane >> 2, c = lane & 3;
     const Tile& t = cu.t;
-    const int K = a.K;
     const int NT = t.n > 8 ? 2 : 1;
     // token rows of this step: lane slice [st * KS + 8Pc, + 8P), zero past the tile
-    const bf16* brow[2];
+    const uint4* brow[2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
         const int j = nt * 8 + g;
         brow[nt] = (nt < NT && j < t.n)
-                       ? a.b[t.map] + static_cast<long long>(t.b_row0 + j) * K +
-                             static_cast<long long>(cu.st) * KS + 8 * P * c
+                       ? reinterpret_cast<const uint4*>(
+                             a.b[t.map] + static_cast<long long>(t.b_row0 + j) * a.K +
+                             static_cast<long long>(cu.st) * KS + 8 * P * c)
                        : nullptr;
     }
     // E4M3: the two row sets' multipliers
@@ -265,35 +263,30 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
 #pragma unroll
         for (int so = 0; so < 2; ++so) fs[so] = fp8_scale(e8[so]);
     }
-    // INT4: scales of the lane's two groups (2c, 2c + 1) for its four rows
-    uint32_t sc[2][4];
-    if constexpr (WF == kGemvInt4) {
-        const bf16* ss = reinterpret_cast<const bf16*>(scales);
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                // row i: set i / 2, lane row g (+ 8 for odd i); group 2c + j
-                const uint32_t v =
-                    __bfloat16_as_ushort(ss[(i >> 1) * 128 + (2 * c + j) * 16 + g + 8 * (i & 1)]);
-                sc[j][i] = __byte_perm(v, 0u, 0x1010);     // the scale in both halves
-            }
-    }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {                     // the lane's two chunks of each row
-        uint4 bv[2][PJ];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int pm = 0; pm < PJ; ++pm)
-                bv[nt][pm] = brow[nt] ? __ldg(reinterpret_cast<const uint4*>(brow[nt]) + j * PJ + pm)
-                                      : make_uint4(0u, 0u, 0u, 0u);
         uint4 av[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             av[i] = gemv_chunk(codes + (i >> 1) * kGemvSetBytes, g + 8 * (i & 1), 2 * c + j);
+        // INT4: the scales of group 2c + j of the lane's four rows
+        uint32_t sc[4];
+        if constexpr (WF == kGemvInt4) {
+            const bf16* ss = reinterpret_cast<const bf16*>(scales);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                // row i: set i / 2, lane row g (+ 8 for odd i)
+                const uint32_t v =
+                    __bfloat16_as_ushort(ss[(i >> 1) * 128 + (2 * c + j) * 16 + g + 8 * (i & 1)]);
+                sc[i] = __byte_perm(v, 0u, 0x1010);     // the scale in both halves
+            }
+        }
 #pragma unroll
         for (int pm = 0; pm < PJ; ++pm) {             // pair m = j * PJ + pm
+            uint4 bv[2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+                bv[nt] = brow[nt] ? __ldg(brow[nt] + j * PJ + pm) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int so = 0; so < 2; ++so) {
                 uint4 q[2];     // the pair's 8 weights of rows 2 so (lane row g) and 2 so + 1 (g + 8)
@@ -302,7 +295,7 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                     const int i = 2 * so + h;
                     if constexpr (WF == kGemvInt4) {
                         q[h] = int4x8_to_bf16x8(u4_word(av[i], pm),
-                                                *reinterpret_cast<const __nv_bfloat162*>(&sc[j][i]));
+                                                *reinterpret_cast<const __nv_bfloat162*>(&sc[i]));
                     } else if constexpr (WF == kGemvFp8) {
                         const uint2 c8 = pm ? make_uint2(av[i].z, av[i].w) : make_uint2(av[i].x, av[i].y);
                         q[h] = fp8x8_to_bf16x8(c8, fs[so]);
@@ -313,10 +306,10 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     if (nt >= NT) break;
-                    ptx::mma_16816_bf16(acc[so][nt], q[0].x, q[1].x, q[0].y, q[1].y, bv[nt][pm].x,
-                                        bv[nt][pm].y);
-                    ptx::mma_16816_bf16(acc2[so][nt], q[0].z, q[1].z, q[0].w, q[1].w, bv[nt][pm].z,
-                                        bv[nt][pm].w);
+                    ptx::mma_16816_bf16(acc[so][nt], q[0].x, q[1].x, q[0].y, q[1].y, bv[nt].x,
+                                        bv[nt].y);
+                    ptx::mma_16816_bf16(acc[so][nt], q[0].z, q[1].z, q[0].w, q[1].w, bv[nt].z,
+                                        bv[nt].w);
                 }
             }
         }
@@ -376,7 +369,7 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
         p_ok = gemv_advance<EPI, WF>(a, pc, nsteps, last, warp);
     }
 
-    float acc[2][2][4], acc2[2][2][4];
+    float acc[2][2][4];
     bool ok = true;
     while (c_ok) {
         // refill the stage consumed last (every lane is past it: __syncwarp below)
@@ -395,7 +388,7 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[so][nt][i] = acc2[so][nt][i] = 0.0f;
+                    for (int i = 0; i < 4; ++i) acc[so][nt][i] = 0.0f;
         }
         int e8[2] = {0, 0};
         if constexpr (WF == kGemvFp8) {
@@ -410,18 +403,10 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
             break;
         }
         gemv_step<WF>(a, cc, codes_ring + stage * kGemvStageBytes, scale_ring + stage * kScale, e8,
-                      acc, acc2, lane);
+                      acc, lane);
         __syncwarp();                       // every lane is done with the stage
         ++qc;
-        if (cc.st == nsteps - 1) {
-#pragma unroll
-            for (int so = 0; so < 2; ++so)
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[so][nt][i] += acc2[so][nt][i];
-            gemv_epilogue<EPI>(a, cc, acc, lane);
-        }
+        if (cc.st == nsteps - 1) gemv_epilogue<EPI>(a, cc, acc, lane);
         c_ok = gemv_advance<EPI, WF>(a, cc, nsteps, last, warp);
     }
     if (!ok && lane == 0) {
