@@ -215,6 +215,28 @@ __device__ __forceinline__ void store_block_bf16(bf16* stg, const float (&v)[kSt
     __syncwarp();
 }
 
+// store_block_bf16 for values already rounded to bf16, two per word: pk[i]
+// holds token rows 2i (low half) and 2i + 1 (high half) of feature lane.
+__device__ __forceinline__ void store_block_packed(bf16* stg, const uint32_t (&pk)[kStageRows / 2],
+                                                   int ncol, bf16* out, long long ld, int row0,
+                                                   int nrows, int fbase, int col_limit, int lane) {
+    uint16_t* s16 = reinterpret_cast<uint16_t*>(stg);
+#pragma unroll
+    for (int j = 0; j < kStageRows; ++j)
+        if (j < ncol) s16[j * 32 + lane] = static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1)));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kStageRows * 4 / 32; ++i) {
+        const int vi = lane + 32 * i;
+        const int r = vi >> 2, part = vi & 3;
+        const int f = fbase + part * 8;
+        if (r < nrows && f < col_limit)
+            *reinterpret_cast<uint4*>(out + (long long)(row0 + r) * ld + f) =
+                *reinterpret_cast<const uint4*>(stg + r * 32 + part * 8);
+    }
+    __syncwarp();
+}
+
 // Lane 0 waits (bounded) and the warp shares the outcome; after a completed
 // wait every lane observes the phase itself (one try_wait, which cannot fail
 // then: the barrier cannot complete its next phase before this warp acts), so
@@ -649,6 +671,7 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
             const int npad = pad16(t.n);
             if (!wait_bounded_warp(&acc_full[ab], aphase, abort_flag, tmo)) break;
             ptx::tc_fence_after();
+            bool released = false;      // acc_empty already arrived on for this tile
             const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 ab * args.acc_stride;
             if constexpr (EPI == kEpiStoreF32) {
@@ -682,7 +705,63 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
                     if (kSwiGLU || f0 + kSlabRows < args.col_limit)
                         ew1 = aexp[t.a_row1 + q * 32 + lane];
                 }
-                for (int s = 0; s < nout; ++s) {
+                // Single-buffered accumulator (tiles of more than 128 tokens): the
+                // SwiGLU epilogue first takes all of its warp's columns out of TMEM
+                // (h rounded to bf16, two per register), frees the accumulator for
+                // the next tile's MMAs, and only then stores.
+                if constexpr (kSwiGLU && !FP8A) {
+                    if (args.acc_bufs == 1) {
+                        constexpr int kMaxChunks = (kMaxN + kChunkStep - 1) / kChunkStep;
+                        uint32_t pk[kMaxChunks][kStageRows / 2];
+#pragma unroll
+                        for (int ci = 0; ci < kMaxChunks; ++ci) {
+                            const int c0 = kStageRows * half + ci * kChunkStep;
+                            if (c0 >= npad) continue;
+                            [[maybe_unused]] const int ex =
+                                F8C ? (c0 + lane < t.n ? bexp[c0 + lane] : 0) : 0;
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                if (c0 + 16 * hh >= npad) continue;
+                                uint32_t g[16], u[16];
+                                ptx::tmem_ld_x16(tq + c0 + 16 * hh, g);
+                                ptx::tmem_ld_x16(tq + args.n_max + c0 + 16 * hh, u);
+                                ptx::tmem_wait_ld();
+#pragma unroll
+                                for (int j = 0; j < 16; j += 2) {
+                                    float v0, v1;
+                                    if constexpr (F8C) {
+                                        const int e0 = __shfl_sync(0xffffffffu, ex, 16 * hh + j);
+                                        const int e1 = __shfl_sync(0xffffffffu, ex, 16 * hh + j + 1);
+                                        v0 = silu_fast(mul_pow2(__uint_as_float(g[j]), ew0 + e0)) *
+                                             mul_pow2(__uint_as_float(u[j]), ew1 + e0);
+                                        v1 = silu_fast(mul_pow2(__uint_as_float(g[j + 1]), ew0 + e1)) *
+                                             mul_pow2(__uint_as_float(u[j + 1]), ew1 + e1);
+                                    } else {
+                                        v0 = silu_fast(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                                        v1 = silu_fast(__uint_as_float(g[j + 1])) *
+                                             __uint_as_float(u[j + 1]);
+                                    }
+                                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+                                    pk[ci][8 * hh + j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+                                }
+                            }
+                        }
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&acc_empty[ab]);
+                        released = true;
+#pragma unroll
+                        for (int ci = 0; ci < kMaxChunks; ++ci) {
+                            const int c0 = kStageRows * half + ci * kChunkStep;
+                            if (c0 >= npad) continue;
+                            const int ncol = min(kStageRows, npad - c0);
+                            store_block_packed(stg, pk[ci], ncol, out, args.out_ld, t.out_row0 + c0,
+                                               min(ncol, t.n - c0), t.out_col0 + q * 32,
+                                               args.col_limit, lane);
+                        }
+                    }
+                }
+                for (int s = 0; s < nout && !released; ++s) {
                     const int fbase = t.out_col0 + s * kSlabRows + q * 32;
                     const uint32_t ts = tq + s * args.n_max;
                     [[maybe_unused]] const int ews = s == 0 ? ew0 : ew1;
@@ -736,9 +815,11 @@ __global__ void __launch_bounds__(ops_convert(OPS) ? kGemmThreadsFP8 : kGemmThre
                     }
                 }
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&acc_empty[ab]);
+            if (!released) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&acc_empty[ab]);
+            }
             if (++ab == static_cast<uint32_t>(args.acc_bufs)) {
                 ab = 0;
                 aphase ^= 1;
