@@ -66,6 +66,10 @@ def parse_args(argv=None):
     p.add_argument("--no-extra", action="store_true",
                    help="time the decode headline only (the default run also times k2_prefill, "
                         "k2_skew and v3 on the same weights)")
+    p.add_argument("--pdl-ab", action="store_true",
+                   help="instead of the bench line: time the layer with programmatic dependent "
+                        "launch off and on, alternating (4 rounds of 50 calls each), and print "
+                        "the medians")
     p.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                    help="override a workload field (T, d, E, k, inter), e.g. a small case of\n"
                         "the same kernels for profiling: --set E=16")
@@ -173,7 +177,8 @@ def source_digest(paths):
 
 KERNEL_SOURCES = ["sparse_moe_ffn_sigmoid_b200/csrc/gemm.cuh", "sparse_moe_ffn_sigmoid_b200/csrc/ptx.cuh",
                   "sparse_moe_ffn_sigmoid_b200/csrc/common.cuh",
-                  "sparse_moe_ffn_sigmoid_b200/csrc/quant.cuh"]
+                  "sparse_moe_ffn_sigmoid_b200/csrc/quant.cuh",
+                  "sparse_moe_ffn_sigmoid_b200/csrc/gemv.cuh"]
 
 
 def profiled_traffic(workload: str, kernel: str):
@@ -528,6 +533,10 @@ def main(argv=None):
     if moe.moe_device_status() != 0:
         raise SystemExit("device status not clean after warm-up")
     launches_per_step = moe.moe_last_launch_count()
+    if args.pdl_ab:
+        if world > 1:
+            raise SystemExit("--pdl-ab runs on one GPU")
+        return run_pdl_ab(moe, args, cfg, step, stream, dev)
 
     touched = touched_experts(moe, cfg, g, dev)
 
@@ -672,6 +681,45 @@ def main(argv=None):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_pdl_ab(moe, args, cfg, step, stream, dev, rounds: int = 4, calls: int = 50):
+    """Programmatic dependent launch off and on, alternating in one process: per
+    round and setting, a few untimed calls, then `calls` layer calls between two
+    CUDA events (no per-kernel events in between: an event recorded between two
+    launches orders them and would hide the overlap).  One JSON line with the
+    per-round times and their medians."""
+    import statistics
+    import torch
+    res = {False: [], True: []}
+    try:
+        for _ in range(rounds):
+            for pdl in (False, True):
+                moe.moe_set_pdl(pdl)
+                for _ in range(5):
+                    step()
+                torch.cuda.synchronize(dev)
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(stream)
+                for _ in range(calls):
+                    step()
+                t1.record(stream)
+                torch.cuda.synchronize(dev)
+                res[pdl].append(t0.elapsed_time(t1) / calls)
+    finally:
+        moe.moe_set_pdl(False)
+    if moe.moe_device_status() != 0:
+        raise SystemExit("device status not clean after the A/B")
+    off, on = statistics.median(res[False]), statistics.median(res[True])
+    print(json.dumps({
+        "metric": "ms per layer call, programmatic dependent launch off / on",
+        "weights": args.weights, "config": {"workload": cfg.name, "T": cfg.T, "E": cfg.E},
+        "rounds": rounds, "calls_per_round": calls,
+        "off_ms": round(off, 4), "on_ms": round(on, 4),
+        "off_rounds": [round(v, 4) for v in res[False]],
+        "on_rounds": [round(v, 4) for v in res[True]],
+        "gain": round(1.0 - on / off, 4)}))
     return 0
 
 
