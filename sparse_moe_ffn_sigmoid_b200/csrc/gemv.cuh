@@ -22,9 +22,9 @@
 // are read from L1 by all of them; CTAs walk the tile list round-robin.
 //
 // Pipeline.  Every warp streams its own units with its own ring of
-// kGemvDepth stages in shared memory: lane 0 issues a step's TMA loads (both
+// gemv_depth() stages in shared memory: lane 0 issues a step's TMA loads (both
 // row sets, 16 rows x 128 bytes each, 128-byte swizzle; INT4 also the sets'
-// group scales) on the stage's mbarrier, kGemvDepth - 1 steps ahead of the
+// group scales) on the stage's mbarrier, gemv_depth() - 1 steps ahead of the
 // step the warp computes; the walk over (unit, step) is flat, so the loads of
 // the next unit start while the current one finishes.  Every wait is bounded.
 //
@@ -52,14 +52,21 @@ constexpr int kGemvRowBytes = 128;             // bytes of a weight row per step
 constexpr int kGemvSetBytes = 16 * kGemvRowBytes;      // one 16-row set per step
 constexpr int kGemvStageBytes = 2 * kGemvSetBytes;     // both sets (1024-byte aligned)
 constexpr int kGemvScaleBytes = 2 * 8 * 16 * 2;        // INT4: 2 sets x 8 groups x 16 rows bf16
-constexpr int kGemvDepth = 3;                  // steps in flight per warp
-constexpr int kGemvCtasPerSm = 2;
+
 
 enum GemvWeights : int {
     kGemvInt4 = 0,   // INT4 codes, a bf16 scale per group of 32 (routed experts)
     kGemvBF16 = 1,   // bf16 weights (the shared expert)
     kGemvFp8 = 2,    // E4M3 codes, a power-of-two scale per 128 x 128 block (routed experts)
 };
+
+// Stages per warp ring and CTAs per SM.  The routed formats run 2 CTAs per SM
+// with 3 stages (the shared memory of an SM holds no more).  The shared
+// expert's launch has few tiles (its token tiles x 256-row blocks), so its
+// warps are few and each streams a long K walk: 1 CTA per SM with 6 stages
+// keeps 5 steps in flight per warp instead of 2.
+__host__ __device__ constexpr int gemv_depth(int wf) { return wf == kGemvBF16 ? 6 : 3; }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int wf) { return wf == kGemvBF16 ? 1 : 2; }
 
 // K elements per step (one 128-byte row chunk) of a weight format.
 __host__ __device__ constexpr int gemv_step_k(int wf) {
@@ -70,8 +77,8 @@ __host__ __device__ constexpr int gemv_step_k(int wf) {
 // code rings, their scale rings (INT4), their stage barriers and abort flags.
 __host__ __device__ constexpr int gemv_smem_bytes(int wf) {
     return 1024 +
-           kGemvWarps * kGemvDepth * (kGemvStageBytes + (wf == kGemvInt4 ? kGemvScaleBytes : 0)) +
-           kGemvWarps * kGemvDepth * 8 + kGemvWarps * 4;
+           kGemvWarps * gemv_depth(wf) * (kGemvStageBytes + (wf == kGemvInt4 ? kGemvScaleBytes : 0)) +
+           kGemvWarps * gemv_depth(wf) * 8 + kGemvWarps * 4;
 }
 
 struct __align__(64) GemvArgs {
@@ -235,8 +242,11 @@ __device__ __forceinline__ void gemv_epilogue(const GemvArgs& a, const GemvCurso
 }
 
 // One step of a unit: the MMAs of its P pairs on both row sets and the unit's
-// (one or two) token n-tiles, accumulating into acc.
-template <int WF>
+// NT token n-tiles (NT = 1: the tile has at most 8 tokens), accumulating into
+// acc.  Lanes whose token column is past the tile read the tile's last token
+// row instead: MMA columns are independent, and the epilogue stores only the
+// tile's own columns, so no load needs a guard.
+template <int WF, int NT>
 __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& cu,
                                           const uint8_t* codes, const uint8_t* scales,
                                           const int (&e8)[2], float (&acc)[2][2][4], int lane) {
@@ -245,17 +255,14 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
     constexpr int PJ = P / 2;                         // pairs per 16-byte chunk of a lane
     const int g = lane >> 2, c = lane & 3;
     const Tile& t = cu.t;
-    const int NT = t.n > 8 ? 2 : 1;
-    // token rows of this step: lane slice [st * KS + 8Pc, + 8P), zero past the tile
-    const uint4* brow[2];
+    // token rows of this step: lane slice [st * KS + 8Pc, + 8P)
+    const uint4* brow[NT];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int j = nt * 8 + g;
-        brow[nt] = (nt < NT && j < t.n)
-                       ? reinterpret_cast<const uint4*>(
-                             a.b[t.map] + static_cast<long long>(t.b_row0 + j) * a.K +
-                             static_cast<long long>(cu.st) * KS + 8 * P * c)
-                       : nullptr;
+    for (int nt = 0; nt < NT; ++nt) {
+        const int j = min(nt * 8 + g, t.n - 1);
+        brow[nt] = reinterpret_cast<const uint4*>(a.b[t.map] +
+                                                  static_cast<long long>(t.b_row0 + j) * a.K +
+                                                  static_cast<long long>(cu.st) * KS + 8 * P * c);
     }
     // E4M3: the two row sets' multipliers
     Fp8Scale fs[2];
@@ -272,21 +279,20 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
         // INT4: the scales of group 2c + j of the lane's four rows
         uint32_t sc[4];
         if constexpr (WF == kGemvInt4) {
-            const bf16* ss = reinterpret_cast<const bf16*>(scales);
+            const uint16_t* ss = reinterpret_cast<const uint16_t*>(scales);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                // row i: set i / 2, lane row g (+ 8 for odd i)
-                const uint32_t v =
-                    __bfloat16_as_ushort(ss[(i >> 1) * 128 + (2 * c + j) * 16 + g + 8 * (i & 1)]);
-                sc[i] = __byte_perm(v, 0u, 0x1010);     // the scale in both halves
+                // row i: set i / 2, lane row g (+ 8 for odd i); the scale in
+                // both halves (v < 2^16, so v * 0x10001 = v | v << 16)
+                const uint32_t v = ss[(i >> 1) * 128 + (2 * c + j) * 16 + g + 8 * (i & 1)];
+                sc[i] = v * 0x10001u;
             }
         }
 #pragma unroll
         for (int pm = 0; pm < PJ; ++pm) {             // pair m = j * PJ + pm
-            uint4 bv[2];
+            uint4 bv[NT];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-                bv[nt] = brow[nt] ? __ldg(brow[nt] + j * PJ + pm) : make_uint4(0u, 0u, 0u, 0u);
+            for (int nt = 0; nt < NT; ++nt) bv[nt] = __ldg(brow[nt] + j * PJ + pm);
 #pragma unroll
             for (int so = 0; so < 2; ++so) {
                 uint4 q[2];     // the pair's 8 weights of rows 2 so (lane row g) and 2 so + 1 (g + 8)
@@ -304,8 +310,7 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                     }
                 }
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    if (nt >= NT) break;
+                for (int nt = 0; nt < NT; ++nt) {
                     ptx::mma_16816_bf16(acc[so][nt], q[0].x, q[1].x, q[0].y, q[1].y, bv[nt].x,
                                         bv[nt].y);
                     ptx::mma_16816_bf16(acc[so][nt], q[0].z, q[1].z, q[0].w, q[1].w, bv[nt].z,
@@ -322,21 +327,22 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
 // writes Y.  The plan lists the shared expert's tiles after the routed ones; a
 // launch takes its kind's range.
 template <int EPI, int WF>
-__global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
+__global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(WF))
     moe_gemv_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ uint8_t gemv_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     constexpr int kScale = (WF == kGemvInt4) ? kGemvScaleBytes : 0;
-    constexpr int kRings = kGemvWarps * kGemvDepth * (kGemvStageBytes + kScale);
+    constexpr int kDepth = gemv_depth(WF);
+    constexpr int kRings = kGemvWarps * kDepth * (kGemvStageBytes + kScale);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t* codes_ring = smem + warp * kGemvDepth * kGemvStageBytes;
-    uint8_t* scale_ring = smem + kGemvWarps * kGemvDepth * kGemvStageBytes + warp * kGemvDepth * kScale;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRings) + warp * kGemvDepth;
+    uint8_t* codes_ring = smem + warp * kDepth * kGemvStageBytes;
+    uint8_t* scale_ring = smem + kGemvWarps * kDepth * kGemvStageBytes + warp * kDepth * kScale;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRings) + warp * kDepth;
     volatile int* abort_flag =
-        reinterpret_cast<volatile int*>(smem + kRings + kGemvWarps * kGemvDepth * 8) + warp;
+        reinterpret_cast<volatile int*>(smem + kRings + kGemvWarps * kDepth * 8) + warp;
     if (lane == 0) {
-        for (int s = 0; s < kGemvDepth; ++s) ptx::mbar_init(&full[s], 1);
+        for (int s = 0; s < kDepth; ++s) ptx::mbar_init(&full[s], 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&a.a_map);
@@ -360,11 +366,11 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
     cc = pc;
     bool c_ok = p_ok;
     uint32_t qp = 0, qc = 0;    // steps issued / consumed by this warp
-    // kGemvDepth - 1 steps in flight before the first is consumed
-    for (int s = 0; s < kGemvDepth - 1 && p_ok; ++s) {
+    // kDepth - 1 steps in flight before the first is consumed
+    for (int s = 0; s < kDepth - 1 && p_ok; ++s) {
         if (lane == 0)
-            gemv_issue<WF>(a, pc, codes_ring + (qp % kGemvDepth) * kGemvStageBytes,
-                           scale_ring + (qp % kGemvDepth) * kScale, &full[qp % kGemvDepth], pol);
+            gemv_issue<WF>(a, pc, codes_ring + (qp % kDepth) * kGemvStageBytes,
+                           scale_ring + (qp % kDepth) * kScale, &full[qp % kDepth], pol);
         ++qp;
         p_ok = gemv_advance<EPI, WF>(a, pc, nsteps, last, warp);
     }
@@ -376,8 +382,8 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
         if (p_ok) {
             if (lane == 0) {
                 ptx::fence_proxy_async_smem();
-                gemv_issue<WF>(a, pc, codes_ring + (qp % kGemvDepth) * kGemvStageBytes,
-                               scale_ring + (qp % kGemvDepth) * kScale, &full[qp % kGemvDepth], pol);
+                gemv_issue<WF>(a, pc, codes_ring + (qp % kDepth) * kGemvStageBytes,
+                               scale_ring + (qp % kDepth) * kScale, &full[qp % kDepth], pol);
             }
             ++qp;
             p_ok = gemv_advance<EPI, WF>(a, pc, nsteps, last, warp);
@@ -397,13 +403,17 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
             e8[0] = __ldg(a.exps + static_cast<long long>(cc.R.set0 / kQuantBlock) * kb + cc.st);
             e8[1] = __ldg(a.exps + static_cast<long long>(cc.R.set1 / kQuantBlock) * kb + cc.st);
         }
-        const uint32_t stage = qc % kGemvDepth;
-        if (!wait_lane0(&full[stage], (qc / kGemvDepth) & 1, abort_flag, tmo, lane)) {
+        const uint32_t stage = qc % kDepth;
+        if (!wait_lane0(&full[stage], (qc / kDepth) & 1, abort_flag, tmo, lane)) {
             ok = false;
             break;
         }
-        gemv_step<WF>(a, cc, codes_ring + stage * kGemvStageBytes, scale_ring + stage * kScale, e8,
-                      acc, lane);
+        if (cc.t.n > 8)
+            gemv_step<WF, 2>(a, cc, codes_ring + stage * kGemvStageBytes,
+                             scale_ring + stage * kScale, e8, acc, lane);
+        else
+            gemv_step<WF, 1>(a, cc, codes_ring + stage * kGemvStageBytes,
+                             scale_ring + stage * kScale, e8, acc, lane);
         __syncwarp();                       // every lane is done with the stage
         ++qc;
         if (cc.st == nsteps - 1) gemv_epilogue<EPI>(a, cc, acc, lane);
@@ -412,7 +422,7 @@ __global__ void __launch_bounds__(kGemvThreads, kGemvCtasPerSm)
     if (!ok && lane == 0) {
         // the loads this warp started land before the CTA exits
         for (uint32_t q = qc; q < qp; ++q)
-            wait_bounded(&full[q % kGemvDepth], (q / kGemvDepth) & 1, nullptr, tmo);
+            wait_bounded(&full[q % kDepth], (q / kDepth) & 1, nullptr, tmo);
     }
 }
 

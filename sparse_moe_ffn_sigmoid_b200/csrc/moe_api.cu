@@ -665,7 +665,8 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
         const int shared_tiles1 = ((T + kGemvTileN - 1) / kGemvTileN) * (inter / kSlabRows);
         const int shared_tiles2 = ((T + kGemvTileN - 1) / kGemvTileN) * (d / (2 * kSlabRows));
         const int wf = i4 ? kGemvInt4 : kGemvFp8;
-        const int grid_r = kGemvCtasPerSm * di.sms;
+        const int grid_r = gemv_ctas_per_sm(wf) * di.sms;
+        const int grid_s = gemv_ctas_per_sm(kGemvBF16) * di.sms;
         for (int gemm = 0; gemm < 2; ++gemm) {
             const bool gu = (gemm == 0);
             const uint64_t rows = gu ? static_cast<uint64_t>(E) * 2 * inter
@@ -708,7 +709,7 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
                 return MOE_ERR_CUDA;
             v.first = ntiles + (gu ? 2 : 3);
             v.last = ntiles + (gu ? 0 : 1);
-            const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_r));
+            const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_s));
             if (gu)
                 launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st, v);
             else
