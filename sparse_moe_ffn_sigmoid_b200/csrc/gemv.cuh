@@ -22,11 +22,12 @@
 // are read from L1 by all of them; CTAs walk the tile list round-robin.
 //
 // Pipeline.  Every warp streams its own units with its own ring of
-// gemv_depth() stages in shared memory: lane 0 issues a step's TMA loads (both
-// row sets, 16 rows x 128 bytes each, 128-byte swizzle; INT4 also the sets'
-// group scales) on the stage's mbarrier, gemv_depth() - 1 steps ahead of the
-// step the warp computes; the walk over (unit, step) is flat, so the loads of
-// the next unit start while the current one finishes.  Every wait is bounded.
+// gemv_depth() stages in shared memory: lane 0 issues a step's TMA loads (one
+// box of both row sets, 32 rows x 128 bytes, 128-byte swizzle; INT4 also one
+// box of the sets' group scales) on the stage's mbarrier, gemv_depth() - 1
+// steps ahead of the step the warp computes; the walk over (unit, step) is
+// flat, so the loads of the next unit start while the current one finishes.
+// Every wait is bounded.
 //
 // K order.  A step is 128 bytes of a weight row: 256 K for INT4 (8 groups), 128
 // for E4M3 (one scale block), 64 for bf16 (the shared expert).  Lane (g, c) =
@@ -82,11 +83,15 @@ __host__ __device__ constexpr int gemv_smem_bytes(int wf) {
 }
 
 struct __align__(64) GemvArgs {
-    // weights, in boxes of 128 bytes x 16 rows, 128-byte swizzle: routed INT4 codes
-    // [code_rows, K / 2] or E4M3 codes [code_rows, K] (uint8), or the shared
-    // expert's bf16 weights [rows, K]
+    // weights: routed INT4 codes [code_rows, K / 2] or E4M3 codes [code_rows, K]
+    // (uint8), or the shared expert's bf16 weights [rows, K], as a 4-D view
+    // (x, row in half, half, expert) with 128-byte swizzle; one box is a unit's
+    // 128-byte step of 16 gate rows and the matching 16 up rows (gate|up) or of
+    // 32 consecutive rows (down)
     CUtensorMap a_map;
-    CUtensorMap s_map;          // INT4 group scales [K / 32, code_rows] bf16, boxes 16 rows x 8 groups
+    // INT4 group scales [K / 32, code_rows] bf16 as (row in half, half, expert,
+    // group): one box is the same rows' 8 groups of a step
+    CUtensorMap s_map;
     const int4* tiles;          // the plan's tile list (token tiles of <= kGemvTileN rows)
     const int* first;           // tiles [*first, *last) of the list (device; null first = 0)
     const int* last;
@@ -96,6 +101,7 @@ struct __align__(64) GemvArgs {
     long long out_ld;
     int K;                      // contraction length, a multiple of the format's step
     int col_limit;              // output features >= col_limit are not stored
+    int expert_rows;            // rows of one expert's stack: 2 * inter (gate|up) or d (down)
     unsigned long long timeout_ns;
 };
 
@@ -104,11 +110,13 @@ struct __align__(64) GemvArgs {
 struct GemvRows {
     int set0, set1;
     int f0;
+    int te, tr;     // the weight box's expert and row-in-half coordinates
     bool ok;
 };
 
 template <int EPI>
-__device__ __forceinline__ GemvRows gemv_rows(const Tile& t, int u, int col_limit) {
+__device__ __forceinline__ GemvRows gemv_rows(const Tile& t, int u, int col_limit,
+                                              int expert_rows) {
     GemvRows R;
     if constexpr (EPI == kEpiSwiGLU) {
         R.set0 = t.a_row0 + 16 * u;        // gate rows
@@ -120,6 +128,8 @@ __device__ __forceinline__ GemvRows gemv_rows(const Tile& t, int u, int col_limi
         R.set1 = R.set0 + 16;
         R.f0 = t.out_col0 + slab * 128 + (u & 3) * 32;
     }
+    R.te = R.set0 / expert_rows;
+    R.tr = R.set0 - R.te * expert_rows;
     // col_limit is a multiple of 64 and f0 of 16 (32 for down units), so a unit's
     // features are all inside or all outside
     R.ok = R.f0 < col_limit;
@@ -146,7 +156,7 @@ __device__ __forceinline__ bool gemv_seek(const GemvArgs& a, GemvCursor& cu, int
             if ((threadIdx.x & 31) == 0) record_status(kStatusInvalidArg);
             continue;
         }
-        cu.R = gemv_rows<EPI>(cu.t, warp, a.col_limit);
+        cu.R = gemv_rows<EPI>(cu.t, warp, a.col_limit, a.expert_rows);
         if (cu.R.ok) {
             cu.st = 0;
             return true;
@@ -163,8 +173,17 @@ __device__ __forceinline__ bool gemv_advance(const GemvArgs& a, GemvCursor& cu, 
     return gemv_seek<EPI, WF>(a, cu, last, warp);
 }
 
-// Lane 0: the TMA loads of one step into a stage (both row sets, and for INT4
-// their scales), completing on `bar`.
+// Waits for a stage: all lanes test its barrier at once (every lane that
+// sees the phase complete has acquired the stage's bytes), and only a stage
+// that has not landed yet takes the bounded lane-0 wait.
+__device__ __forceinline__ bool gemv_wait_stage(uint64_t* bar, uint32_t parity,
+                                                volatile int* abort_flag, uint64_t tmo, int lane) {
+    if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
+    return wait_lane0(bar, parity, abort_flag, tmo, lane);
+}
+
+// Lane 0: the TMA loads of one step into a stage, completing on `bar`: one
+// box of both row sets' codes and, for INT4, one box of their group scales.
 template <int WF>
 __device__ __forceinline__ void gemv_issue(const GemvArgs& a, const GemvCursor& cu, uint8_t* codes,
                                            uint8_t* scales, uint64_t* bar, uint64_t pol) {
@@ -172,13 +191,9 @@ __device__ __forceinline__ void gemv_issue(const GemvArgs& a, const GemvCursor& 
     // x in the map's elements: 128 bytes per step (uint8 codes) or 64 bf16
     const int x = cu.st * (WF == kGemvBF16 ? kGemvRowBytes / 2 : kGemvRowBytes);
     ptx::mbar_arrive_expect_tx(bar, bytes);
-    ptx::tma_load_2d_hint(codes, &a.a_map, bar, x, cu.R.set0, pol);
-    ptx::tma_load_2d_hint(codes + kGemvSetBytes, &a.a_map, bar, x, cu.R.set1, pol);
-    if constexpr (WF == kGemvInt4) {
-        ptx::tma_load_2d_hint(scales, &a.s_map, bar, cu.R.set0, 8 * cu.st, pol);
-        ptx::tma_load_2d_hint(scales + kGemvScaleBytes / 2, &a.s_map, bar, cu.R.set1, 8 * cu.st,
-                              pol);
-    }
+    ptx::tma_load_4d_hint(codes, &a.a_map, bar, x, cu.R.tr, 0, cu.R.te, pol);
+    if constexpr (WF == kGemvInt4)
+        ptx::tma_load_4d_hint(scales, &a.s_map, bar, cu.R.tr, 0, cu.R.te, 8 * cu.st, pol);
 }
 
 __device__ __forceinline__ uint32_t u4_word(const uint4& v, int i) {
@@ -282,9 +297,10 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
             const uint16_t* ss = reinterpret_cast<const uint16_t*>(scales);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                // row i: set i / 2, lane row g (+ 8 for odd i); the scale in
-                // both halves (v < 2^16, so v * 0x10001 = v | v << 16)
-                const uint32_t v = ss[(i >> 1) * 128 + (2 * c + j) * 16 + g + 8 * (i & 1)];
+                // row i: set i / 2, lane row g (+ 8 for odd i) of the box's
+                // [group][set][16 rows]; the scale in both halves (v < 2^16,
+                // so v * 0x10001 = v | v << 16)
+                const uint32_t v = ss[(2 * c + j) * 32 + (i >> 1) * 16 + g + 8 * (i & 1)];
                 sc[i] = v * 0x10001u;
             }
         }
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(WF))
             e8[1] = __ldg(a.exps + static_cast<long long>(cc.R.set1 / kQuantBlock) * kb + cc.st);
         }
         const uint32_t stage = qc % kDepth;
-        if (!wait_lane0(&full[stage], (qc / kDepth) & 1, abort_flag, tmo, lane)) {
+        if (!gemv_wait_stage(&full[stage], (qc / kDepth) & 1, abort_flag, tmo, lane)) {
             ok = false;
             break;
         }

@@ -457,38 +457,42 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // 16 rows with the 128-byte swizzle, as uint8 codes [rows, row_bytes] or bf16
 // [rows, cols]; INT4 group scales [cols / 32, rows] bf16 in boxes of 16 rows x
 // 8 groups (one 256-element step), unswizzled.
-bool make_map_gemv_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes) {
+// Decode GEMM maps (gemv.cuh): 4-D views (x, row in half, half, expert) of a
+// row-major stack of experts of expert_rows rows each.  half_rows > 0 (gate|up:
+// the up rows sit half_rows = inter rows after the gate rows): boxes of 16
+// rows x 2 halves, a unit's gate rows and the matching up rows in one box;
+// half_rows = 0 (down): boxes of 32 rows.
+bool make_map_gemv(CUtensorMap* m, CUtensorMapDataType type, size_t esize, const void* base,
+                   uint64_t rows, uint64_t cols, uint64_t expert_rows, uint64_t half_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {row_bytes, rows};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemvRowBytes), 16};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const uint64_t row_bytes = cols * esize;
+    const uint64_t in_half = half_rows ? half_rows : expert_rows;
+    const cuuint64_t dims[4] = {cols, in_half, half_rows ? 2u : 1u, rows / expert_rows};
+    const cuuint64_t strides[3] = {row_bytes, in_half * row_bytes, expert_rows * row_bytes};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(kGemvRowBytes / esize), half_rows ? 16u : 32u,
+                               half_rows ? 2u : 1u, 1u};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, type, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_map_gemv_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+// INT4 group scales [cols / 32, rows] bf16 as (row in half, half, expert,
+// group): boxes of the same rows as make_map_gemv's x the 8 groups of a step,
+// laid out [group][half][rows] in shared memory.
+bool make_map_gemv_scales(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                          uint64_t expert_rows, uint64_t half_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * sizeof(bf16)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemvRowBytes / sizeof(bf16)), 16};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_map_gemv_scales(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {rows, cols / kInt4Group};
-    const cuuint64_t strides[1] = {rows * sizeof(bf16)};
-    const cuuint32_t box[2] = {16, static_cast<cuuint32_t>(gemv_step_k(kGemvInt4) / kInt4Group)};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+    const uint64_t in_half = half_rows ? half_rows : expert_rows;
+    const cuuint64_t dims[4] = {in_half, half_rows ? 2u : 1u, rows / expert_rows, cols / kInt4Group};
+    const cuuint64_t strides[3] = {in_half * sizeof(bf16), expert_rows * sizeof(bf16),
+                                   rows * sizeof(bf16)};
+    const cuuint32_t box[4] = {half_rows ? 16u : 32u, half_rows ? 2u : 1u, 1u,
+                               static_cast<cuuint32_t>(gemv_step_k(kGemvInt4) / kInt4Group)};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -685,11 +689,16 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             v.col_limit = gu ? inter : d;
             v.timeout_ns = g_timeout_ns.load();
             // routed tiles: codes (and INT4 scales)
+            const uint64_t half = gu ? static_cast<uint64_t>(inter) : 0;
+            const uint64_t erows = gu ? 2ull * inter : static_cast<uint64_t>(d);
+            v.expert_rows = static_cast<int>(erows);
             const bool maps_ok =
-                i4 ? make_map_gemv_u8(&v.a_map, gu ? i4->gate_up : i4->down, rows, K / 2) &&
+                i4 ? make_map_gemv(&v.a_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                                   gu ? i4->gate_up : i4->down, rows, K / 2, erows, half) &&
                          make_map_gemv_scales(&v.s_map, gu ? i4->gate_up_scale : i4->down_scale,
-                                              rows, K)
-                   : make_map_gemv_u8(&v.a_map, gu ? f8->gate_up : f8->down, rows, K);
+                                              rows, K, erows, half)
+                   : make_map_gemv(&v.a_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                                   gu ? f8->gate_up : f8->down, rows, K, erows, half);
             if (!maps_ok) return record_cuda_failure(__func__, "tensor map encoding failed");
             const int grid1 = std::max(1, std::min(gu ? max_tiles1 : max_tiles2, grid_r));
             if (wf == kGemvInt4) {
@@ -705,8 +714,9 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             }
             rec.count();
             // the shared expert's tiles: bf16 weights
-            if (!make_map_gemv_bf16(&v.a_map, gu ? ws_gate_up : ws_down, gu ? 2ull * inter : d, K))
-                return MOE_ERR_CUDA;
+            if (!make_map_gemv(&v.a_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sizeof(bf16),
+                               gu ? ws_gate_up : ws_down, erows, K, erows, half))
+                return record_cuda_failure(__func__, "tensor map encoding failed");
             v.first = ntiles + (gu ? 2 : 3);
             v.last = ntiles + (gu ? 0 : 1);
             const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_s));
