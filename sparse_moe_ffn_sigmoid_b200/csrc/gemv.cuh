@@ -47,7 +47,6 @@
 namespace moe {
 
 constexpr int kGemvWarps = 8;                  // one warp per unit of a tile
-constexpr int kGemvThreads = 32 * kGemvWarps;
 constexpr int kGemvTileN = 16;                 // token rows per tile: two MMA n-tiles
 constexpr int kGemvRowBytes = 128;             // bytes of a weight row per step
 constexpr int kGemvSetBytes = 16 * kGemvRowBytes;      // one 16-row set per step
@@ -61,13 +60,18 @@ enum GemvWeights : int {
     kGemvFp8 = 2,    // E4M3 codes, a power-of-two scale per 128 x 128 block (routed experts)
 };
 
-// Stages per warp ring and CTAs per SM.  The routed formats run 2 CTAs per SM
-// with 3 stages (the shared memory of an SM holds no more).  The shared
-// expert's launch has few tiles (its token tiles x 256-row blocks), so its
-// warps are few and each streams a long K walk: 1 CTA per SM with 6 stages
-// keeps 5 steps in flight per warp instead of 2.
+// Stages per warp ring; 2 CTAs per SM.  The routed formats run 3 stages (the
+// shared memory of an SM holds no more).  The shared expert's launch has few
+// tiles (its token tiles x 256-row blocks), so its warps are few and each
+// streams a long K walk: 6 stages keep 5 steps in flight per warp instead of 2.
 __host__ __device__ constexpr int gemv_depth(int wf) { return wf == kGemvBF16 ? 6 : 3; }
-__host__ __device__ constexpr int gemv_ctas_per_sm(int wf) { return wf == kGemvBF16 ? 1 : 2; }
+// CTAs per tile: the shared expert's launch splits each tile's 8 units over 2
+// CTAs of 4 warps, so that its few tiles still reach every SM (one SM's TMA
+// stream, not its compute, bounds a unit's pace there).
+__host__ __device__ constexpr int gemv_split(int wf) { return wf == kGemvBF16 ? 2 : 1; }
+__host__ __device__ constexpr int gemv_warps(int wf) { return kGemvWarps / gemv_split(wf); }
+__host__ __device__ constexpr int gemv_threads(int wf) { return 32 * gemv_warps(wf); }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int wf) { return 2; }
 
 // K elements per step (one 128-byte row chunk) of a weight format.
 __host__ __device__ constexpr int gemv_step_k(int wf) {
@@ -78,8 +82,8 @@ __host__ __device__ constexpr int gemv_step_k(int wf) {
 // code rings, their scale rings (INT4), their stage barriers and abort flags.
 __host__ __device__ constexpr int gemv_smem_bytes(int wf) {
     return 1024 +
-           kGemvWarps * gemv_depth(wf) * (kGemvStageBytes + (wf == kGemvInt4 ? kGemvScaleBytes : 0)) +
-           kGemvWarps * gemv_depth(wf) * 8 + kGemvWarps * 4;
+           gemv_warps(wf) * gemv_depth(wf) * (kGemvStageBytes + (wf == kGemvInt4 ? kGemvScaleBytes : 0)) +
+           gemv_warps(wf) * gemv_depth(wf) * 8 + gemv_warps(wf) * 4;
 }
 
 struct __align__(64) GemvArgs {
@@ -144,12 +148,13 @@ struct GemvCursor {
     GemvRows R;
 };
 
-// Moves `cu` to the first unit of this warp at tile index >= cu.i (stride
-// gridDim.x) that has work; false when there is none.  A tile that does not
-// belong to this kernel's plan is recorded and skipped (nothing is read).
+// Moves `cu` to the first unit `unit` at tile index >= cu.i (this CTA's
+// stride through the list) that has work; false when there is none.  A tile
+// that does not belong to this kernel's plan is recorded and skipped (nothing
+// is read).
 template <int EPI, int WF>
 __device__ __forceinline__ bool gemv_seek(const GemvArgs& a, GemvCursor& cu, int last, int warp) {
-    for (; cu.i < last; cu.i += gridDim.x) {
+    for (; cu.i < last; cu.i += gridDim.x / gemv_split(WF)) {
         cu.t = tile_at(a.tiles, cu.i);
         if (cu.t.n <= 0) continue;
         if (cu.t.n > kGemvTileN || cu.t.map != (WF == kGemvBF16 ? 1 : 0)) {
@@ -169,7 +174,7 @@ template <int EPI, int WF>
 __device__ __forceinline__ bool gemv_advance(const GemvArgs& a, GemvCursor& cu, int nsteps,
                                              int last, int warp) {
     if (++cu.st < nsteps) return true;
-    cu.i += gridDim.x;
+    cu.i += gridDim.x / gemv_split(WF);
     return gemv_seek<EPI, WF>(a, cu, last, warp);
 }
 
@@ -343,20 +348,24 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
 // writes Y.  The plan lists the shared expert's tiles after the routed ones; a
 // launch takes its kind's range.
 template <int EPI, int WF>
-__global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(WF))
+__global__ void __launch_bounds__(gemv_threads(WF), gemv_ctas_per_sm(WF))
     moe_gemv_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ uint8_t gemv_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemv_smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     constexpr int kScale = (WF == kGemvInt4) ? kGemvScaleBytes : 0;
     constexpr int kDepth = gemv_depth(WF);
-    constexpr int kRings = kGemvWarps * kDepth * (kGemvStageBytes + kScale);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t* codes_ring = smem + warp * kDepth * kGemvStageBytes;
-    uint8_t* scale_ring = smem + kGemvWarps * kDepth * kGemvStageBytes + warp * kDepth * kScale;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRings) + warp * kDepth;
+    constexpr int kWarps = gemv_warps(WF);
+    constexpr int kSplit = gemv_split(WF);
+    constexpr int kRings = kWarps * kDepth * (kGemvStageBytes + kScale);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // this warp's unit of each tile (of kGemvWarps), and the CTA's first tile
+    const int warp = (blockIdx.x % kSplit) * kWarps + w;
+    uint8_t* codes_ring = smem + w * kDepth * kGemvStageBytes;
+    uint8_t* scale_ring = smem + kWarps * kDepth * kGemvStageBytes + w * kDepth * kScale;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRings) + w * kDepth;
     volatile int* abort_flag =
-        reinterpret_cast<volatile int*>(smem + kRings + kGemvWarps * kDepth * 8) + warp;
+        reinterpret_cast<volatile int*>(smem + kRings + kWarps * kDepth * 8) + w;
     if (lane == 0) {
         for (int s = 0; s < kDepth; ++s) ptx::mbar_init(&full[s], 1);
         *abort_flag = 0;
@@ -377,7 +386,7 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_ctas_per_sm(WF))
     const uint64_t tmo = a.timeout_ns;
 
     GemvCursor pc, cc;          // producer (loads) and consumer (MMAs) positions
-    pc.i = first + blockIdx.x;
+    pc.i = first + blockIdx.x / kSplit;
     bool p_ok = gemv_seek<EPI, WF>(a, pc, last, warp);
     cc = pc;
     bool c_ok = p_ok;

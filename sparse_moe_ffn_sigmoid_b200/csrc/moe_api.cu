@@ -670,7 +670,7 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
         const int shared_tiles2 = ((T + kGemvTileN - 1) / kGemvTileN) * (d / (2 * kSlabRows));
         const int wf = i4 ? kGemvInt4 : kGemvFp8;
         const int grid_r = gemv_ctas_per_sm(wf) * di.sms;
-        const int grid_s = gemv_ctas_per_sm(kGemvBF16) * di.sms;
+        const int grid_s = gemv_ctas_per_sm(kGemvBF16) * di.sms;   // a multiple of the split
         for (int gemm = 0; gemm < 2; ++gemm) {
             const bool gu = (gemm == 0);
             const uint64_t rows = gu ? static_cast<uint64_t>(E) * 2 * inter
@@ -703,14 +703,14 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             const int grid1 = std::max(1, std::min(gu ? max_tiles1 : max_tiles2, grid_r));
             if (wf == kGemvInt4) {
                 if (gu)
-                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>, grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st, v);
+                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>, grid1, gemv_threads(wf), gemv_smem_bytes(kGemvInt4), st, v);
                 else
-                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>, grid1, kGemvThreads, gemv_smem_bytes(kGemvInt4), st, v);
+                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvInt4>, grid1, gemv_threads(wf), gemv_smem_bytes(kGemvInt4), st, v);
             } else {
                 if (gu)
-                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>, grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st, v);
+                    launch(moe_gemv_kernel<kEpiSwiGLU, kGemvFp8>, grid1, gemv_threads(wf), gemv_smem_bytes(kGemvFp8), st, v);
                 else
-                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>, grid1, kGemvThreads, gemv_smem_bytes(kGemvFp8), st, v);
+                    launch(moe_gemv_kernel<kEpiStoreBF16, kGemvFp8>, grid1, gemv_threads(wf), gemv_smem_bytes(kGemvFp8), st, v);
             }
             rec.count();
             // the shared expert's tiles: bf16 weights
@@ -719,11 +719,12 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
                 return record_cuda_failure(__func__, "tensor map encoding failed");
             v.first = ntiles + (gu ? 2 : 3);
             v.last = ntiles + (gu ? 0 : 1);
-            const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_s));
+            const int split = gemv_split(kGemvBF16);
+            const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_s / split)) * split;
             if (gu)
-                launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st, v);
+                launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), st, v);
             else
-                launch(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, grid2, kGemvThreads, gemv_smem_bytes(kGemvBF16), st, v);
+                launch(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), st, v);
             if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
             rec.mark(st);
             if (gu) rec.skip(st);   // no activation quantization
