@@ -288,7 +288,7 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
     Fp8Scale fs[2];
     if constexpr (WF == kGemvFp8) {
 #pragma unroll
-        for (int so = 0; so < 2; ++so) fs[so] = fp8_scale(e8[so]);
+        for (int so = 0; so < 2; ++so) fs[so] = fp8_scale_m112(e8[so]);
     }
 #pragma unroll
     for (int j = 0; j < 2; ++j) {                     // the lane's two chunks of each row
@@ -325,7 +325,7 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                                                 *reinterpret_cast<const __nv_bfloat162*>(&sc[i]));
                     } else if constexpr (WF == kGemvFp8) {
                         const uint2 c8 = pm ? make_uint2(av[i].z, av[i].w) : make_uint2(av[i].x, av[i].y);
-                        q[h] = fp8x8_to_bf16x8(c8, fs[so]);
+                        q[h] = fp8x8_to_bf16x8_cvt(c8, fs[so]);
                     } else {
                         q[h] = av[i];
                     }

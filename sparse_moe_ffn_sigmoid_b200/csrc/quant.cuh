@@ -141,6 +141,46 @@ __device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 v, const Fp8Scale& sc) {
     return out;
 }
 
+// Two E4M3 codes (the bytes of v16, the low byte first) -> one bf16x2 word whose
+// values are code * 2^-112, bit for bit.  The hardware conversion to f16x2 is
+// exact (every E4M3 value, subnormals included, is a normal f16 number or zero);
+// an f16 number with exponent field E and mantissa m, moved three bits down
+// under its sign, is the bf16 number with exponent field E and mantissa m >> 3,
+// i.e. its value times 2^(15 - 127); E4M3 values leave the low seven mantissa
+// bits of the f16 number zero, so nothing is lost and nothing crosses into the
+// other lane.
+__device__ __forceinline__ uint32_t fp8x2_to_bf16x2_pow2m112(uint16_t v16) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v16));
+    return ((h & 0x7FFF7FFFu) >> 3) | (h & 0x80008000u);
+}
+
+// Multipliers for a block exponent s with the 2^-112 form above: m1 =
+// 2^(112 + min(s, 15)), m2 = 2^(s - min(s, 15)), both normal bf16 numbers for
+// s in [-238, 142]; each product is exact.
+__device__ __forceinline__ Fp8Scale fp8_scale_m112(int s) {
+    const int a = min(s, 15);
+    return Fp8Scale{bf16x2_pow2(112 + a), bf16x2_pow2(s - a)};
+}
+
+// Eight E4M3 codes (little-endian in `v`) -> eight bf16 values code * 2^s, exact
+// (sc from fp8_scale_m112).
+__device__ __forceinline__ uint4 fp8x8_to_bf16x8_cvt(uint2 v, const Fp8Scale& sc) {
+    const uint32_t w[4] = {fp8x2_to_bf16x2_pow2m112(static_cast<uint16_t>(v.x)),
+                           fp8x2_to_bf16x2_pow2m112(static_cast<uint16_t>(v.x >> 16)),
+                           fp8x2_to_bf16x2_pow2m112(static_cast<uint16_t>(v.y)),
+                           fp8x2_to_bf16x2_pow2m112(static_cast<uint16_t>(v.y >> 16))};
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        const __nv_bfloat162 y = __hmul2(__hmul2(x, sc.m1), sc.m2);
+        o[i] = *reinterpret_cast<const uint32_t*>(&y);
+    }
+    return out;
+}
+
 // ------------------------------------------------------------ INT4 storage
 // "Kimi K2.5 deep dive", CH7.2: the K2.5 routed experts' weights are 4-bit
 // integers, symmetric, one scale per group of 32 K elements of a row ("Kimi
