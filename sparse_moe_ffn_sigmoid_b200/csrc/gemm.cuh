@@ -330,8 +330,9 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 }
                 ptx::fence_proxy_async_smem();
             } else if (routed && w_ok) {
-                const Fp8Scale s0 = fp8_scale(__ldg(sc0 + ks * kBK / kQuantBlock));
-                const Fp8Scale s1 = nslab == 2 ? fp8_scale(__ldg(sc1 + ks * kBK / kQuantBlock)) : s0;
+                const Fp8Scale s0 = fp8_scale_m112(__ldg(sc0 + ks * kBK / kQuantBlock));
+                const Fp8Scale s1 =
+                    nslab == 2 ? fp8_scale_m112(__ldg(sc1 + ks * kBK / kQuantBlock)) : s0;
                 const uint8_t* src = ring8 + r8.stage * a8_bytes;
                 uint8_t* dst = ring_a + rq.stage * a_bytes;
                 // all of this thread's code loads first, then the conversions:
@@ -345,7 +346,7 @@ __device__ __forceinline__ void convert_weights(const GemmArgs& args, const uint
                 for (int j = 0; j < kUnits; ++j)
                     *reinterpret_cast<uint4*>(dst + dst_off + (j / 8) * kSlabBytes +
                                               (j % 8) * 16 * (kBK * 2)) =
-                        fp8x8_to_bf16x8(codes[j], j < 8 ? s0 : s1);
+                        fp8x8_to_bf16x8_cvt(codes[j], j < 8 ? s0 : s1);
                 ptx::fence_proxy_async_smem();
             }
             // every thread of the group reaches its barrier once per step of the group

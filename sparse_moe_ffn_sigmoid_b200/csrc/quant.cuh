@@ -90,25 +90,8 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quantize_kernel(const bf16*
     }
 }
 
-// Four E4M3 codes (the bytes of v, little-endian) -> two bf16x2 words whose
-// values are code * 2^-120, bit for bit: each code's sign moves from bit 7 to
-// bit 15 of its 16-bit lane and its seven magnitude bits eeeemmm from [6:0]
-// to [10:4].  A bf16 with exponent field 0000eeee and mantissa mmm0000 is
-// 2^(eeee-127) * 1.mmm for eeee > 0, and 2^-126 * 0.mmm (a subnormal) for
-// eeee = 0, which is the E4M3 value (2^(eeee-7) * 1.mmm, or 2^-6 * 0.mmm)
-// times 2^-120 in both cases.
-__device__ __forceinline__ void fp8x4_to_bf16x4_pow2m120(uint32_t v, uint32_t& lo, uint32_t& hi) {
-    const uint32_t mag = v & 0x7F7F7F7Fu;
-    const uint32_t sgn = v & 0x80808080u;
-    // byte_perm 0x1404: [0, byte0, 0, byte1]; 0x3424: [0, byte2, 0, byte3]
-    lo = (__byte_perm(mag, 0u, 0x1404) >> 4) | __byte_perm(sgn, 0u, 0x1404);
-    hi = (__byte_perm(mag, 0u, 0x3424) >> 4) | __byte_perm(sgn, 0u, 0x3424);
-}
-
-// Multipliers for a block exponent s: code * 2^-120 * m1 * m2 = code * 2^s,
-// with m1 = 2^(120 + min(s, 7)) and m2 = 2^(s - min(s, 7)), both normal bf16
-// numbers for s in [-124, 127]; each product is exact (a power-of-two scaling
-// of a value with at most four significant bits inside bf16's range).
+// A pair of bf16x2 multipliers m1, m2 (both lanes alike) that turn a scaled
+// E4M3 value into code * 2^s in two exact power-of-two multiplies.
 struct Fp8Scale {
     __nv_bfloat162 m1, m2;
 };
@@ -118,27 +101,6 @@ __device__ __forceinline__ __nv_bfloat162 bf16x2_pow2(int e) {
     const uint32_t b = static_cast<uint32_t>(e + 127) << 7;
     const uint32_t w = b | (b << 16);
     return *reinterpret_cast<const __nv_bfloat162*>(&w);
-}
-
-__device__ __forceinline__ Fp8Scale fp8_scale(int s) {
-    const int a = min(s, 7);
-    return Fp8Scale{bf16x2_pow2(120 + a), bf16x2_pow2(s - a)};
-}
-
-// Eight E4M3 codes (little-endian in `v`) -> eight bf16 values code * 2^s, exact.
-__device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 v, const Fp8Scale& sc) {
-    uint32_t w[4];
-    fp8x4_to_bf16x4_pow2m120(v.x, w[0], w[1]);
-    fp8x4_to_bf16x4_pow2m120(v.y, w[2], w[3]);
-    uint4 out;
-    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-        const __nv_bfloat162 y = __hmul2(__hmul2(x, sc.m1), sc.m2);
-        o[i] = *reinterpret_cast<const uint32_t*>(&y);
-    }
-    return out;
 }
 
 // Two E4M3 codes (the bytes of v16, the low byte first) -> one bf16x2 word whose
