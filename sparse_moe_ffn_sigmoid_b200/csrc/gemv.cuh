@@ -316,6 +316,25 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
             for (int nt = 0; nt < NT; ++nt) bv[nt] = __ldg(brow[nt] + j * PJ + pm);
 #pragma unroll
             for (int so = 0; so < 2; ++so) {
+                if constexpr (WF == kGemvInt4) {
+                    // each MMA's A fragment in operand order: pairs (0, 1), then
+                    // (2, 3), of the lane's rows g and g + 8
+                    const uint32_t w0 = u4_word(av[2 * so], pm), w1 = u4_word(av[2 * so + 1], pm);
+                    const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162*>(&sc[2 * so]);
+                    const __nv_bfloat162 s1 = *reinterpret_cast<const __nv_bfloat162*>(&sc[2 * so + 1]);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t a0 = int4_pair_to_bf16x2(w0, 2 * half, s0);
+                        const uint32_t a1 = int4_pair_to_bf16x2(w1, 2 * half, s1);
+                        const uint32_t a2 = int4_pair_to_bf16x2(w0, 2 * half + 1, s0);
+                        const uint32_t a3 = int4_pair_to_bf16x2(w1, 2 * half + 1, s1);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            ptx::mma_16816_bf16(acc[so][nt], a0, a1, a2, a3,
+                                                half ? bv[nt].z : bv[nt].x, half ? bv[nt].w : bv[nt].y);
+                    }
+                    continue;
+                }
                 uint4 q[2];     // the pair's 8 weights of rows 2 so (lane row g) and 2 so + 1 (g + 8)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {

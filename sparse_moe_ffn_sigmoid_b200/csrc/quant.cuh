@@ -194,6 +194,16 @@ __global__ void __launch_bounds__(32 * kInt4Warps) int4_quantize_kernel(
 // Eight packed codes (one word, layout above) -> eight bf16 weights bf16(q * s):
 // 0x4300 | n is the bf16 value 128 + n, so (128 + n) - 136 = q exactly, and one
 // bf16 multiply rounds q * s to nearest-even.
+// Pair i (elements 2i and 2i + 1 of the word's eight) of int4x8_to_bf16x8.
+__device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t wd, int i, __nv_bfloat162 s2) {
+    const uint32_t v = ((wd >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    const uint32_t off_bits = 0x43084308u;               // 136.0 in both halves
+    const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&off_bits));
+    const __nv_bfloat162 y = __hmul2(q, s2);
+    return *reinterpret_cast<const uint32_t*>(&y);
+}
+
 __device__ __forceinline__ uint4 int4x8_to_bf16x8(uint32_t wd, __nv_bfloat162 s2) {
     const uint32_t magic = 0x43004300u;
     uint32_t v[4];
