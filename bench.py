@@ -101,20 +101,76 @@ def host_cores():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """SM clock and clock-event (throttle) reasons sampled while the timed region
+    runs: NVML polled every 2 ms from a thread (so a 20-step decode run of about
+    70 ms still gets dozens of samples), else nvidia-smi's loop mode.  Reads only;
+    no setting of the GPU is changed."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    PERIOD_MS = 20          # a 20-step decode run lasts about 70 ms
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clock-event reason bits of the four names above
+    NVML_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4}
+    PERIOD_S = 0.002
+    PERIOD_MS = 20          # nvidia-smi fallback
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.samples = []       # (time, sm MHz, reasons set), NVML
+        self.smax = None
+        self._stop = threading.Event()
+        self.thread = None
+
+    def _nvml_handle(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+        except Exception:
+            return None
+        self._nvml = pynvml
+        try:
+            # the GPU this process uses, by PCI address (NVML counts GPUs physically)
+            import torch
+            pr = torch.cuda.get_device_properties(self.gpu)
+            bus = "%08X:%02X:%02X.0" % (getattr(pr, "pci_domain_id"), getattr(pr, "pci_bus_id"),
+                                        getattr(pr, "pci_device_id"))
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            pass
+        try:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        except Exception:
+            return None
+
+    def _poll_nvml(self, h):
+        nv = self._nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self._stop.is_set():
+            try:
+                t = time.time()
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = get_reasons(h) if get_reasons else 0
+                self.samples.append((t, float(sm), {n for n, b in self.NVML_BITS.items() if bits & b}))
+            except Exception:
+                return
+            time.sleep(self.PERIOD_S)
 
     def __enter__(self):
+        h = self._nvml_handle()
+        if h is not None:
+            try:
+                self.smax = float(self._nvml.nvmlDeviceGetMaxClockInfo(h, self._nvml.NVML_CLOCK_SM))
+            except Exception:
+                self.smax = None
+            self.thread = threading.Thread(target=self._poll_nvml, args=(h,), daemon=True)
+            self.thread.start()
+            time.sleep(0.05)
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
@@ -142,11 +198,18 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        else:
+            self._stop.set()
+            if self.thread is not None:
+                self.thread.join(timeout=1.0)
         return False
 
     def summary(self, t0, t1):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], self.smax, set()
+        for ts, mhz, rs in self.samples:
+            if t0 <= ts <= t1:
+                sm.append(mhz)
+                reasons |= rs
         for ts, line in self.lines:
             if not (t0 <= ts <= t1):
                 continue
@@ -158,13 +221,15 @@ class ClockSampler:
                 smax = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        src = "nvml" if self.samples else "nvidia-smi"
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0,
+                    "source": src}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": src}
 
 
 def source_digest(paths):

@@ -333,28 +333,26 @@ __device__ __forceinline__ void gemv_step(const GemvArgs& a, const GemvCursor& c
                             ptx::mma_16816_bf16(acc[so][nt], a0, a1, a2, a3,
                                                 half ? bv[nt].z : bv[nt].x, half ? bv[nt].w : bv[nt].y);
                     }
-                    continue;
-                }
-                uint4 q[2];     // the pair's 8 weights of rows 2 so (lane row g) and 2 so + 1 (g + 8)
+                } else {
+                    uint4 q[2];     // the pair's 8 weights of rows 2 so (g) and 2 so + 1 (g + 8)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int i = 2 * so + h;
-                    if constexpr (WF == kGemvInt4) {
-                        q[h] = int4x8_to_bf16x8(u4_word(av[i], pm),
-                                                *reinterpret_cast<const __nv_bfloat162*>(&sc[i]));
-                    } else if constexpr (WF == kGemvFp8) {
-                        const uint2 c8 = pm ? make_uint2(av[i].z, av[i].w) : make_uint2(av[i].x, av[i].y);
-                        q[h] = fp8x8_to_bf16x8_cvt(c8, fs[so]);
-                    } else {
-                        q[h] = av[i];
+                    for (int h = 0; h < 2; ++h) {
+                        const int i = 2 * so + h;
+                        if constexpr (WF == kGemvFp8) {
+                            const uint2 c8 =
+                                pm ? make_uint2(av[i].z, av[i].w) : make_uint2(av[i].x, av[i].y);
+                            q[h] = fp8x8_to_bf16x8_cvt(c8, fs[so]);
+                        } else {
+                            q[h] = av[i];
+                        }
                     }
-                }
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    ptx::mma_16816_bf16(acc[so][nt], q[0].x, q[1].x, q[0].y, q[1].y, bv[nt].x,
-                                        bv[nt].y);
-                    ptx::mma_16816_bf16(acc[so][nt], q[0].z, q[1].z, q[0].w, q[1].w, bv[nt].z,
-                                        bv[nt].w);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        ptx::mma_16816_bf16(acc[so][nt], q[0].x, q[1].x, q[0].y, q[1].y, bv[nt].x,
+                                            bv[nt].y);
+                        ptx::mma_16816_bf16(acc[so][nt], q[0].z, q[1].z, q[0].w, q[1].w, bv[nt].z,
+                                            bv[nt].w);
+                    }
                 }
             }
         }
