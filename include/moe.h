@@ -241,9 +241,11 @@ int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, 
  *   wq_gate_up [E, 2*inter, d] uint8, wq_gate_up_exp [E, 2*inter/128, d/128] int8
  *   wq_down    [E, d, inter]   uint8, wq_down_exp    [E, d/128, inter/128]   int8
  * Everything else (router, shared expert, activations, output) is as in
- * moe_layer_forward, bf16.  d and inter must be multiples of 128.  The
- * routed weights are dequantized in shared memory just before the tensor
- * cores read them; nothing in HBM holds a bf16 copy.  Errors as in
+ * moe_layer_forward, bf16.  d and inter must be multiples of 128.  Decode-
+ * sized batches (T*k <= 4*E) dequantize the routed weights in registers for
+ * warp-level tensor-core MMAs; larger batches dequantize them in shared memory
+ * just before the tcgen05 tensor cores read them.  Both compute with the same
+ * weights, code * 2^s exactly, and nothing in HBM holds a bf16 copy.  Errors as in
  * moe_layer_forward.  The _ws form takes a caller-owned workspace of
  * moe_workspace_size(T, d, E, k, inter) bytes, like moe_layer_forward_ws.
  */
@@ -283,8 +285,11 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
  *
  * moe_layer_forward_w4a16: the layer of moe_layer_forward with the routed
  * experts' weights as (codes, scales) from moe_quantize_int4; router, shared
- * expert, activations and output bf16 as there.  The codes are dequantized in
- * shared memory just before the tensor cores read them.  Errors as in
+ * expert, activations and output bf16 as there.  Decode-sized batches
+ * (T*k <= 4*E, d and inter multiples of 256) dequantize the codes in registers
+ * for warp-level tensor-core MMAs; other batches dequantize them in shared
+ * memory just before the tcgen05 tensor cores read them.  Both compute with
+ * the same weights bf16(q * s).  Errors as in
  * moe_layer_forward; the _ws form takes moe_workspace_size(T, d, E, k, inter)
  * bytes.
  */
