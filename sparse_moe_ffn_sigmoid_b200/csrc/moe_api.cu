@@ -639,6 +639,17 @@ struct Int4Experts {
     const bf16* down_scale;
 };
 
+// A second stream of the calling thread in the current context, with a fork
+// and a join event: the decode GEMMs run the shared expert's tiles on it beside
+// the routed tiles.  One per thread and context, so calls from several threads
+// never share events; created on first use and kept for the process.
+struct SideStream {
+    unsigned long long ctx_id;
+    cudaStream_t s;
+    cudaEvent_t fork, join;
+};
+int side_stream(SideStream** out);
+
 // gather + gate|up + down over a planned tile list.
 //   rows_b0: rows of the permuted token matrix (T*k); h_rows / y rows: rows_b0 (+ T if shared)
 //   f8 / i4: routed weights in FP8 or INT4 (then w_gate_up / w_down are unused),
@@ -671,6 +682,9 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
         const int wf = i4 ? kGemvInt4 : kGemvFp8;
         const int grid_r = gemv_ctas_per_sm(wf) * di.sms;
         const int grid_s = gemv_ctas_per_sm(kGemvBF16) * di.sms;   // a multiple of the split
+        SideStream* side = nullptr;
+        const int src = side_stream(&side);
+        if (src != MOE_OK) return src;
         for (int gemm = 0; gemm < 2; ++gemm) {
             const bool gu = (gemm == 0);
             const uint64_t rows = gu ? static_cast<uint64_t>(E) * 2 * inter
@@ -701,6 +715,13 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
                                    gu ? f8->gate_up : f8->down, rows, K, erows, half);
             if (!maps_ok) return record_cuda_failure(__func__, "tensor map encoding failed");
             const int grid1 = std::max(1, std::min(gu ? max_tiles1 : max_tiles2, grid_r));
+            // fork: the shared expert's tiles (below) run on the side stream beside
+            // the routed ones, which they neither read nor write (x or their own h
+            // rows in, their own h or Y rows out); launched after the routed grid,
+            // they take the SMs its last wave leaves idle
+            if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+                cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+                return record_cuda_failure(__func__, cudaGetErrorString(cudaGetLastError()));
             if (wf == kGemvInt4) {
                 if (gu)
                     launch(moe_gemv_kernel<kEpiSwiGLU, kGemvInt4>, grid1, gemv_threads(wf), gemv_smem_bytes(kGemvInt4), st, v);
@@ -721,11 +742,17 @@ int launch_ffn(const DeviceInfo& di, const bf16* x, const int* row_token, const 
             v.last = ntiles + (gu ? 0 : 1);
             const int split = gemv_split(kGemvBF16);
             const int grid2 = std::max(1, std::min(gu ? shared_tiles1 : shared_tiles2, grid_s / split)) * split;
+            t_after_own_kernel = false;     // first kernel on the side stream: fully ordered
             if (gu)
-                launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), st, v);
+                launch(moe_gemv_kernel<kEpiSwiGLU, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), side->s, v);
             else
-                launch(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), st, v);
+                launch(moe_gemv_kernel<kEpiStoreBF16, kGemvBF16>, grid2, gemv_threads(kGemvBF16), gemv_smem_bytes(kGemvBF16), side->s, v);
             if (launch_rc(__func__) != MOE_OK) return MOE_ERR_CUDA;
+            // join: the stream goes on once both halves of this GEMM are done
+            if (cudaEventRecord(side->join, side->s) != cudaSuccess ||
+                cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
+                return record_cuda_failure(__func__, cudaGetErrorString(cudaGetLastError()));
+            t_after_own_kernel = false;     // the next kernel follows an event wait
             rec.mark(st);
             if (gu) rec.skip(st);   // no activation quantization
         }
@@ -1096,6 +1123,26 @@ int noalloc_scratch(void** out) {
     }
     if (have_id || current_context_id(&id)) g_noalloc.push_back({id, p});
     *out = p;
+    return MOE_OK;
+}
+
+thread_local std::vector<SideStream> t_side;
+
+int side_stream(SideStream** out) {
+    unsigned long long id = 0;
+    if (!current_context_id(&id)) return record_cuda_failure(__func__, "no current CUDA context");
+    for (SideStream& e : t_side)
+        if (e.ctx_id == id) {
+            *out = &e;
+            return MOE_OK;
+        }
+    SideStream e{id, nullptr, nullptr, nullptr};
+    if (cudaStreamCreateWithFlags(&e.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&e.join, cudaEventDisableTiming) != cudaSuccess)
+        return record_cuda_failure(__func__, cudaGetErrorString(cudaGetLastError()));
+    t_side.push_back(e);
+    *out = &t_side.back();
     return MOE_OK;
 }
 
