@@ -245,7 +245,11 @@ int moe_quantize_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, 
  * sized batches (T*k <= 4*E) dequantize the routed weights in registers for
  * warp-level tensor-core MMAs; larger batches dequantize them in shared memory
  * just before the tcgen05 tensor cores read them.  Both compute with the same
- * weights, code * 2^s exactly, and nothing in HBM holds a bf16 copy.  Errors as in
+ * weights, code * 2^s exactly, and nothing in HBM holds a bf16 copy.  Decode-
+ * sized batches run the shared expert's tiles on a second stream of the calling
+ * thread (created on first use, one per thread and CUDA context), forked from
+ * `stream` by an event and joined back into it by another before the combine:
+ * the call stays ordered on `stream` and can be captured in a CUDA graph.  Errors as in
  * moe_layer_forward.  The _ws form takes a caller-owned workspace of
  * moe_workspace_size(T, d, E, k, inter) bytes, like moe_layer_forward_ws.
  */
@@ -289,7 +293,8 @@ int moe_layer_forward_fp8_ws(const uint16_t* x, const uint16_t* w_router, const 
  * (T*k <= 4*E, d and inter multiples of 256) dequantize the codes in registers
  * for warp-level tensor-core MMAs; other batches dequantize them in shared
  * memory just before the tcgen05 tensor cores read them.  Both compute with
- * the same weights bf16(q * s).  Errors as in
+ * the same weights bf16(q * s).  Decode-sized batches use a second stream for
+ * the shared expert's tiles as moe_layer_forward_fp8 does.  Errors as in
  * moe_layer_forward; the _ws form takes moe_workspace_size(T, d, E, k, inter)
  * bytes.
  */
