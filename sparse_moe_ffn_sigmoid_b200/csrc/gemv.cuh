@@ -19,7 +19,10 @@
 // the matching 128 up rows, down tiles two 128-row blocks.  The 8 warps of a CTA
 // take the 8 units of one tile (two sets of 16 weight rows each: 16 gate + the
 // matching 16 up rows, or 32 consecutive down rows), so the tile's token rows
-// are read from L1 by all of them; CTAs walk the tile list round-robin.
+// are read from L1 by all of them; CTAs walk the tile list round-robin.  The
+// shared expert's bf16 tiles are a launch of their own (the plan lists them
+// after the routed ones), which the host runs on a second stream beside the
+// routed launch.
 //
 // Pipeline.  Every warp streams its own units with its own ring of
 // gemv_depth() stages in shared memory: lane 0 issues a step's TMA loads (one
@@ -53,7 +56,6 @@ constexpr int kGemvSetBytes = 16 * kGemvRowBytes;      // one 16-row set per ste
 constexpr int kGemvStageBytes = 2 * kGemvSetBytes;     // both sets (1024-byte aligned)
 constexpr int kGemvScaleBytes = 2 * 8 * 16 * 2;        // INT4: 2 sets x 8 groups x 16 rows bf16
 
-
 enum GemvWeights : int {
     kGemvInt4 = 0,   // INT4 codes, a bf16 scale per group of 32 (routed experts)
     kGemvBF16 = 1,   // bf16 weights (the shared expert)
@@ -66,12 +68,11 @@ enum GemvWeights : int {
 // streams a long K walk: 6 stages keep 5 steps in flight per warp instead of 2.
 __host__ __device__ constexpr int gemv_depth(int wf) { return wf == kGemvBF16 ? 6 : 3; }
 // CTAs per tile: the shared expert's launch splits each tile's 8 units over 2
-// CTAs of 4 warps, so that its few tiles still reach every SM (one SM's TMA
-// stream, not its compute, bounds a unit's pace there).
+// CTAs of 4 warps, so that its few tiles reach more SMs.
 __host__ __device__ constexpr int gemv_split(int wf) { return wf == kGemvBF16 ? 2 : 1; }
 __host__ __device__ constexpr int gemv_warps(int wf) { return kGemvWarps / gemv_split(wf); }
 __host__ __device__ constexpr int gemv_threads(int wf) { return 32 * gemv_warps(wf); }
-__host__ __device__ constexpr int gemv_ctas_per_sm(int wf) { return 2; }
+__host__ __device__ constexpr int gemv_ctas_per_sm(int) { return 2; }
 
 // K elements per step (one 128-byte row chunk) of a weight format.
 __host__ __device__ constexpr int gemv_step_k(int wf) {
