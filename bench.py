@@ -429,6 +429,14 @@ def time_extra_workload(moe, cfg, inp, dev, warmup, peaks, peak_src, gpu_index):
         "ideal_ms": {"tensor_burst": acc["flops"] / (burst * 1e12) * 1e3,
                      "tensor_sustained": acc["flops"] / (sust * 1e12) * 1e3,
                      "hbm": acc["weight_bytes"] / (hbm_peak * 1e9) * 1e3},
+        # the attainable bound: the slower of the weight stream and the tensor
+        # time at the burst peak, and the step's fraction of it
+        "attainable": {"ms": max(acc["weight_bytes"] / (hbm_peak * 1e9),
+                                 acc["flops"] / (burst * 1e12)) * 1e3,
+                       "bound": "hbm" if acc["weight_bytes"] / (hbm_peak * 1e9) >=
+                                acc["flops"] / (burst * 1e12) else "tensor",
+                       "frac": max(acc["weight_bytes"] / (hbm_peak * 1e9),
+                                   acc["flops"] / (burst * 1e12)) * 1e3 / ms},
         "clocks": clocks,
         # ms x median SM MHz / 1000: the step in millions of SM cycles, so that a
         # power-capped clock shows as a lower MHz at an unchanged cycle count
@@ -688,9 +696,14 @@ def main(argv=None):
                 "algorithmic_flops_per_launch": acc["gate_up_flops"],
                 "avg_launch_ms": k_ms, "peak_source": src}
         t_tc = acc["flops"] / (peak * 1e12)
+        t_tc_burst = acc["flops"] / (peaks["bf16_tflops"] * (2.0 if w8a8 else 1.0) * 1e12)
         t_hbm = acc["weight_bytes"] / (peaks["hbm_gbs"] * 1e9)
         layer_roof = {"bound": "tensor", "ideal_ms": t_tc * 1e3, "frac": t_tc / (ms_step / 1e3),
                       "hbm_ideal_ms": t_hbm * 1e3, "hbm_frac": t_hbm / (ms_step / 1e3),
+                      # the attainable bound: the slower of the weight stream and
+                      # the tensor time at the burst peak
+                      "attainable_ms": max(t_tc_burst, t_hbm) * 1e3,
+                      "attainable_frac": max(t_tc_burst, t_hbm) / (ms_step / 1e3),
                       "flops": acc["flops"], "weight_bytes": acc["weight_bytes"],
                       "touched_experts": touched}
     roof["traffic"] = profiled_traffic(
