@@ -58,3 +58,32 @@ def test_ep_layer_gloo_matches_oracle(cfg, world, splits, monkeypatch):
     g = make_inputs(cfg, seed=5)
     ref, ridx, rw, gap = oracle.moe_forward(g, cfg.k, cfg.scale)
     PR.check_output(PR.bf16_np(got), ref, skip_rows=np.nonzero(gap < PR.TIE_EPS)[0])
+
+
+class _OneRank:
+    """A comm stand-in that only reports its size (no exchange is reached)."""
+
+    def __init__(self, world):
+        self.rank, self.world = 0, world
+
+    def all_to_all(self, out, inp, out_splits, in_splits):
+        raise AssertionError("the constructor checks run before any exchange")
+
+
+def test_ep_layer_rejects_uneven_expert_split():
+    from sparse_moe_ffn_sigmoid_b200 import ep
+    cfg = MoEConfig("ep_check", T=4, d=64, E=6, k=2, inter=64, scale=2.827)
+    g = make_inputs(cfg, seed=0)
+    with pytest.raises(ValueError, match="do not split evenly"):
+        ep.ExpertParallelMoE(_OneRank(4), g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                             g["ws_gate_up"], g["ws_down"], cfg.k, cfg.scale, ops=object())
+
+
+def test_ep_layer_rejects_wrong_local_expert_count():
+    from sparse_moe_ffn_sigmoid_b200 import ep
+    cfg = MoEConfig("ep_check", T=4, d=64, E=8, k=2, inter=64, scale=2.827)
+    g = make_inputs(cfg, seed=0)
+    # rank of 2 must hold E/R = 4 experts; give it all 8
+    with pytest.raises(ValueError, match="expected E/R = 4"):
+        ep.ExpertParallelMoE(_OneRank(2), g["w_router"], g["bias"], g["w_gate_up"], g["w_down"],
+                             g["ws_gate_up"], g["ws_down"], cfg.k, cfg.scale, ops=object())
