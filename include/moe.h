@@ -435,9 +435,11 @@ void moe_set_wait_timeout_ns(uint64_t timeout_ns);
  * a call after its first may be scheduled while the call's previous kernel is
  * still running; it runs its set-up (barriers, tensor memory, descriptor
  * prefetch) meanwhile and waits for that kernel before reading any result.
- * The first kernel of every call waits for whatever the stream held before.
- * Results are the same either way.  Applies to launches issued after the call
- * (process-wide).
+ * The first kernel of every call waits for whatever the stream held before,
+ * and so does every kernel that follows an event wait (the decode GEMMs' second
+ * stream and its join).  Results are the same either way.  Applies to launches
+ * issued after the call (process-wide).  With several host threads sharing one
+ * stream it is untested and best left off.
  */
 void moe_set_pdl(int enable);
 
